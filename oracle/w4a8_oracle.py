@@ -1,0 +1,267 @@
+"""CPU oracle for the W4A8 quantized GEMM — TEST INFRASTRUCTURE ONLY.
+
+Only the tests, the smoke check and the benchmark's CPU-baseline leg may
+import this module. The product (the CUDA library and its Python binding)
+never calls it, and it shares no code with the product.
+
+It is a plain, slow, obviously-correct restatement of what the path
+computes, with numpy. Every step is the definition itself; nothing is
+blocked, fused or reordered.
+
+What the pages fix and what this file reads into them
+-----------------------------------------------------
+* W4A8: 4-bit weights against 8-bit activations, with a *progressive*
+  (two-level) weight quantization chosen so that dequantizing a weight inside
+  the GEMM is cheap ("QServe/QoQ" abstract quoted in lmdeploy issue
+  "[Feature] Support W4A8KV4 Quantization(QServe/QoQ)", Motivation).
+  The two levels used here: a per-output-channel fp16 scale s1 (level 1) and,
+  per group of 128 inputs, a uint4 zero z and an integer scale s2 in [1, 8]
+  (level 2), so that the level-2 dequantized weight W8 = (q - z) * s2 is an
+  exact int8 in [-120, 120] and the GEMM runs on int8 tensor cores.
+* Dequantization must not overflow the 8-bit lanes it is computed in
+  ("LiquidGEMM: Hardware-Efficient W4A8 GEMM Kernel ...", Method: LiquidQuant
+  dequantizes four elements with two arithmetic operations and no overflow).
+  The oracle dequantizes element by element; the bytewise form is pinned in
+  the tests.
+* Activations: 8-bit, per-token symmetric with a dynamic scale (the dynamic
+  per-token baseline that "PrefixQuant: Static Quantization Beats Dynamic
+  through Prefixed Outliers in LLMs" compares against, Key Findings).
+* Offline weight reordering ("QServe/QoQ" abstract: compute-aware weight
+  reordering; "QUICK: Quantization-aware Interleaving and Conflict-free
+  Kernel ...", abstract: offline interleaving; "Fast Matrix Multiplications
+  for Lookup Table-Quantized LLMs", abstract: offline restructuring). The
+  packed byte layout below is this library's own; the oracle writes it from
+  its definition so the CUDA packer can be checked byte for byte.
+
+Readings where the pages are silent (each is listed in the design notes):
+activation codes are rint (half to even) of A / float(sA) with an IEEE fp32
+divide, where sA = fp16(amax / 127) is the *stored* scale, clamped to
+[-127, 127]; amax == 0 gives sA = 0 and zero codes; the epilogue is
+fp16_rn(float(acc) * (float(sA) * float(s1))) in fp32; the weight quantizer's
+s1 / s2 / z selection rule is this file's `quantize_weights`.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+GROUP = 128
+TILE_N = 128
+TILE_K = 128
+TILE_CODE_BYTES = TILE_N * TILE_K // 2  # 8192
+TILE_META_BYTES = TILE_N  # 128
+TILE_BYTES = TILE_CODE_BYTES + TILE_META_BYTES  # 8320
+HEADER_BYTES = 64
+MAGIC = 0x38413457  # b"W4A8" little-endian
+LAYOUT_VERSION = 1
+
+
+# ---------------------------------------------------------------------------
+# Activation quantization (per token, symmetric int8)
+# ---------------------------------------------------------------------------
+def quantize_act(A: np.ndarray):
+    """Per-token symmetric int8 quantization of fp16 activations.
+
+    For each row m:  amax = max_k |A[m,k]|;  sA = fp16_rn(amax / 127) with an
+    fp32 divide;  A8 = clamp(rint(A / float(sA)), -127, 127) with an fp32
+    divide (rint: half to even); sA == 0 gives all-zero codes.
+    rowsum[m] = sum_k A8[m,k] (int32).
+
+    Returns (A8 int8 [M,K], sA fp16 [M], rowsum int32 [M]).
+    """
+    assert A.dtype == np.float16 and A.ndim == 2
+    Af = A.astype(np.float32)
+    amax = np.max(np.abs(Af), axis=1) if A.shape[1] else np.zeros(A.shape[0], np.float32)
+    s = amax / np.float32(127.0)
+    sA = s.astype(np.float16)
+    sf = sA.astype(np.float32)
+    A8 = np.zeros(A.shape, dtype=np.int8)
+    nz = sf != 0
+    if np.any(nz):
+        quot = Af[nz] / sf[nz][:, None]
+        A8[nz] = np.clip(np.rint(quot), -127, 127).astype(np.int8)
+    rowsum = A8.astype(np.int64).sum(axis=1).astype(np.int32)
+    return A8, sA, rowsum
+
+
+# ---------------------------------------------------------------------------
+# Progressive (two-level) weight quantization
+# ---------------------------------------------------------------------------
+def quantize_weights(W: np.ndarray, group: int = GROUP):
+    """Two-level quantization of fp32 weights W [N, K].
+
+    Level 1, per output channel n: the range of group g is
+    r_g = max(max W_g, 0) - min(min W_g, 0); s1[n] = fp16_rn(max_g r_g / 120)
+    (fp32 divide); a zero s1 is replaced by 1.  t = W / float(s1) (fp32).
+    Level 2, per (n, group): lo = min(min t, 0), hi = max(max t, 0);
+    s2 = clamp(ceil((hi - lo) / 15), 1, 8); z = clamp(rint(-lo / s2), 0, 15);
+    q = clamp(rint(t / s2) + z, 0, 15).  All divides are fp32.
+
+    Returns (q uint8 [N,K], z uint8 [N,G], s2 uint8 [N,G], s1 fp16 [N]).
+    """
+    assert W.dtype == np.float32 and W.ndim == 2
+    N, K = W.shape
+    assert K % group == 0
+    G = K // group
+    Wg = W.reshape(N, G, group)
+    r = np.maximum(Wg.max(axis=2), np.float32(0)) - np.minimum(Wg.min(axis=2), np.float32(0))
+    R = r.max(axis=1)
+    s1 = (R / np.float32(120.0)).astype(np.float16)
+    s1[s1 == 0] = np.float16(1.0)
+    t = Wg / s1.astype(np.float32)[:, None, None]
+    lo = np.minimum(t.min(axis=2), np.float32(0))
+    hi = np.maximum(t.max(axis=2), np.float32(0))
+    s2 = np.clip(np.ceil((hi - lo) / np.float32(15.0)), 1, 8).astype(np.int32)
+    s2f = s2.astype(np.float32)
+    z = np.clip(np.rint(-lo / s2f), 0, 15).astype(np.int32)
+    q = np.clip(np.rint(t / s2f[:, :, None]) + z[:, :, None], 0, 15).astype(np.uint8)
+    return q.reshape(N, K), z.astype(np.uint8), s2.astype(np.uint8), s1
+
+
+def dequant_weights(q: np.ndarray, z: np.ndarray, s2: np.ndarray, group: int = GROUP) -> np.ndarray:
+    """Level-2 dequantization: W8[n,k] = (q[n,k] - z[n,k//g]) * s2[n,k//g], exact int8."""
+    N, K = q.shape
+    zk = np.repeat(z.astype(np.int32), group, axis=1)
+    sk = np.repeat(s2.astype(np.int32), group, axis=1)
+    w8 = (q.astype(np.int32) - zk) * sk
+    return w8.astype(np.int8)
+
+
+# ---------------------------------------------------------------------------
+# Packed weight blob (offline reordering)
+# ---------------------------------------------------------------------------
+def packed_bytes(N: int, K: int, group: int = GROUP) -> int:
+    """Header + (N/128)*(K/128) tiles of 8320 bytes + s1 padded to 16 bytes."""
+    tiles = (N // TILE_N) * (K // TILE_K)
+    s1_bytes = (2 * N + 15) // 16 * 16
+    return HEADER_BYTES + tiles * TILE_BYTES + s1_bytes
+
+
+def code_byte_offset(r: int, kk: int):
+    """Byte offset inside a tile's code area of row r, in-tile k index kk,
+    and whether the code is the high nibble.
+
+    Row r's codes for k = 8j .. 8j+7 form 32-bit word j (j = 0..15): byte b
+    holds k = 8j+b in its low nibble and k = 8j+4+b in its high nibble.
+    Word j of row r sits at word index ((j // 4) * 128 + r) * 4 + j % 4, so
+    the four words j = 4c .. 4c+3 (k = 32c .. 32c+31) of a row are one
+    16-byte vector and 32 consecutive rows read 512 contiguous bytes.
+    """
+    j, within = divmod(kk, 8)
+    high = within >= 4
+    b = within - 4 if high else within
+    word = ((j // 4) * TILE_N + r) * 4 + (j % 4)
+    return word * 4 + b, high
+
+
+def pack_weights(q, z, s2, s1, group: int = GROUP) -> np.ndarray:
+    """Writes the packed blob element by element from the layout definition.
+
+    Header (64 bytes, little-endian): u32 magic 'W4A8', u32 version 1,
+    i64 N, i64 K, i32 group, u32 tile bytes (8320), u64 byte offset of s1;
+    the rest zero.  Tile (nt, kt) starts at 64 + (nt*(K/128) + kt)*8320: 8192
+    code bytes (see `code_byte_offset`), then 128 meta bytes, row r's being
+    z | ((s2 - 1) << 4) of group kt.  After the tiles: s1 as N fp16 values,
+    zero padded to a multiple of 16 bytes.
+    """
+    assert group == GROUP
+    N, K = q.shape
+    assert N % TILE_N == 0 and K % TILE_K == 0
+    KT = K // TILE_K
+    out = np.zeros(packed_bytes(N, K, group), dtype=np.uint8)
+    s1_off = HEADER_BYTES + (N // TILE_N) * KT * TILE_BYTES
+    hdr = bytearray(HEADER_BYTES)
+    hdr[0:4] = MAGIC.to_bytes(4, "little")
+    hdr[4:8] = LAYOUT_VERSION.to_bytes(4, "little")
+    hdr[8:16] = int(N).to_bytes(8, "little", signed=True)
+    hdr[16:24] = int(K).to_bytes(8, "little", signed=True)
+    hdr[24:28] = int(group).to_bytes(4, "little", signed=True)
+    hdr[28:32] = TILE_BYTES.to_bytes(4, "little")
+    hdr[32:40] = int(s1_off).to_bytes(8, "little")
+    out[:HEADER_BYTES] = np.frombuffer(bytes(hdr), dtype=np.uint8)
+    # code bytes: byte b of word j of row r in tile (nt, kt) holds
+    # k = 8j+b (low nibble) and k = 8j+4+b (high nibble)
+    n = np.arange(N)[:, None, None, None]
+    kt = np.arange(KT)[None, :, None, None]
+    j = np.arange(16)[None, None, :, None]
+    b = np.arange(4)[None, None, None, :]
+    r = n % TILE_N
+    k_lo = kt * TILE_K + 8 * j + b
+    k_hi = k_lo + 4
+    byte = (q[n, k_lo].astype(np.uint16) | (q[n, k_hi].astype(np.uint16) << 4)).astype(np.uint8)
+    word = ((j // 4) * TILE_N + r) * 4 + (j % 4)
+    dest = HEADER_BYTES + ((n // TILE_N) * KT + kt) * TILE_BYTES + word * 4 + b
+    out[dest.ravel()] = byte.ravel()
+    n = np.arange(N)[:, None]
+    # meta bytes
+    g = np.arange(K // group)[None, :]
+    meta = (z.astype(np.uint16) | ((s2.astype(np.uint16) - 1) << 4)).astype(np.uint8)
+    mdest = HEADER_BYTES + (n // TILE_N * KT + g) * TILE_BYTES + TILE_CODE_BYTES + n % TILE_N
+    out[mdest.ravel()] = meta.ravel()
+    out[s1_off:s1_off + 2 * N] = np.frombuffer(s1.astype(np.float16).tobytes(), dtype=np.uint8)
+    return out
+
+
+def unpack_weights(blob: np.ndarray):
+    """Inverse of `pack_weights`: returns (q, z, s2, s1, N, K)."""
+    hdr = bytes(blob[:HEADER_BYTES])
+    assert int.from_bytes(hdr[0:4], "little") == MAGIC
+    N = int.from_bytes(hdr[8:16], "little", signed=True)
+    K = int.from_bytes(hdr[16:24], "little", signed=True)
+    group = int.from_bytes(hdr[24:28], "little", signed=True)
+    s1_off = int.from_bytes(hdr[32:40], "little")
+    KT = K // TILE_K
+    q = np.zeros((N, K), dtype=np.uint8)
+    z = np.zeros((N, K // group), dtype=np.uint8)
+    s2 = np.zeros((N, K // group), dtype=np.uint8)
+    n = np.arange(N)[:, None]
+    k = np.arange(K)[None, :]
+    nt, r = n // TILE_N, n % TILE_N
+    kt, kk = k // TILE_K, k % TILE_K
+    j, within = kk // 8, kk % 8
+    high = within >= 4
+    b = np.where(high, within - 4, within)
+    word = ((j // 4) * TILE_N + r) * 4 + (j % 4)
+    src = HEADER_BYTES + (nt * KT + kt) * TILE_BYTES + word * 4 + b
+    byte = blob[src]
+    q[:] = np.where(high, byte >> 4, byte & 0x0F)
+    g = np.arange(K // group)[None, :]
+    msrc = HEADER_BYTES + (nt * KT + g) * TILE_BYTES + TILE_CODE_BYTES + r
+    meta = blob[msrc]
+    z[:] = meta & 0x0F
+    s2[:] = (meta >> 4) + 1
+    s1 = np.frombuffer(bytes(blob[s1_off:s1_off + 2 * N]), dtype=np.float16).copy()
+    return q, z, s2, s1, N, K
+
+
+# ---------------------------------------------------------------------------
+# GEMM
+# ---------------------------------------------------------------------------
+def gemm_acc(A8: np.ndarray, W8: np.ndarray) -> np.ndarray:
+    """acc[m,n] = sum_k A8[m,k] * W8[n,k] (int32).
+
+    Computed as an fp64 matmul of the integer values, which is exact here:
+    every product and partial sum is an integer of magnitude below
+    127 * 120 * K < 2**53.
+    """
+    assert A8.dtype == np.int8 and W8.dtype == np.int8
+    assert A8.shape[1] == W8.shape[1]
+    assert 127 * 120 * A8.shape[1] < 2 ** 31
+    acc = A8.astype(np.float64) @ W8.astype(np.float64).T
+    return acc.astype(np.int64).astype(np.int32)
+
+
+def epilogue(acc: np.ndarray, sA: np.ndarray, s1: np.ndarray) -> np.ndarray:
+    """Y[m,n] = fp16_rn(float(acc[m,n]) * (float(sA[m]) * float(s1[n]))), fp32."""
+    scale = sA.astype(np.float32)[:, None] * s1.astype(np.float32)[None, :]
+    with np.errstate(over="ignore"):
+        return (acc.astype(np.float32) * scale).astype(np.float16)
+
+
+def w4a8_gemm(A8, sA, q, z, s2, s1, group: int = GROUP) -> np.ndarray:
+    """Y = fp16(sA[m] * s1[n] * sum_k A8[m,k] * (q[n,k] - z) * s2)."""
+    return epilogue(gemm_acc(A8, dequant_weights(q, z, s2, group)), sA, s1)
+
+
+def w4a8_gemm_packed(A8, sA, blob) -> np.ndarray:
+    q, z, s2, s1, N, K = unpack_weights(blob)
+    return w4a8_gemm(A8, sA, q, z, s2, s1)

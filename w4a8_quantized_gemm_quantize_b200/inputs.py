@@ -1,0 +1,115 @@
+"""Seeded synthetic inputs for the W4A8 GEMM workloads.
+
+This module only draws random numbers and names the layer shapes. It holds
+none of the quantization or GEMM arithmetic: both the CUDA path and the CPU
+oracle consume what it returns.
+
+Workloads (the low-bit LLM-serving layers the pages study: Llama-3-8B and
+Qwen1.5-72B linears, "QServe/QoQ" abstract on the lmdeploy issue
+"[Feature] Support W4A8KV4 Quantization(QServe/QoQ)", Motivation):
+
+* ``tiny``     M=16, K=512, N=256; codes drawn directly (q, z ~ U[0,15],
+               s2 ~ U{1..8}, s1 ~ U[0.001, 0.01] as fp16).
+* ``decode``   M in {1, 8, 16, 32} on the four Llama-3-8B linears.
+* ``serving``  M in {64, 128, 256, 512} on the same linears.
+* ``prefill``  M in {2048, 8192} on the same linears.
+* ``qwen72b``  M in {1, 32, 256, 4096} on the four Qwen1.5-72B linears.
+
+Activations are fp16 N(0, 1) with round(0.01*K) outlier channels scaled by
+20; the outlier channels depend on K only, so every token of a layer shares
+them. Dense weights are fp32 N(0, std) with std 0.02 (Llama) or 0.015 (Qwen).
+"""
+from __future__ import annotations
+
+import hashlib
+from dataclasses import dataclass
+
+import numpy as np
+
+GROUP = 128
+
+LLAMA3_8B_LINEARS = (
+    ("qkv", 6144, 4096),
+    ("o", 4096, 4096),
+    ("gate_up", 28672, 4096),
+    ("down", 4096, 14336),
+)
+QWEN15_72B_LINEARS = (
+    ("qkv", 24576, 8192),
+    ("o", 8192, 8192),
+    ("gate_up", 49152, 8192),
+    ("down", 8192, 24576),
+)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    ms: tuple
+    linears: tuple  # (layer name, N, K)
+    weight_std: float  # 0.0 means: draw codes directly (tiny case)
+
+
+WORKLOADS = {
+    "tiny": Workload("tiny", (16,), (("tiny", 256, 512),), 0.0),
+    "decode": Workload("decode", (1, 8, 16, 32), LLAMA3_8B_LINEARS, 0.02),
+    "serving": Workload("serving", (64, 128, 256, 512), LLAMA3_8B_LINEARS, 0.02),
+    "prefill": Workload("prefill", (2048, 8192), LLAMA3_8B_LINEARS, 0.02),
+    "qwen72b": Workload("qwen72b", (1, 32, 256, 4096), QWEN15_72B_LINEARS, 0.015),
+}
+
+
+def seed_of(*parts) -> int:
+    """A 63-bit seed derived from a descriptor tuple (stable across runs)."""
+    h = hashlib.sha256(repr(parts).encode()).digest()
+    return int.from_bytes(h[:8], "little") & ((1 << 63) - 1)
+
+
+def n_outlier_channels(K: int) -> int:
+    """round(0.01*K), halves rounded up (K=512 -> 5, 4096 -> 41, 14336 -> 143)."""
+    return int(np.floor(0.01 * K + 0.5))
+
+
+def outlier_channels(K: int) -> np.ndarray:
+    rng = np.random.default_rng(seed_of("outlier-channels", K))
+    return np.sort(rng.choice(K, size=n_outlier_channels(K), replace=False))
+
+
+def activations(M: int, K: int, seed: int, outlier_scale: float = 20.0) -> np.ndarray:
+    """fp16 [M, K] row-major: N(0,1) with the layer's outlier channels x20."""
+    rng = np.random.default_rng(seed)
+    a = rng.standard_normal((M, K), dtype=np.float32)
+    ch = outlier_channels(K)
+    if ch.size:
+        a[:, ch] *= np.float32(outlier_scale)
+    return a.astype(np.float16)
+
+
+def dense_weights(N: int, K: int, std: float, seed: int) -> np.ndarray:
+    """fp32 [N, K] row-major, N(0, std)."""
+    rng = np.random.default_rng(seed)
+    w = rng.standard_normal((N, K), dtype=np.float32)
+    w *= np.float32(std)
+    return w
+
+
+def uniform_codes(N: int, K: int, seed: int, group: int = GROUP):
+    """Codes drawn directly: q, z ~ U[0,15]; s2 ~ U{1..8}; s1 ~ U[0.001, 0.01] fp16.
+
+    Returns (q uint8 [N,K], z uint8 [N,K/group], s2 uint8 [N,K/group], s1 fp16 [N]).
+    """
+    rng = np.random.default_rng(seed)
+    G = K // group
+    q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    z = rng.integers(0, 16, size=(N, G), dtype=np.uint8)
+    s2 = rng.integers(1, 9, size=(N, G), dtype=np.uint8)
+    s1 = rng.uniform(0.001, 0.01, size=N).astype(np.float16)
+    return q, z, s2, s1
+
+
+def activation_seed(workload: str, M: int, K: int) -> int:
+    return seed_of("act", workload, M, K)
+
+
+def weight_seed(workload: str, N: int, K: int) -> int:
+    return seed_of("weight", workload, N, K)
