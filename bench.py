@@ -1,0 +1,502 @@
+"""Benchmark of the W4A8 hot path on B200: activation quantization + W4A8 GEMM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode]
+                    [--impl w4a8|reference]
+
+One step = one pass of the hot path over the workload's cases: for every
+(M, layer) pair, `w4a8_quantize_act` of that layer's fp16 activations, then
+`w4a8_gemm` against the layer's packed 4-bit weights. Weight quantization and
+packing are offline (done once before timing). Default workload: Llama-3-8B
+decode linears (qkv 6144x4096, o 4096x4096, gate_up 28672x4096,
+down 4096x14336) at M in {1, 8, 16, 32}, group 128; 16 GEMMs per step.
+
+Each M value streams its own copy of the packed weights, so a step touches
+436 MB of distinct weights (> the 126 MB L2) and no GEMM finds its weights in
+L2. The W warm-up steps run eagerly; the K timed steps are one CUDA graph
+(K steps unrolled) replayed once between two events, with an event pair
+around every GEMM launch for the per-kernel roofline.
+
+`value` is the weight-stream rate: packed weight bytes streamed per second
+over the whole step (quantization included), summed over ranks.
+
+`--impl reference` times the CPU oracle on the host cores instead (bounded
+sample of the same workload), printing the same kind of line.
+
+Multi-GPU: the path does not shard across GPUs here (replicas only): every
+rank runs the whole workload on its own GPU; the time is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from w4a8_quantized_gemm_quantize_b200 import inputs as I  # noqa: E402
+
+METRIC = "W4A8 GEMM TOPS & weight GB/s vs M on 1 B200, as % of INT8/HBM roofline"
+TILE_BYTES = 8320
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 vs 2.25 PFLOP/s bf16)
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "w4a8_gemm_dram_traffic.json")
+KERNEL_SOURCES = ("gemm.cuh", "ptx.cuh", "pack.cuh", "w4a8_api.cu")
+
+
+# ------------------------------------------------------------ workload facts
+def weight_bytes(N, K):
+    """Packed weight bytes a GEMM must stream: codes + meta + s1."""
+    return (N // 128) * (K // 128) * TILE_BYTES + 2 * N
+
+
+def algorithmic_bytes(M, N, K):
+    """Bytes a W4A8 GEMM must move at least: packed weights, int8
+    activations, the activation scales, the fp16 output."""
+    return weight_bytes(N, K) + M * K + 2 * M + 2 * M * N
+
+
+def gemm_ops(M, N, K):
+    return 2 * M * N * K
+
+
+def cases_of(workload):
+    wl = I.WORKLOADS[workload]
+    return [(M, name, N, K) for M in wl.ms for (name, N, K) in wl.linears]
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": HBM_FALLBACK_GBS, "bf16_tflops": BF16_FALLBACK_TFLOPS,
+                "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "w4a8_quantized_gemm_quantize_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload):
+    """DRAM bytes per GEMM launch from a committed ncu summary, if it was taken
+    on the current kernel sources (else None)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if t.get("kernel_source_hash") != kernel_source_hash():
+        return None
+    return t.get("per_launch_bytes", {}).get(workload)
+
+
+# ------------------------------------------------------------------- ranks
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def max_over_ranks(value: float, world: int) -> float:
+    """Max of a per-rank scalar over all ranks (identity with one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML in a thread."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+        0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+        0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+    }
+
+    def __init__(self, torch_device, period_s=0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            handle = None
+            try:
+                import torch
+                uuid = str(torch.cuda.get_device_properties(torch_device).uuid)
+                handle = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                handle = None
+            if handle is None:
+                vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+                idx = torch_device.index or 0
+                if vis and vis.split(",")[idx].strip().isdigit():
+                    idx = int(vis.split(",")[idx])
+                handle = pynvml.nvmlDeviceGetHandleByIndex(idx)
+            self.h = handle
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.ok = False
+
+    def _reasons(self):
+        try:
+            return self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception:
+            return self.nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons())
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# -------------------------------------------------------------- CPU oracle
+_ORACLE_WEIGHTS = {}
+
+
+def cpu_oracle_run(workload, budget_s, reps=1):
+    """Times the CPU oracle (quantize_act + GEMM with the fp32 epilogue) on
+    this host over a bounded sample of the workload's cases; returns
+    (weight GB/s, description of the sample, threads used)."""
+    from oracle import w4a8_oracle as O
+    cases = cases_of(workload)
+    prepared = _ORACLE_WEIGHTS
+    done_bytes, done_time, done = 0, 0.0, []
+    t_start = time.perf_counter()
+    for (M, name, N, K) in cases:
+        if time.perf_counter() - t_start > budget_s and done:
+            break
+        wl = I.WORKLOADS[workload]
+        key = (workload, N, K)
+        if key not in prepared:
+            if wl.weight_std == 0.0:
+                prepared[key] = I.uniform_codes(N, K, I.weight_seed(workload, N, K))
+            else:
+                W = I.dense_weights(N, K, wl.weight_std, I.weight_seed(workload, N, K))
+                prepared[key] = O.quantize_weights(W)
+        q, z, s2, s1 = prepared[key]
+        A = I.activations(M, K, I.activation_seed(workload, M, K))
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            A8, sA, _ = O.quantize_act(A)
+            O.w4a8_gemm(A8, sA, q, z, s2, s1)
+            done_time += time.perf_counter() - t0
+            done_bytes += weight_bytes(N, K)
+        done.append(f"M={M} {name} {N}x{K}")
+    threads = cpu_threads()
+    return done_bytes / done_time / 1e9, done, threads, done_time
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = max((int(p.get("num_threads", 1)) for p in threadpool_info()), default=1)
+        return n
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------- GPU arm
+def run_gpu(args, world, rank, local):
+    import torch
+    import w4a8_quantized_gemm_quantize_b200 as w4a8
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = I.WORKLOADS[args.workload]
+    cases = cases_of(args.workload)
+    n_copies = len(wl.ms)  # one weight copy per M value: no GEMM reuses L2-resident weights
+
+    # ---- offline: quantize + pack the weights (untimed), one copy per M
+    blobs = {}
+    for (name, N, K) in wl.linears:
+        if wl.weight_std == 0.0:
+            q, z, s2, s1 = (torch.from_numpy(x).to(dev) for x in I.uniform_codes(N, K, I.weight_seed(args.workload, N, K)))
+        else:
+            W = torch.from_numpy(I.dense_weights(N, K, wl.weight_std, I.weight_seed(args.workload, N, K))).to(dev)
+            q, z, s2, s1 = w4a8.quantize_weights(W)
+            del W
+        blob = w4a8.pack_weights(q, z, s2, s1)
+        del q, z, s2
+        blobs[(name, 0)] = blob
+        for c in range(1, n_copies):
+            blobs[(name, c)] = blob.clone()
+    torch.cuda.synchronize()
+
+    # ---- activations and outputs, resident in HBM
+    acts, outs = {}, {}
+    ws = torch.zeros(max(w4a8.workspace_bytes(M, N, K) for (M, _, N, K) in cases), dtype=torch.uint8, device=dev)
+    for (M, name, N, K) in cases:
+        acts[(M, name)] = torch.from_numpy(I.activations(M, K, I.activation_seed(args.workload, M, K))).to(dev)
+        outs[(M, name)] = (torch.empty((M, K), dtype=torch.int8, device=dev),
+                           torch.empty((M,), dtype=torch.float16, device=dev),
+                           torch.empty((M,), dtype=torch.int32, device=dev),
+                           torch.empty((M, N), dtype=torch.float16, device=dev))
+    copy_of = {M: i for i, M in enumerate(wl.ms)}
+
+    def step(events=None, h2d=None, d2h=None):
+        for i, (M, name, N, K) in enumerate(cases):
+            A = acts[(M, name)]
+            if h2d is not None:
+                A.copy_(h2d[(M, name)], non_blocking=True)
+            A8, sA, rs, Y = outs[(M, name)]
+            w4a8.quantize_act(A, out=(A8, sA, rs))
+            if events is not None:
+                events[i][0].record()
+            w4a8.gemm(A8, sA, blobs[(name, copy_of[M])], N, K, out=Y, workspace=ws)
+            if events is not None:
+                events[i][1].record()
+            if d2h is not None:
+                d2h[(M, name)].copy_(Y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert w4a8.get_device_error(dev) == 0
+
+    # ---- capture K steps (unrolled) with an event pair around every GEMM
+    K_steps = args.steps
+    ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in cases]
+          for _ in range(K_steps)]
+    g = torch.cuda.CUDAGraph()
+    cap_stream = torch.cuda.Stream(dev)
+    cap_stream.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(cap_stream):
+        with torch.cuda.graph(g, stream=cap_stream):
+            for s in range(K_steps):
+                step(events=ev[s])
+    torch.cuda.current_stream(dev).wait_stream(cap_stream)
+    g.replay()  # untimed replay: settles clocks and caches
+    torch.cuda.synchronize()
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream(dev)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        t0.record(stream)
+        g.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = t0.elapsed_time(t1)
+    max_ms = max_over_ranks(elapsed_ms, world)
+    assert w4a8.get_device_error(dev) == 0
+
+    per_case_ms = np.zeros(len(cases))
+    for s in range(K_steps):
+        for i in range(len(cases)):
+            per_case_ms[i] += ev[s][i][0].elapsed_time(ev[s][i][1])
+    per_case_ms /= K_steps
+    del g
+
+    # ---- end to end through the public API: pinned host A in, Y out
+    h2d = {k: torch.from_numpy(I.activations(M, K, I.activation_seed(args.workload, M, K))).pin_memory()
+           for (M, name, N, K) in cases for k in [(M, name)]}
+    d2h = {(M, name): torch.empty((M, N), dtype=torch.float16).pin_memory() for (M, name, N, K) in cases}
+    step(h2d=h2d, d2h=d2h)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K_steps):
+        step(h2d=h2d, d2h=d2h)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    # the copies of the e2e run carry the same activations: outputs must match
+    for (M, name, N, K) in cases:
+        assert torch.equal(d2h[(M, name)], outs[(M, name)][3].cpu())
+
+    return dict(elapsed_ms=elapsed_ms, max_ms=max_ms, per_case_ms=per_case_ms, clocks=clk.summary(),
+                e2e_ms=e2e_ms, cases=cases, n_copies=n_copies,
+                h2d_bytes=sum(M * K * 2 for (M, _, N, K) in cases),
+                d2h_bytes=sum(M * N * 2 for (M, _, N, K) in cases),
+                gpu_name=torch.cuda.get_device_name(dev))
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--impl", default="w4a8", choices=["w4a8", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the CPU-oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        return main_reference(args, world, rank)
+
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    r = run_gpu(args, world, rank, local)
+    cases = r["cases"]
+    peaks = load_peaks()
+    wbytes = sum(weight_bytes(N, K) for (M, _, N, K) in cases)
+    abytes = [algorithmic_bytes(M, N, K) for (M, _, N, K) in cases]
+    ops = [gemm_ops(M, N, K) for (M, _, N, K) in cases]
+    ms_step = r["max_ms"] / args.steps
+    value = world * wbytes / (ms_step * 1e-3) / 1e9
+    tops = world * sum(ops) / (ms_step * 1e-3) / 1e12
+
+    # roofline of the dominant kernel (the GEMM)
+    per = r["per_case_ms"]
+    gemm_ms = float(per.sum())
+    int8_peak_tops = peaks["bf16_tflops"] * INT8_OVER_BF16
+    hbm = peaks["hbm_gbs"]
+    roof_t = [max(b / (hbm * 1e9), o / (int8_peak_tops * 1e12)) * 1e3 for b, o in zip(abytes, ops)]
+    hbm_bound = sum(b / (hbm * 1e9) >= o / (int8_peak_tops * 1e12) for b, o in zip(abytes, ops)) * 2 >= len(cases)
+    if hbm_bound:
+        achieved = sum(abytes) / (gemm_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                    "frac": round(achieved / hbm, 4)}
+    else:
+        achieved = sum(ops) / (gemm_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": int8_peak_tops,
+                    "unit": "TOPS", "frac": round(achieved / int8_peak_tops, 4)}
+    traffic = recorded_traffic(args.workload)
+    roofline["traffic"] = traffic
+    roofline["peak_source"] = (f"{peaks['source']} HBM copy" if hbm_bound else
+                               f"{peaks['source']} bf16 burst x {INT8_OVER_BF16:g} (nominal int8/bf16 ratio)")
+    roofline["kernel"] = "w4a8_gemm_kernel"
+    roofline["roofline_time_frac"] = round(sum(roof_t) / gemm_ms, 4)
+    roofline["launches"] = len(cases) * args.steps
+
+    per_case = []
+    for (M, name, N, K), t, b, o, rt in zip(cases, per, abytes, ops, roof_t):
+        per_case.append({"M": M, "layer": name, "N": N, "K": K, "us": round(t * 1e3, 2),
+                         "weight_GBs": round(weight_bytes(N, K) / (t * 1e-3) / 1e9, 1),
+                         "tops": round(o / (t * 1e-3) / 1e12, 2), "roofline_frac": round(rt / t, 3)})
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": args.workload, "cases": len(cases),
+                   "shapes": [f"M={M} {n} {N}x{K}" for (M, n, N, K) in cases][:: max(1, len(cases) // 16)],
+                   "group": 128, "weights_per_step_MB": round(wbytes / 1e6, 1),
+                   "l2": f"inputs larger than L2: {r['n_copies']} weight copies, {wbytes / 1e6:.0f} MB per step",
+                   "parallelism": f"replicas x{world}", "timing": "one CUDA graph of K unrolled steps"},
+        "tops": round(tops, 2),
+        "gpu_launches": 2 * len(cases) * args.steps,
+        "roofline": roofline,
+        "e2e": {"value": round(world * wbytes / (r["e2e_ms"] / args.steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"]},
+        "clocks": r["clocks"],
+        "cases": per_case,
+        "gpu": r["gpu_name"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{len(sample)} of {len(cases)} cases ({'; '.join(sample)}), "
+                                          f"{t:.1f} s of oracle time"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def main_reference(args, world, rank):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return
+    cases = cases_of(args.workload)
+    cpu_oracle_run(args.workload, 0.0)  # untimed warm-up (one case)
+    t0 = time.perf_counter()
+    tot_bytes, tot_t, samples = 0.0, 0.0, []
+    for _ in range(args.steps):
+        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds / max(args.steps, 1))
+        tot_t += t
+        tot_bytes += v * t * 1e9
+        samples = sample
+    value = tot_bytes / tot_t / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
+        "config": {"workload": args.workload, "cases": len(cases), "group": 128},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"per step: {len(samples)} of {len(cases)} cases ({'; '.join(samples)})"},
+        "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "wall_s": round(time.perf_counter() - t0, 1),
+    }
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * w4a8.h — C ABI of the B200 (sm_100a) W4A8 quantized GEMM library.
+ *
+ * The operation is the W4A8 GEMM of QServe/QoQ: 4-bit weights, 8-bit
+ * activations, with a progressive (two-level) weight quantization that keeps
+ * dequantization inside the GEMM cheap ("QServe/QoQ" abstract, quoted in the
+ * lmdeploy issue "[Feature] Support W4A8KV4 Quantization(QServe/QoQ)",
+ * Motivation; "LiquidGEMM: Hardware-Efficient W4A8 GEMM Kernel for
+ * High-Performance LLM Serving", Method):
+ *
+ *   W8[n,k] = (q[n,k] - z[n,g]) * s2[n,g]        g = k / 128, exact int8
+ *   acc[m,n] = sum_k A8[m,k] * W8[n,k]            int32
+ *   Y[m,n]  = fp16_rn(float(acc) * (float(sA[m]) * float(s1[n])))
+ *
+ * with q, z in [0, 15] (uint4), s2 in [1, 8], s1 a per-output-channel fp16
+ * scale and (A8, sA) the per-token symmetric int8 quantization of the fp16
+ * activations.
+ *
+ * Conventions for every call:
+ *  - All data pointers are DEVICE pointers, allocated and owned by the
+ *    caller; the library allocates, frees and synchronizes nothing (except
+ *    w4a8_get_device_error, which synchronizes the given stream).
+ *  - Work is enqueued on `stream` (NULL = the legacy default stream) and is
+ *    asynchronous; a returned W4A8_OK means "validated and launched".
+ *  - Arguments are validated on the host before any launch; on error nothing
+ *    is launched. A launch failure returns W4A8_ERR_CUDA after reading (and
+ *    thereby clearing) the CUDA runtime's last error.
+ *  - Data pointers must be 16-byte aligned unless stated otherwise.
+ *  - Matrices are row-major and dense (leading dimension = row length).
+ */
+#ifndef W4A8_H_
+#define W4A8_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(W4A8_BUILD)
+#define W4A8_API __attribute__((visibility("default")))
+#else
+#define W4A8_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* w4a8_stream_t;
+
+typedef enum {
+  W4A8_OK = 0,
+  W4A8_ERR_INVALID_ARG = 1,       /* null pointer, negative size, bad option */
+  W4A8_ERR_UNSUPPORTED_SHAPE = 2, /* shape outside the documented limits */
+  W4A8_ERR_MISALIGNED = 3,        /* pointer not aligned as required */
+  W4A8_ERR_WORKSPACE = 4,         /* workspace missing or too small */
+  W4A8_ERR_CUDA = 5,              /* CUDA runtime / launch error */
+  W4A8_ERR_DEVICE = 6             /* a kernel gave up a bounded wait (see below) */
+} w4a8_status_t;
+
+/* Device error word values (w4a8_get_device_error). */
+#define W4A8_DEVERR_NONE 0
+#define W4A8_DEVERR_PRODUCER_WAIT 1
+#define W4A8_DEVERR_MMA_WAIT 2
+#define W4A8_DEVERR_DEQUANT_WAIT 3
+#define W4A8_DEVERR_EPILOGUE_WAIT 4
+#define W4A8_DEVERR_DRAIN_WAIT 5
+
+/* Human-readable name of a status code (static string, never NULL). */
+W4A8_API const char* w4a8_status_string(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+W4A8_API int w4a8_version(void);
+
+/*
+ * Per-token symmetric int8 quantization of activations (the 8-bit activation
+ * side of W4A8; per-token dynamic scaling as in the "PrefixQuant" page, Key
+ * Findings). For each row m:
+ *   amax = max_k |A[m,k]|
+ *   sA[m] = fp16_rn(amax / 127)                       (IEEE fp32 divide)
+ *   A8[m,k] = clamp(rint(A[m,k] / float(sA[m])), -127, 127)
+ *                                     (IEEE fp32 divide, ties to even)
+ *   sA[m] == 0 gives A8[m,:] = 0;  rowsum[m] = sum_k A8[m,k].
+ * A: fp16 [M, K]. A8: int8 [M, K]. sA: fp16 [M] (2-byte aligned).
+ * rowsum: int32 [M] (4-byte aligned) or NULL.
+ * Limits: M >= 0 (M == 0 is a no-op), 0 < K <= 65536, K % 8 == 0.
+ * Non-finite inputs are a precondition violation (codes unspecified).
+ */
+W4A8_API w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, int8_t* A8, void* sA, int32_t* rowsum,
+                                w4a8_stream_t stream);
+
+/*
+ * Offline two-level weight quantization (the "progressive quantization" of
+ * the QServe/QoQ abstract), fp32 W [N, K] -> (q, z, s2, s1):
+ *   level 1 (row n): r_g = max(max W_g, 0) - min(min W_g, 0) over each
+ *     group g of 128; s1[n] = fp16_rn(max_g r_g / 120), 1 if that is 0;
+ *     t = W / float(s1[n]).
+ *   level 2 (group): lo = min(min t, 0), hi = max(max t, 0);
+ *     s2 = clamp(ceil((hi - lo) / 15), 1, 8);  z = clamp(rint(-lo / s2), 0, 15);
+ *     q = clamp(rint(t / s2) + z, 0, 15).          (IEEE fp32 divides)
+ * so that (q - z) * s2 lies in [-120, 120].
+ * q: uint8 [N, K] one code per byte. z, s2: uint8 [N, K/128] (no alignment
+ * requirement). s1: fp16 [N] (2-byte aligned).
+ * Limits: group == 128, K % 128 == 0, 0 < K <= 65536, N >= 0.
+ */
+W4A8_API w4a8_status_t w4a8_quantize_weights(const float* W, int64_t N, int64_t K, int32_t group, uint8_t* q, uint8_t* z,
+                                    uint8_t* s2, void* s1, w4a8_stream_t stream);
+
+/* Size in bytes of the packed blob for an N x K weight (0 if unsupported). */
+W4A8_API size_t w4a8_packed_bytes(int64_t N, int64_t K, int32_t group);
+
+/*
+ * Offline reordering of (q, z, s2, s1) into the GEMM's packed blob
+ * (compute-aware weight reordering, "QServe/QoQ" abstract; offline
+ * interleaving, "QUICK" abstract). Layout, little-endian:
+ *   header, 64 bytes: u32 magic "W4A8", u32 version 1, i64 N, i64 K,
+ *     i32 group, u32 tile bytes (8320), u64 byte offset of s1, zeros.
+ *   tiles: (N/128) x (K/128) tiles of 8320 bytes; tile (nt, kt) at
+ *     64 + (nt * K/128 + kt) * 8320 holds 8192 code bytes then 128 meta bytes.
+ *     Row r (n = 128 nt + r) keeps the codes of in-tile k = 8j .. 8j+7 in
+ *     32-bit word j, byte b holding k = 8j+b (low nibble) and k = 8j+4+b
+ *     (high nibble); word j of row r is word ((j/4)*128 + r)*4 + j%4 of the
+ *     tile. Meta byte r = z | ((s2 - 1) << 4) of group kt.
+ *   s1: N fp16 values, zero padded to a multiple of 16 bytes.
+ * q/z/s2/s1 as produced by w4a8_quantize_weights (q and s1 16-byte aligned).
+ * packed: packed_bytes >= w4a8_packed_bytes(N, K, group).
+ * Limits: group == 128, N % 128 == 0, K % 128 == 0, 0 < K <= 65536.
+ */
+W4A8_API w4a8_status_t w4a8_pack_weights(const uint8_t* q, const uint8_t* z, const uint8_t* s2, const void* s1, int64_t N,
+                                int64_t K, int32_t group, void* packed, size_t packed_bytes, w4a8_stream_t stream);
+
+/*
+ * Workspace for w4a8_gemm / w4a8_gemm_debug_acc / w4a8_gemm_ex: int32
+ * partial sums and per-tile tickets used when one output tile's k-range is
+ * split across CTAs (the decode regime). The caller zero-fills it ONCE before
+ * first use; every call that completes without a device error leaves it
+ * zero-filled again. Calls that share a workspace must not overlap in time.
+ * A workspace of the returned size serves every M' <= M, N' <= N.
+ */
+W4A8_API size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/*
+ * Y = fp16(sA[m] * s1[n] * sum_k A8[m,k] * W8[n,k]), W8 decoded from the
+ * packed blob in registers (see the top of this file).
+ * A8: int8 [M, K] (from w4a8_quantize_act). sA: fp16 [M] (2-byte aligned).
+ * packed: the blob of w4a8_pack_weights for exactly this N and K.
+ * Y: fp16 [M, N]. workspace: see w4a8_gemm_workspace_bytes; with too small a
+ * workspace (including NULL / 0) the call uses a schedule that needs none.
+ * Limits: M >= 0 (M == 0 is a no-op), N % 128 == 0, K % 128 == 0,
+ * 0 < K <= 65536, M * N < 2^62.
+ */
+W4A8_API w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
+                        void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream);
+
+/*
+ * Debug entry point: the same GEMM, writing the raw int32 accumulators
+ * acc[m,n] = sum_k A8[m,k] * W8[n,k] to `acc` [M, N] instead of Y.
+ */
+W4A8_API w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const void* packed, int64_t M, int64_t N, int64_t K,
+                                  int32_t* acc, void* workspace, size_t workspace_bytes, w4a8_stream_t stream);
+
+/* Scheduling overrides for tests and tuning (zero = automatic). */
+typedef struct {
+  int32_t schedule;  /* 0 auto, 1 whole tiles per CTA, 2 split k-ranges (needs workspace) */
+  int32_t block_m;   /* tokens per tile: 0 auto, or 16, 32, 64, 128 */
+  int32_t max_ctas;  /* 0 auto (one CTA per SM), else an upper bound on the grid */
+  int32_t reserved;  /* must be 0 */
+} w4a8_gemm_opts_t;
+
+/*
+ * w4a8_gemm with overrides. Exactly one of Y (fp16 output) and acc (int32
+ * accumulators) must be non-NULL; sA may be NULL when acc is given.
+ * opts may be NULL (= all automatic).
+ */
+W4A8_API w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
+                           void* Y, int32_t* acc, void* workspace, size_t workspace_bytes,
+                           const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
+
+/*
+ * Synchronizes `stream`, then stores the current device's error word in
+ * *code (W4A8_DEVERR_*; 0 = no kernel gave up a wait). Returns W4A8_ERR_CUDA
+ * if the synchronization itself fails. The word stays set until cleared.
+ */
+W4A8_API w4a8_status_t w4a8_get_device_error(w4a8_stream_t stream, int32_t* code);
+
+/* Resets the current device's error word to 0 (stream-ordered). */
+W4A8_API w4a8_status_t w4a8_clear_device_error(w4a8_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A8_H_ */

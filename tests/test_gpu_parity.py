@@ -1,0 +1,279 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on
+the same seeded inputs.
+
+Bars: int8 activation codes, fp16 scales, rowsums, weight codes and the
+packed blob are bit/byte-exact; the int32 accumulators are bit-exact; the
+fp16 output is within 1 fp16 ulp of the oracle (both sides round the same
+fp32 epilogue, so it is expected to be exact; the test allows the 1-ulp
+tolerance that the specification grants).
+
+The oracle always derives its own codes from the seeded fp32 / fp16 inputs;
+nothing it consumes comes from the GPU.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import w4a8_quantized_gemm_quantize_b200 as w4a8
+from w4a8_quantized_gemm_quantize_b200 import inputs as I
+from oracle import w4a8_oracle as O
+from tests._util import max_ulp_fp16
+
+pytestmark = pytest.mark.gpu
+
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+DEV = torch.device("cuda:0")
+
+
+def dev(a: np.ndarray):
+    return torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+@pytest.fixture(autouse=True)
+def _no_device_error():
+    w4a8.clear_device_error(DEV)
+    yield
+    assert w4a8.get_device_error(DEV) == 0
+
+
+# -------------------------------------------------------- quantize_act
+def special_rows(K):
+    rows = [np.zeros(K), np.full(K, 3.0), np.full(K, -65504.0), np.full(K, 6e-8)]
+    r = np.zeros(K)
+    r[K // 3] = 1e-3
+    rows.append(r)
+    r = np.linspace(-1, 1, K)
+    rows.append(r)
+    return np.stack(rows).astype(np.float16)
+
+
+@pytest.mark.parametrize("M,K", [(1, 512), (3, 4096), (17, 14336), (64, 24576), (5, 65536), (300, 1024), (2, 8)])
+def test_quantize_act_bit_exact(M, K):
+    A = I.activations(M, K, I.seed_of("t-qa", M, K))
+    if K >= 8:
+        S = special_rows(K)
+        A = np.concatenate([A, S], axis=0)
+    A8, sA, rs = w4a8.quantize_act(dev(A))
+    torch.cuda.synchronize()
+    oA8, osA, ors = O.quantize_act(A)
+    assert (host(A8) == oA8).all()
+    assert (host(sA).view(np.uint16) == osA.view(np.uint16)).all()
+    assert (host(rs) == ors).all()
+
+
+def test_quantize_act_empty():
+    A = torch.empty((0, 256), dtype=torch.float16, device=DEV)
+    A8, sA, rs = w4a8.quantize_act(A)
+    assert A8.shape == (0, 256)
+
+
+# ----------------------------------------------------- quantize_weights
+@pytest.mark.parametrize("N,K,std", [(256, 512, 0.02), (384, 4096, 0.015), (128, 14336, 0.02), (130, 128, 1.0)])
+def test_quantize_weights_bit_exact(N, K, std):
+    W = I.dense_weights(N, K, std, I.seed_of("t-qw", N, K))
+    W[0] = 0.0                       # all-zero row: s1 = 1, zero codes
+    W[1, :128] = 0.0                 # an all-zero group
+    W[2] = np.abs(W[2])              # one-signed rows
+    W[3] = -np.abs(W[3])
+    q, z, s2, s1 = w4a8.quantize_weights(dev(W))
+    torch.cuda.synchronize()
+    oq, oz, os2, os1 = O.quantize_weights(W)
+    assert (host(q) == oq).all()
+    assert (host(z) == oz).all()
+    assert (host(s2) == os2).all()
+    assert (host(s1).view(np.uint16) == os1.view(np.uint16)).all()
+
+
+# ----------------------------------------------------------------- pack
+@pytest.mark.parametrize("N,K", [(128, 128), (256, 512), (384, 1152)])
+def test_pack_byte_exact(N, K):
+    q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-pack", N, K))
+    blob = w4a8.pack_weights(dev(q), dev(z), dev(s2), dev(s1))
+    torch.cuda.synchronize()
+    ob = O.pack_weights(q, z, s2, s1)
+    assert (host(blob) == ob).all()
+
+
+# ----------------------------------------------------------------- GEMM
+def gpu_path_from_codes(q, z, s2, s1):
+    return w4a8.pack_weights(dev(q), dev(z), dev(s2), dev(s1))
+
+
+def check_gemm(A, q, z, s2, s1, schedules=((0, 0, 0),)):
+    """A fp16 host, codes host; runs the GPU path from the same inputs."""
+    M, K = A.shape
+    N = q.shape[0]
+    blob = gpu_path_from_codes(q, z, s2, s1)
+    A8, sA, _ = w4a8.quantize_act(dev(A))
+    oA8, osA, _ = O.quantize_act(A)
+    oacc = O.gemm_acc(oA8, O.dequant_weights(q, z, s2))
+    oY = O.epilogue(oacc, osA, s1)
+    ws = torch.zeros(w4a8.workspace_bytes(M, N, K), dtype=torch.uint8, device=DEV)
+    for sched, bm, ctas in schedules:
+        acc = w4a8.gemm_ex(A8, None, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
+                           workspace=ws, schedule=sched, block_m=bm, max_ctas=ctas)
+        Y = w4a8.gemm_ex(A8, sA, blob, N, K, Y=torch.empty((M, N), dtype=torch.float16, device=DEV),
+                         workspace=ws, schedule=sched, block_m=bm, max_ctas=ctas)
+        torch.cuda.synchronize()
+        ha = host(acc)
+        bad = np.argwhere(ha != oacc)
+        assert bad.size == 0, (sched, bm, ctas, bad[:5], ha[tuple(bad[0])], oacc[tuple(bad[0])])
+        assert max_ulp_fp16(host(Y), oY) <= 1, (sched, bm, ctas)
+        assert not host(ws).any(), "workspace must be left zero-filled"
+    return oY
+
+
+ALL_SCHEDULES = [(0, 0, 0)] + [(s, bm, c) for s in (1, 2) for bm in (16, 32, 64, 128) for c in (0, 7)]
+
+
+@pytest.mark.parametrize("M", [1, 16, 33])
+def test_gemm_tiny_config_all_schedules(M):
+    """The tiny case (K=512, N=256, codes drawn directly) through every
+    schedule, token-tile size and a small grid (more work per CTA)."""
+    N, K = 256, 512
+    q, z, s2, s1 = I.uniform_codes(N, K, I.weight_seed("tiny", N, K))
+    A = I.activations(M, K, I.activation_seed("tiny", M, K))
+    check_gemm(A, q, z, s2, s1, ALL_SCHEDULES)
+
+
+@pytest.mark.parametrize("M,N,K", [(3, 384, 1024), (17, 512, 640), (65, 256, 2048), (129, 384, 512),
+                                   (200, 128, 384), (1, 1024, 4096), (300, 640, 256)])
+def test_gemm_ragged_shapes(M, N, K):
+    q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-g", N, K))
+    A = I.activations(M, K, I.seed_of("t-a", M, K))
+    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (1, 0, 0), (2, 0, 0), (2, 16, 5), (1, 128, 3)])
+
+
+def test_gemm_extreme_codes():
+    """Largest |W8| = 120 with largest |A8| = 127 over K = 65536: |acc| reaches
+    127 * 120 * 65536 = 998,768,640 (no int32 overflow)."""
+    N, K, M = 128, 65536, 2
+    q = np.zeros((N, K), np.uint8)
+    q[::2] = 15
+    z = np.zeros((N, K // 128), np.uint8)
+    z[1::2] = 15
+    s2 = np.full((N, K // 128), 8, np.uint8)
+    s1 = np.full(N, 1e-3, np.float16)
+    A = np.full((M, K), 1.0, np.float16)
+    A[1] = -1.0
+    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (2, 0, 0)])
+
+
+def test_gemm_zero_rows_and_columns():
+    N, K, M = 256, 512, 20
+    q, z, s2, s1 = I.uniform_codes(N, K, 77)
+    q[5] = np.repeat(z[5], 128)      # a weight row that dequantizes to 0
+    A = I.activations(M, K, 78)
+    A[4] = 0                         # a zero token: sA = 0
+    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (2, 16, 0)])
+
+
+def test_gemm_empty_m():
+    N, K = 256, 512
+    q, z, s2, s1 = I.uniform_codes(N, K, 5)
+    blob = gpu_path_from_codes(q, z, s2, s1)
+    A8 = torch.empty((0, K), dtype=torch.int8, device=DEV)
+    sA = torch.empty((0,), dtype=torch.float16, device=DEV)
+    Y = w4a8.gemm(A8, sA, blob, N, K)
+    assert Y.shape == (0, N)
+
+
+def test_gemm_without_workspace_uses_whole_tiles():
+    N, K, M = 512, 1024, 8
+    q, z, s2, s1 = I.uniform_codes(N, K, 9)
+    A = I.activations(M, K, 10)
+    blob = gpu_path_from_codes(q, z, s2, s1)
+    A8, sA, _ = w4a8.quantize_act(dev(A))
+    empty_ws = torch.zeros(16, dtype=torch.uint8, device=DEV)
+    Y = w4a8.gemm(A8, sA, blob, N, K, workspace=empty_ws)
+    oA8, osA, _ = O.quantize_act(A)
+    oY = O.w4a8_gemm(oA8, osA, q, z, s2, s1)
+    torch.cuda.synchronize()
+    assert max_ulp_fp16(host(Y), oY) <= 1
+
+
+def test_gemm_split_k_requires_workspace():
+    N, K, M = 256, 512, 4
+    q, z, s2, s1 = I.uniform_codes(N, K, 11)
+    blob = gpu_path_from_codes(q, z, s2, s1)
+    A8 = torch.zeros((M, K), dtype=torch.int8, device=DEV)
+    with pytest.raises(w4a8.W4A8Error, match="WORKSPACE"):
+        w4a8.gemm_ex(A8, None, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
+                     workspace=torch.zeros(16, dtype=torch.uint8, device=DEV), schedule=2)
+
+
+# ------------------------------------------- full-size workload checks
+def _full_size_case(workload, lin, M, n_random_cols=64):
+    """Runs the GPU path end to end from the seeded fp32 weights and fp16
+    activations at full size (the launch configuration the benchmark uses)
+    and compares every token against the oracle on sampled output channels:
+    two whole 128-channel tiles plus random channels. The oracle quantizes
+    only the weight rows it needs (rows are independent)."""
+    wl = I.WORKLOADS[workload]
+    name, N, K = lin
+    W = I.dense_weights(N, K, wl.weight_std, I.weight_seed(workload, N, K))
+    A = I.activations(M, K, I.activation_seed(workload, M, K))
+    Wd = dev(W)
+    q, z, s2, s1 = w4a8.quantize_weights(Wd)
+    blob = w4a8.pack_weights(q, z, s2, s1)
+    del Wd
+    A8, sA, rs = w4a8.quantize_act(dev(A))
+    ws = torch.zeros(w4a8.workspace_bytes(M, N, K), dtype=torch.uint8, device=DEV)
+    Y = w4a8.gemm(A8, sA, blob, N, K, workspace=ws)
+    acc = w4a8.gemm_debug_acc(A8, blob, N, K, workspace=ws)
+    torch.cuda.synchronize()
+    # activations: full comparison
+    oA8, osA, ors = O.quantize_act(A)
+    assert (host(A8) == oA8).all() and (host(sA).view(np.uint16) == osA.view(np.uint16)).all()
+    assert (host(rs) == ors).all()
+    # sampled output channels
+    rng = np.random.default_rng(I.seed_of("cols", workload, N, K, M))
+    nt = N // 128
+    tiles = [0, int(rng.integers(1, nt))]
+    cols = np.unique(np.concatenate([np.arange(t * 128, t * 128 + 128) for t in tiles] +
+                                    [rng.choice(N, n_random_cols, replace=False)]))
+    oq, oz, os2, os1 = O.quantize_weights(W[cols])
+    assert (host(q[cols]) == oq).all() and (host(z[cols]) == oz).all()
+    assert (host(s2[cols]) == os2).all() and (host(s1[cols]).view(np.uint16) == os1.view(np.uint16)).all()
+    oacc = O.gemm_acc(oA8, O.dequant_weights(oq, oz, os2))
+    oY = O.epilogue(oacc, osA, os1)
+    ha = host(acc)[:, cols]
+    assert (ha == oacc).all()
+    assert max_ulp_fp16(host(Y)[:, cols], oY) <= 1
+    # the packed tiles of one whole n-tile, byte for byte
+    t = tiles[0]
+    KT = K // 128
+    sub = O.pack_weights(*O.quantize_weights(W[t * 128:(t + 1) * 128]))
+    hb = host(blob)
+    assert (hb[64 + t * KT * 8320:64 + (t + 1) * KT * 8320] == sub[64:64 + KT * 8320]).all()
+    assert not host(ws).any()
+
+
+@pytest.mark.parametrize("lin", I.LLAMA3_8B_LINEARS, ids=lambda l: l[0])
+@pytest.mark.parametrize("M", I.WORKLOADS["decode"].ms)
+def test_full_size_decode(lin, M):
+    _full_size_case("decode", lin, M)
+
+
+@pytest.mark.parametrize("lin", I.LLAMA3_8B_LINEARS, ids=lambda l: l[0])
+@pytest.mark.parametrize("M", [64, 512])
+def test_full_size_serving(lin, M):
+    _full_size_case("serving", lin, M)
+
+
+@pytest.mark.parametrize("lin", [I.LLAMA3_8B_LINEARS[1], I.LLAMA3_8B_LINEARS[3]], ids=lambda l: l[0])
+def test_full_size_prefill(lin):
+    _full_size_case("prefill", lin, 2048)
+
+
+@pytest.mark.parametrize("lin", [I.QWEN15_72B_LINEARS[1], I.QWEN15_72B_LINEARS[3]], ids=lambda l: l[0])
+@pytest.mark.parametrize("M", [1, 32])
+def test_full_size_qwen(lin, M):
+    _full_size_case("qwen72b", lin, M)

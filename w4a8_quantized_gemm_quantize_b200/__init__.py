@@ -1,0 +1,248 @@
+"""Python binding of the B200 W4A8 quantized GEMM library (libw4a8.so).
+
+Argument marshalling only: every computation runs in the CUDA kernels of
+libw4a8.so, called through its C ABI (include/w4a8.h) on the caller's
+current torch CUDA stream. There is no CPU or PyTorch fallback: if the
+library is missing or the tensors are not on a CUDA device, the calls raise.
+
+    A8, sA, rowsum = quantize_act(A)             # fp16 [M,K] -> int8, fp16, int32
+    q, z, s2, s1 = quantize_weights(W)           # fp32 [N,K] -> two-level codes
+    blob = pack_weights(q, z, s2, s1)            # offline reordering
+    Y = gemm(A8, sA, blob, N, K)                 # fp16 [M,N]
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "W4A8Error", "lib", "library_path", "EXPORTED_SYMBOLS", "status_string", "quantize_act",
+    "quantize_weights", "packed_bytes", "pack_weights", "workspace_bytes", "Workspace", "gemm",
+    "gemm_debug_acc", "gemm_ex", "get_device_error", "clear_device_error",
+]
+
+_PKG_DIR = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG_DIR, "libw4a8.so")
+
+EXPORTED_SYMBOLS = (
+    "w4a8_status_string", "w4a8_version", "w4a8_quantize_act", "w4a8_quantize_weights",
+    "w4a8_packed_bytes", "w4a8_pack_weights", "w4a8_gemm_workspace_bytes", "w4a8_gemm",
+    "w4a8_gemm_debug_acc", "w4a8_gemm_ex", "w4a8_get_device_error", "w4a8_clear_device_error",
+)
+
+SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K = 0, 1, 2
+
+
+class W4A8Error(RuntimeError):
+    pass
+
+
+class GemmOpts(ctypes.Structure):
+    _fields_ = [("schedule", ctypes.c_int32), ("block_m", ctypes.c_int32),
+                ("max_ctas", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libw4a8.so (built in-tree by the package's build module)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise W4A8Error(
+            f"{library_path} is missing: build it with `python -m w4a8_quantized_gemm_quantize_b200.build`")
+    L = ctypes.CDLL(library_path)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+    sig = {
+        "w4a8_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "w4a8_version": (ctypes.c_int, []),
+        "w4a8_quantize_act": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp]),
+        "w4a8_quantize_weights": (ctypes.c_int, [vp, i64, i64, i32, vp, vp, vp, vp, vp]),
+        "w4a8_packed_bytes": (sz, [i64, i64, i32]),
+        "w4a8_pack_weights": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i32, vp, sz, vp]),
+        "w4a8_gemm_workspace_bytes": (sz, [i64, i64, i64]),
+        "w4a8_gemm": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "w4a8_gemm_debug_acc": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "w4a8_gemm_ex": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, vp, vp, vp, sz,
+                                        ctypes.POINTER(GemmOpts), vp]),
+        "w4a8_get_device_error": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_int32)]),
+        "w4a8_clear_device_error": (ctypes.c_int, [vp]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def status_string(code: int) -> str:
+    return lib().w4a8_status_string(int(code)).decode()
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise W4A8Error(f"{what}: {status_string(code)}")
+
+
+# --------------------------------------------------------------- helpers
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device):
+    torch = _torch()
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise W4A8Error("tensors must live on a CUDA device (no CPU path exists)")
+            if not t.is_contiguous():
+                raise W4A8Error("tensors must be contiguous")
+
+
+# ------------------------------------------------------------------- API
+def quantize_act(A, out=None):
+    """fp16 [M, K] -> (A8 int8 [M, K], sA fp16 [M], rowsum int32 [M])."""
+    torch = _torch()
+    _require_cuda(A)
+    if A.dtype != torch.float16 or A.dim() != 2:
+        raise W4A8Error("A must be a 2-D fp16 tensor")
+    M, K = A.shape
+    if out is None:
+        A8 = torch.empty((M, K), dtype=torch.int8, device=A.device)
+        sA = torch.empty((M,), dtype=torch.float16, device=A.device)
+        rowsum = torch.empty((M,), dtype=torch.int32, device=A.device)
+    else:
+        A8, sA, rowsum = out
+        _require_cuda(A8, sA, rowsum)
+    _check(lib().w4a8_quantize_act(_ptr(A), M, K, _ptr(A8), _ptr(sA), _ptr(rowsum), _stream(A.device)),
+           "w4a8_quantize_act")
+    return A8, sA, rowsum
+
+
+def quantize_weights(W, group: int = 128):
+    """fp32 [N, K] -> (q uint8 [N,K], z uint8 [N,K/g], s2 uint8 [N,K/g], s1 fp16 [N])."""
+    torch = _torch()
+    _require_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise W4A8Error("W must be a 2-D fp32 tensor")
+    N, K = W.shape
+    G = K // group if group > 0 else 0
+    q = torch.empty((N, K), dtype=torch.uint8, device=W.device)
+    z = torch.empty((N, G), dtype=torch.uint8, device=W.device)
+    s2 = torch.empty((N, G), dtype=torch.uint8, device=W.device)
+    s1 = torch.empty((N,), dtype=torch.float16, device=W.device)
+    _check(lib().w4a8_quantize_weights(_ptr(W), N, K, group, _ptr(q), _ptr(z), _ptr(s2), _ptr(s1),
+                                       _stream(W.device)), "w4a8_quantize_weights")
+    return q, z, s2, s1
+
+
+def packed_bytes(N: int, K: int, group: int = 128) -> int:
+    return int(lib().w4a8_packed_bytes(N, K, group))
+
+
+def pack_weights(q, z, s2, s1, group: int = 128):
+    """Codes -> packed blob (uint8 tensor of packed_bytes(N, K))."""
+    torch = _torch()
+    _require_cuda(q, z, s2, s1)
+    N, K = q.shape
+    nbytes = packed_bytes(N, K, group)
+    if nbytes == 0:
+        raise W4A8Error(f"unsupported weight shape {N}x{K} (group {group})")
+    blob = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
+    _check(lib().w4a8_pack_weights(_ptr(q), _ptr(z), _ptr(s2), _ptr(s1), N, K, group, _ptr(blob), nbytes,
+                                   _stream(q.device)), "w4a8_pack_weights")
+    return blob
+
+
+def workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().w4a8_gemm_workspace_bytes(M, N, K))
+
+
+class Workspace:
+    """A zero-filled GEMM workspace that grows on demand (kept zero by the kernels)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf = None
+
+    def get(self, M: int, N: int, K: int):
+        torch = _torch()
+        need = workspace_bytes(M, N, K)
+        if need == 0:
+            return None
+        if self.buf is None or self.buf.numel() < need:
+            self.buf = torch.zeros((need,), dtype=torch.uint8, device=self.device)
+        return self.buf
+
+
+_default_ws = {}
+
+
+def _workspace_for(device, M, N, K):
+    key = str(device)
+    ws = _default_ws.get(key)
+    if ws is None:
+        ws = _default_ws[key] = Workspace(device)
+    return ws.get(M, N, K)
+
+
+def _gemm_common(A8, sA, blob, N, K, Y, acc, workspace, opts):
+    torch = _torch()
+    _require_cuda(A8, sA, blob, Y, acc, workspace)
+    M = A8.shape[0]
+    if A8.dtype != torch.int8 or A8.shape[1] != K:
+        raise W4A8Error("A8 must be int8 [M, K]")
+    if workspace is None:
+        workspace = _workspace_for(A8.device, M, N, K)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    o = None if opts is None else ctypes.byref(GemmOpts(*opts))
+    code = lib().w4a8_gemm_ex(_ptr(A8), _ptr(sA), _ptr(blob), M, N, K, _ptr(Y), _ptr(acc), _ptr(workspace),
+                              ws_bytes, o, _stream(A8.device))
+    _check(code, "w4a8_gemm_ex")
+
+
+def gemm(A8, sA, blob, N: int, K: int, out=None, workspace=None, opts=None):
+    """Y fp16 [M, N] = fp16(sA * s1 * (A8 @ W8^T))."""
+    torch = _torch()
+    M = A8.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A8.device)
+    _gemm_common(A8, sA, blob, N, K, Y, None, workspace, opts)
+    return Y
+
+
+def gemm_debug_acc(A8, blob, N: int, K: int, out=None, workspace=None, opts=None):
+    """int32 [M, N] accumulators sum_k A8[m,k] * W8[n,k]."""
+    torch = _torch()
+    M = A8.shape[0]
+    acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=A8.device)
+    _gemm_common(A8, None, blob, N, K, None, acc, workspace, opts)
+    return acc
+
+
+def gemm_ex(A8, sA, blob, N: int, K: int, Y=None, acc=None, workspace=None, schedule=0, block_m=0,
+            max_ctas=0):
+    """GEMM with explicit scheduling overrides (for tests and tuning)."""
+    _gemm_common(A8, sA, blob, N, K, Y, acc, workspace, (schedule, block_m, max_ctas, 0))
+    return Y if Y is not None else acc
+
+
+def get_device_error(device=None) -> int:
+    code = ctypes.c_int32(0)
+    _check(lib().w4a8_get_device_error(_stream(device), ctypes.byref(code)), "w4a8_get_device_error")
+    return int(code.value)
+
+
+def clear_device_error(device=None):
+    _check(lib().w4a8_clear_device_error(_stream(device)), "w4a8_clear_device_error")

@@ -1,0 +1,93 @@
+// Offline weight reordering into the GEMM's tile-native packed layout
+// (compute-aware reordering of the codes, as in the "QServe/QoQ" abstract;
+// offline interleaving so dequantized values never go back through shared
+// memory, as in the "QUICK" abstract).
+//
+// Blob = 64-byte header, then (N/128) x (K/128) tiles of 8320 bytes, then s1.
+// Tile (nt, kt) = 8192 code bytes + 128 meta bytes:
+//   row r's codes for in-tile k = 8j .. 8j+7 form 32-bit word j: byte b has
+//   k = 8j+b in its low nibble and k = 8j+4+b in its high nibble; word j of
+//   row r is at word index ((j/4)*128 + r)*4 + j%4. So a thread owning row r
+//   reads k = 32c .. 32c+31 as one 16-byte vector, a warp reads 512
+//   contiguous bytes, and `w & 0x0F0F0F0F` / `(w >> 4) & 0x0F0F0F0F` yield
+//   four consecutive k in the byte lanes of one register.
+//   meta byte r = z | ((s2 - 1) << 4) for group kt.
+// Header: u32 magic 'W4A8', u32 version 1, i64 N, i64 K, i32 group,
+// u32 tile bytes, u64 byte offset of s1; zero elsewhere.
+#pragma once
+#include "ptx.cuh"
+
+namespace w4a8 {
+
+constexpr int kTileN = 128;
+constexpr int kTileK = 128;
+constexpr int kTileCodeBytes = kTileN * kTileK / 2;  // 8192
+constexpr int kTileBytes = kTileCodeBytes + kTileN;  // 8320
+constexpr int kHeaderBytes = 64;
+constexpr uint32_t kMagic = 0x38413457u;  // "W4A8"
+constexpr uint32_t kLayoutVersion = 1u;
+
+// One thread per (row n, 32-k chunk): 32 codes in, one 16-byte vector out.
+__global__ void pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K,
+                                  uint8_t* __restrict__ tiles) {
+  const int64_t KC = K >> 5;  // 32-k chunks per row
+  const int64_t total = N * KC;
+  const int64_t KT = K >> 7;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / KC;
+    const int64_t kc = i - n * KC;  // global 32-chunk index
+    const uint4* src = reinterpret_cast<const uint4*>(q + n * K + kc * 32);
+    const uint4 a = src[0], b = src[1];
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};  // 4 codes per word, k ascending
+    uint32_t out[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      // word for k = 8jj .. 8jj+7 of this chunk: low nibbles k..k+3, high k+4..k+7
+      out[jj] = (in[2 * jj] & 0x0F0F0F0Fu) | ((in[2 * jj + 1] & 0x0F0F0F0Fu) << 4);
+    }
+    const int64_t nt = n >> 7, r = n & 127;
+    const int64_t kt = kc >> 2, c = kc & 3;
+    uint8_t* tile = tiles + (nt * KT + kt) * kTileBytes;
+    *reinterpret_cast<uint4*>(tile + (c * kTileN + r) * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+__global__ void pack_meta_kernel(const uint8_t* __restrict__ z, const uint8_t* __restrict__ s2,
+                                 const __half* __restrict__ s1, int64_t N, int64_t K, uint8_t* __restrict__ blob,
+                                 int64_t s1_offset) {
+  const int64_t G = K >> 7;
+  const int64_t total = N * G;
+  uint8_t* tiles = blob + kHeaderBytes;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / G, g = i - n * G;
+    const uint8_t meta = static_cast<uint8_t>((z[i] & 0x0F) | (((s2[i] - 1) & 0x0F) << 4));
+    tiles[((n >> 7) * G + g) * kTileBytes + kTileCodeBytes + (n & 127)] = meta;
+  }
+  __half* s1_out = reinterpret_cast<__half*>(blob + s1_offset);
+  const int64_t s1_padded = ((2 * N + 15) / 16) * 8;  // in halves
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < s1_padded;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    s1_out[i] = i < N ? s1[i] : __ushort_as_half(0);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < kHeaderBytes / 4) {
+    uint32_t w = 0;
+    switch (threadIdx.x) {
+      case 0: w = kMagic; break;
+      case 1: w = kLayoutVersion; break;
+      case 2: w = static_cast<uint32_t>(N); break;
+      case 3: w = static_cast<uint32_t>(static_cast<uint64_t>(N) >> 32); break;
+      case 4: w = static_cast<uint32_t>(K); break;
+      case 5: w = static_cast<uint32_t>(static_cast<uint64_t>(K) >> 32); break;
+      case 6: w = 128u; break;
+      case 7: w = static_cast<uint32_t>(kTileBytes); break;
+      case 8: w = static_cast<uint32_t>(s1_offset); break;
+      case 9: w = static_cast<uint32_t>(static_cast<uint64_t>(s1_offset) >> 32); break;
+      default: w = 0; break;
+    }
+    reinterpret_cast<uint32_t*>(blob)[threadIdx.x] = w;
+  }
+}
+
+}  // namespace w4a8

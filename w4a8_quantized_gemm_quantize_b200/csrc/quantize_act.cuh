@@ -1,0 +1,111 @@
+// Per-token symmetric int8 quantization of fp16 activations.
+//
+// Row m: amax = max_k |A|; sA = fp16_rn(amax / 127) (IEEE fp32 divide);
+// A8 = clamp(rint(A / float(sA)), -127, 127) (IEEE fp32 divide, rint half to
+// even); sA == 0 gives zero codes; rowsum = sum_k A8. This is the dynamic
+// per-token 8-bit activation scheme of W4A8 serving ("QServe/QoQ" abstract,
+// 8-bit activations; "PrefixQuant ...", Key Findings: per-token dynamic
+// quantization).
+//
+// HBM-bound (2 bytes read + 1 byte written per element). One CTA per row;
+// each thread keeps its slice of the row in registers (16-byte vectors), so
+// the row is read from HBM once, reduced, then quantized from registers.
+#pragma once
+#include "ptx.cuh"
+
+namespace w4a8 {
+
+template <int THREADS>
+__device__ __forceinline__ float block_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < THREADS / 32 ? red[lane] : 0.0f;
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  v = red[0];
+  __syncthreads();
+  return v;
+}
+
+template <int THREADS>
+__device__ __forceinline__ int block_sum(int v, int* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < THREADS / 32 ? red[lane] : 0;
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[0] = v;
+  }
+  __syncthreads();
+  return red[0];
+}
+
+__device__ __forceinline__ int quant_one(float x, float sf) {
+  int q = __float2int_rn(__fdiv_rn(x, sf));
+  return max(-127, min(127, q));
+}
+
+// VPT: 16-byte vectors (8 halves) per thread; K <= THREADS * VPT * 8.
+template <int THREADS, int VPT>
+__global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __restrict__ A, int64_t K,
+                                                                int8_t* __restrict__ A8, __half* __restrict__ sA,
+                                                                int32_t* __restrict__ rowsum) {
+  __shared__ float fred[32];
+  __shared__ int ired[32];
+  const int64_t m = blockIdx.x;
+  const uint4* row = reinterpret_cast<const uint4*>(A + m * K);
+  const int nvec = static_cast<int>(K >> 3);
+  uint4 v[VPT];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * THREADS;
+    if (idx < nvec) {
+      v[i] = __ldcs(row + idx);  // streamed once
+      const __half2* h = reinterpret_cast<const __half2*>(&v[i]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+  }
+  amax = block_max<THREADS>(amax, fred);
+  const __half s_h = __float2half_rn(__fdiv_rn(amax, 127.0f));
+  const float sf = __half2float(s_h);
+  int local = 0;
+  uint2* out = reinterpret_cast<uint2*>(A8 + m * K);
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * THREADS;
+    if (idx < nvec) {
+      const __half2* h = reinterpret_cast<const __half2*>(&v[i]);
+      uint32_t packed[2] = {0u, 0u};
+      if (sf != 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __half22float2(h[j]);
+          const int q0 = quant_one(f.x, sf), q1 = quant_one(f.y, sf);
+          local += q0 + q1;
+          packed[j >> 1] |= ((static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8))
+                            << ((j & 1) * 16);
+        }
+      }
+      out[idx] = make_uint2(packed[0], packed[1]);
+    }
+  }
+  if (rowsum != nullptr) {
+    const int total = block_sum<THREADS>(local, ired);
+    if (threadIdx.x == 0) rowsum[m] = total;
+  }
+  if (threadIdx.x == 0) sA[m] = s_h;
+}
+
+}  // namespace w4a8

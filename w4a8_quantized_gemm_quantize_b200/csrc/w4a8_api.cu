@@ -1,0 +1,320 @@
+// C ABI of the W4A8 library: argument validation, schedule selection, tensor
+// map encoding and kernel launches. Declarations and the contract of every
+// entry point are in include/w4a8.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <mutex>
+
+#include "gemm.cuh"
+#include "pack.cuh"
+#include "quantize_act.cuh"
+#include "quantize_weights.cuh"
+#include "w4a8.h"
+
+namespace w4a8 {
+
+__device__ int g_device_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int64_t kMaxK = 65536;
+
+struct DeviceInfo {
+  bool ready = false;
+  int sms = 0;
+  int* err = nullptr;  // device address of g_device_error
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+w4a8_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return W4A8_OK;
+  (void)cudaGetLastError();
+  return W4A8_ERR_CUDA;
+}
+
+w4a8_status_t launch_status() { return cuda_status(cudaGetLastError()); }
+
+// Per-device facts, fetched once with that device current.
+w4a8_status_t device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cuda_status(cudaErrorInvalidDevice);
+  if (dev < 0 || dev >= kMaxDevices) return W4A8_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return launch_status();
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return launch_status();
+    d.err = static_cast<int*>(p);
+    if (g_encode == nullptr) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || fn == nullptr)
+        return launch_status();
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+    }
+    d.ready = true;
+  }
+  *out = &d;
+  return W4A8_OK;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int64_t packed_s1_offset(int64_t N, int64_t K) { return kHeaderBytes + (N / kTileN) * (K / kTileK) * kTileBytes; }
+
+// ------------------------------------------------------------------ GEMM
+template <class C>
+w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs args, int grid,
+                              cudaStream_t stream) {
+  static bool attr_done[kMaxDevices] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!attr_done[dev]) {
+    if (cudaFuncSetAttribute(w4a8_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return launch_status();
+    attr_done[dev] = true;
+  }
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(C::BN)};
+  const cuuint32_t estr[2] = {1u, 1u};
+  if (g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(A8), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return W4A8_ERR_CUDA;
+  w4a8_gemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, args);
+  return launch_status();
+}
+
+// Tile configurations: tokens per tile, shared-memory stages, TMEM weight
+// stages, accumulator buffers.
+using Cfg16 = GemmCfg<16, 12, 8, 2>;
+using Cfg32 = GemmCfg<32, 12, 8, 2>;
+using Cfg64 = GemmCfg<64, 10, 8, 2>;
+using Cfg128 = GemmCfg<128, 8, 8, 2>;
+
+size_t ws_counter_bytes(int64_t M, int64_t N) {
+  const int64_t tiles = (N / kTileN) * ((M + 15) / 16);  // the most tiles any block_m gives
+  return static_cast<size_t>((tiles * 4 + 255) / 256 * 256);
+}
+
+}  // namespace
+
+w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
+                        void* Y, int32_t* acc, void* ws, size_t ws_bytes, const w4a8_gemm_opts_t* opts,
+                        cudaStream_t stream) {
+  w4a8_gemm_opts_t o = {0, 0, 0, 0};
+  if (opts != nullptr) o = *opts;
+  if (o.reserved != 0 || o.schedule < 0 || o.schedule > 2 || o.max_ctas < 0) return W4A8_ERR_INVALID_ARG;
+  if (!(o.block_m == 0 || o.block_m == 16 || o.block_m == 32 || o.block_m == 64 || o.block_m == 128))
+    return W4A8_ERR_INVALID_ARG;
+  if (M < 0 || N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if ((Y == nullptr) == (acc == nullptr)) return W4A8_ERR_INVALID_ARG;
+  if (K == 0 || K % kTileK != 0 || K > kMaxK || N % kTileN != 0) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M > INT32_MAX || N > INT32_MAX || (N > 0 && M > (int64_t(1) << 62) / N)) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0 || N == 0) return W4A8_OK;
+  if (A8 == nullptr || packed == nullptr || (acc == nullptr && sA == nullptr)) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(A8, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(acc, 16) || !aligned(sA, 2) ||
+      !aligned(ws, 256))
+    return W4A8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  w4a8_status_t st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+
+  int bn = o.block_m;
+  if (bn == 0) bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  const int n_tiles = static_cast<int>(N / kTileN);
+  const int m_tiles = static_cast<int>((M + bn - 1) / bn);
+  const int64_t num_tiles64 = static_cast<int64_t>(n_tiles) * m_tiles;
+  if (num_tiles64 > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  const int num_tiles = static_cast<int>(num_tiles64);
+  const int KB = static_cast<int>(K / kTileK);
+  int max_ctas = dev->sms;
+  if (o.max_ctas > 0 && o.max_ctas < max_ctas) max_ctas = o.max_ctas;
+
+  const size_t need_ws = ws_counter_bytes(M, N) + static_cast<size_t>(M) * N * 4;
+  const bool ws_ok = ws != nullptr && ws_bytes >= need_ws;
+  int stream_k;
+  if (o.schedule == 2) {
+    if (!ws_ok) return W4A8_ERR_WORKSPACE;
+    stream_k = 1;
+  } else if (o.schedule == 1) {
+    stream_k = 0;
+  } else {
+    // whole tiles once there are enough of them to fill the machine twice
+    stream_k = (ws_ok && num_tiles < 2 * max_ctas) ? 1 : 0;
+  }
+  int grid;
+  if (stream_k) {
+    const int64_t units = static_cast<int64_t>(num_tiles) * KB;
+    grid = static_cast<int>(units < max_ctas ? units : max_ctas);
+  } else {
+    grid = num_tiles < max_ctas ? num_tiles : max_ctas;
+  }
+
+  GemmArgs a;
+  a.tiles = static_cast<const uint8_t*>(packed) + kHeaderBytes;
+  a.s1 = reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + packed_s1_offset(N, K));
+  a.sA = static_cast<const __half*>(sA);
+  a.Y = static_cast<__half*>(Y);
+  a.acc_out = acc;
+  a.ws_cnt = stream_k ? static_cast<int32_t*>(ws) : nullptr;
+  a.ws_acc = stream_k ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_counter_bytes(M, N)) : nullptr;
+  a.err = dev->err;
+  a.M = static_cast<int>(M);
+  a.N = static_cast<int>(N);
+  a.KB = KB;
+  a.m_tiles = m_tiles;
+  a.num_tiles = num_tiles;
+  a.stream_k = stream_k;
+  switch (bn) {
+    case 16: return launch_gemm_cfg<Cfg16>(A8, M, K, a, grid, stream);
+    case 32: return launch_gemm_cfg<Cfg32>(A8, M, K, a, grid, stream);
+    case 64: return launch_gemm_cfg<Cfg64>(A8, M, K, a, grid, stream);
+    default: return launch_gemm_cfg<Cfg128>(A8, M, K, a, grid, stream);
+  }
+}
+
+}  // namespace w4a8
+
+using namespace w4a8;
+
+extern "C" {
+
+const char* w4a8_status_string(int status) {
+  switch (status) {
+    case W4A8_OK: return "W4A8_OK";
+    case W4A8_ERR_INVALID_ARG: return "W4A8_ERR_INVALID_ARG";
+    case W4A8_ERR_UNSUPPORTED_SHAPE: return "W4A8_ERR_UNSUPPORTED_SHAPE";
+    case W4A8_ERR_MISALIGNED: return "W4A8_ERR_MISALIGNED";
+    case W4A8_ERR_WORKSPACE: return "W4A8_ERR_WORKSPACE";
+    case W4A8_ERR_CUDA: return "W4A8_ERR_CUDA";
+    case W4A8_ERR_DEVICE: return "W4A8_ERR_DEVICE";
+    default: return "W4A8_ERR_UNKNOWN";
+  }
+}
+
+int w4a8_version(void) { return 100; }
+
+w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, int8_t* A8, void* sA, int32_t* rowsum,
+                                w4a8_stream_t stream) {
+  if (M < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if (K == 0 || K % 8 != 0 || K > kMaxK || M > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return W4A8_OK;
+  if (A == nullptr || A8 == nullptr || sA == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(A8, 16) || !aligned(sA, 2) || !aligned(rowsum, 4)) return W4A8_ERR_MISALIGNED;
+  const __half* a = static_cast<const __half*>(A);
+  __half* s = static_cast<__half*>(sA);
+  const int grid = static_cast<int>(M);
+  const int64_t nvec = K / 8;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (nvec <= 128) quantize_act_kernel<128, 1><<<grid, 128, 0, st>>>(a, K, A8, s, rowsum);
+  else if (nvec <= 256) quantize_act_kernel<256, 1><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
+  else if (nvec <= 512) quantize_act_kernel<256, 2><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
+  else if (nvec <= 1024) quantize_act_kernel<256, 4><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
+  else if (nvec <= 2048) quantize_act_kernel<256, 8><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
+  else if (nvec <= 4096) quantize_act_kernel<512, 8><<<grid, 512, 0, st>>>(a, K, A8, s, rowsum);
+  else quantize_act_kernel<1024, 8><<<grid, 1024, 0, st>>>(a, K, A8, s, rowsum);
+  return launch_status();
+}
+
+w4a8_status_t w4a8_quantize_weights(const float* W, int64_t N, int64_t K, int32_t group, uint8_t* q, uint8_t* z,
+                                    uint8_t* s2, void* s1, w4a8_stream_t stream) {
+  if (N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if (group != 128 || K == 0 || K % 128 != 0 || K > kMaxK || N > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (N == 0) return W4A8_OK;
+  if (W == nullptr || q == nullptr || z == nullptr || s2 == nullptr || s1 == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(W, 16) || !aligned(q, 16) || !aligned(s1, 2)) return W4A8_ERR_MISALIGNED;
+  quantize_weights_kernel<256><<<static_cast<int>(N), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      W, K, q, z, s2, static_cast<__half*>(s1));
+  return launch_status();
+}
+
+size_t w4a8_packed_bytes(int64_t N, int64_t K, int32_t group) {
+  if (group != 128 || N <= 0 || K <= 0 || N % 128 != 0 || K % 128 != 0 || K > kMaxK) return 0;
+  return static_cast<size_t>(packed_s1_offset(N, K) + (2 * N + 15) / 16 * 16);
+}
+
+w4a8_status_t w4a8_pack_weights(const uint8_t* q, const uint8_t* z, const uint8_t* s2, const void* s1, int64_t N,
+                                int64_t K, int32_t group, void* packed, size_t packed_bytes,
+                                w4a8_stream_t stream) {
+  if (N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if (group != 128 || N == 0 || K == 0 || N % 128 != 0 || K % 128 != 0 || K > kMaxK)
+    return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (q == nullptr || z == nullptr || s2 == nullptr || s1 == nullptr || packed == nullptr)
+    return W4A8_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(s1, 2) || !aligned(packed, 16)) return W4A8_ERR_MISALIGNED;
+  if (packed_bytes < w4a8_packed_bytes(N, K, group)) return W4A8_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* blob = static_cast<uint8_t*>(packed);
+  const int64_t chunks = N * (K / 32);
+  const int64_t blocks1 = (chunks + 255) / 256;
+  pack_codes_kernel<<<static_cast<int>(blocks1 < 65535 * 16 ? blocks1 : 65535 * 16), 256, 0, st>>>(
+      q, N, K, blob + kHeaderBytes);
+  if (cudaPeekAtLastError() != cudaSuccess) return launch_status();
+  const int64_t metas = N * (K / 128);
+  const int64_t blocks2 = (metas + 255) / 256;
+  pack_meta_kernel<<<static_cast<int>(blocks2 < 65535 ? blocks2 : 65535), 256, 0, st>>>(
+      z, s2, static_cast<const __half*>(s1), N, K, blob, packed_s1_offset(N, K));
+  return launch_status();
+}
+
+size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  (void)K;
+  if (M <= 0 || N <= 0) return 0;
+  return ws_counter_bytes(M, N) + static_cast<size_t>(M) * N * 4;
+}
+
+w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
+                        void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
+  if (Y == nullptr) return W4A8_ERR_INVALID_ARG;
+  return gemm_impl(A8, sA, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const void* packed, int64_t M, int64_t N, int64_t K,
+                                  int32_t* acc, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
+  if (acc == nullptr) return W4A8_ERR_INVALID_ARG;
+  return gemm_impl(A8, nullptr, packed, M, N, K, nullptr, acc, workspace, workspace_bytes, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
+                           void* Y, int32_t* acc, void* workspace, size_t workspace_bytes,
+                           const w4a8_gemm_opts_t* opts, w4a8_stream_t stream) {
+  return gemm_impl(A8, sA, packed, M, N, K, Y, acc, workspace, workspace_bytes, opts,
+                   reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4a8_status_t w4a8_get_device_error(w4a8_stream_t stream, int32_t* code) {
+  if (code == nullptr) return W4A8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  w4a8_status_t st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return launch_status();
+  int v = 0;
+  if (cudaMemcpy(&v, dev->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return launch_status();
+  *code = v;
+  return W4A8_OK;
+}
+
+w4a8_status_t w4a8_clear_device_error(w4a8_stream_t stream) {
+  DeviceInfo* dev = nullptr;
+  w4a8_status_t st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+  return cuda_status(cudaMemsetAsync(dev->err, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"
