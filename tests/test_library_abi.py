@@ -111,6 +111,8 @@ def test_gemm_validation(L):
     assert ex(FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
     both = FAKE
     assert ex(FAKE, FAKE, FAKE, 4, 128, 256, FAKE, both, None, 0, None, None) == 1  # Y and acc
+    assert L.w4a8_gemm_debug_acc(FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1  # no acc
+    assert ex(None, None, None, 0, 128, 256, None, None, None, 0, None, None) == 0   # M == 0
 
 
 def test_python_binding_refuses_cpu_tensors(L):

@@ -121,10 +121,10 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const void* packed, in
   if (!(o.block_m == 0 || o.block_m == 16 || o.block_m == 32 || o.block_m == 64 || o.block_m == 128))
     return W4A8_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
-  if ((Y == nullptr) == (acc == nullptr)) return W4A8_ERR_INVALID_ARG;
   if (K == 0 || K % kTileK != 0 || K > kMaxK || N % kTileN != 0) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M > INT32_MAX || N > INT32_MAX || (N > 0 && M > (int64_t(1) << 62) / N)) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0 || N == 0) return W4A8_OK;
+  if ((Y == nullptr) == (acc == nullptr)) return W4A8_ERR_INVALID_ARG;
   if (A8 == nullptr || packed == nullptr || (acc == nullptr && sA == nullptr)) return W4A8_ERR_INVALID_ARG;
   if (!aligned(A8, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(acc, 16) || !aligned(sA, 2) ||
       !aligned(ws, 256))
@@ -279,14 +279,12 @@ size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
 
 w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
                         void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
-  if (Y == nullptr) return W4A8_ERR_INVALID_ARG;
   return gemm_impl(A8, sA, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const void* packed, int64_t M, int64_t N, int64_t K,
                                   int32_t* acc, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
-  if (acc == nullptr) return W4A8_ERR_INVALID_ARG;
   return gemm_impl(A8, nullptr, packed, M, N, K, nullptr, acc, workspace, workspace_bytes, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
 }
