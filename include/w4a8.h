@@ -176,6 +176,37 @@ W4A8_API w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const void
                            const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
 
 /*
+ * Allocation-free GEMM: the same computation and results as w4a8_gemm, for
+ * callers that cannot hand the library a workspace. This entry point has no
+ * counterpart in the papers; it exists for deployment. Typical callers: a
+ * plugin or custom operator inside a host engine that plans all device
+ * memory itself and gives the operator no scratch buffer, or a serving loop
+ * that must not touch the device allocator once it has started.
+ *
+ * Instead of a caller-provided workspace it uses one scratch array compiled
+ * into the library (a file-scope __device__ array of
+ * W4A8_NOALLOC_SCRATCH_BYTES = 8 MiB, 256-byte aligned). Every GPU that
+ * loads the library holds that array until the process exits.
+ *  - Set-up: the first call on a device (with that device current) looks up
+ *    the array's device address with cudaGetSymbolAddress and caches it.
+ *    Make that first call before any stream capture on the device.
+ *  - Each call clears the part of the array it needs (cudaMemsetAsync on
+ *    `stream`) and then launches the GEMM; it calls no cudaMalloc, cudaFree
+ *    or other allocating routine.
+ *  - The array is shared by every call on a device and keeps the last call's
+ *    contents: calls whose GPU work overlaps in time (different streams
+ *    without ordering between them) race on it and give wrong results.
+ *  - Shapes whose scratch need, w4a8_gemm_workspace_bytes(M, N, K), exceeds
+ *    W4A8_NOALLOC_SCRATCH_BYTES are rejected with W4A8_ERR_WORKSPACE and
+ *    nothing is launched (every M <= 32 fits for N <= 49152; M = 64 fits for
+ *    N <= 32640; larger M or N may not).
+ * Arguments, layouts and the other limits are those of w4a8_gemm.
+ */
+#define W4A8_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+W4A8_API w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N,
+                                         int64_t K, void* Y, w4a8_stream_t stream);
+
+/*
  * Synchronizes `stream`, then stores the current device's error word in
  * *code (W4A8_DEVERR_*; 0 = no kernel gave up a wait). Returns W4A8_ERR_CUDA
  * if the synchronization itself fails. The word stays set until cleared.

@@ -18,7 +18,7 @@ import os
 __all__ = [
     "W4A8Error", "lib", "library_path", "EXPORTED_SYMBOLS", "status_string", "quantize_act",
     "quantize_weights", "packed_bytes", "pack_weights", "workspace_bytes", "Workspace", "gemm",
-    "gemm_debug_acc", "gemm_ex", "get_device_error", "clear_device_error",
+    "gemm_debug_acc", "gemm_ex", "gemm_noalloc", "get_device_error", "clear_device_error",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -28,6 +28,7 @@ EXPORTED_SYMBOLS = (
     "w4a8_status_string", "w4a8_version", "w4a8_quantize_act", "w4a8_quantize_weights",
     "w4a8_packed_bytes", "w4a8_pack_weights", "w4a8_gemm_workspace_bytes", "w4a8_gemm",
     "w4a8_gemm_debug_acc", "w4a8_gemm_ex", "w4a8_get_device_error", "w4a8_clear_device_error",
+    "w4a8_gemm_noalloc",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K = 0, 1, 2
@@ -69,6 +70,7 @@ def lib() -> ctypes.CDLL:
                                         ctypes.POINTER(GemmOpts), vp]),
         "w4a8_get_device_error": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_int32)]),
         "w4a8_clear_device_error": (ctypes.c_int, [vp]),
+        "w4a8_gemm_noalloc": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -236,6 +238,22 @@ def gemm_ex(A8, sA, blob, N: int, K: int, Y=None, acc=None, workspace=None, sche
     """GEMM with explicit scheduling overrides (for tests and tuning)."""
     _gemm_common(A8, sA, blob, N, K, Y, acc, workspace, (schedule, block_m, max_ctas, 0))
     return Y if Y is not None else acc
+
+
+NOALLOC_SCRATCH_BYTES = 8 << 20
+
+
+def gemm_noalloc(A8, sA, blob, N: int, K: int, out=None):
+    """The GEMM through the allocation-free entry point: the library's own
+    built-in scratch array replaces the workspace (see w4a8_gemm_noalloc in
+    include/w4a8.h), so no workspace is passed or allocated."""
+    torch = _torch()
+    _require_cuda(A8, sA, blob, out)
+    M = A8.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A8.device)
+    _check(lib().w4a8_gemm_noalloc(_ptr(A8), _ptr(sA), _ptr(blob), M, N, K, _ptr(Y), _stream(A8.device)),
+           "w4a8_gemm_noalloc")
+    return Y
 
 
 def get_device_error(device=None) -> int:

@@ -315,4 +315,36 @@ w4a8_status_t w4a8_clear_device_error(w4a8_stream_t stream) {
   return cuda_status(cudaMemsetAsync(dev->err, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// ------------------------------------------------- allocation-free GEMM
+// Scratch for w4a8_gemm_noalloc: a file-scope device array instead of a
+// caller workspace. In host code `g_noalloc_scratch` only names the symbol;
+// its device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_BYTES];
+static void* g_noalloc_addr[64] = {};
+static std::mutex g_noalloc_mu;
+
+w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N,
+                                int64_t K, void* Y, w4a8_stream_t stream) {
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (M <= 0 || N <= 0) return gemm_impl(A8, sA, packed, M, N, K, Y, nullptr, nullptr, 0, nullptr, st);
+  const size_t need = w4a8_gemm_workspace_bytes(M, N, K);
+  if (need > W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return cuda_status(cudaErrorInvalidDevice);
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_addr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return cuda_status(cudaErrorInvalidSymbol);
+      g_noalloc_addr[dev] = p;
+    }
+    scratch = g_noalloc_addr[dev];
+  }
+  // the split-k tickets and partial sums must start at zero
+  if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return launch_status();
+  return gemm_impl(A8, sA, packed, M, N, K, Y, nullptr, scratch, need, nullptr, st);
+}
+
 }  // extern "C"
