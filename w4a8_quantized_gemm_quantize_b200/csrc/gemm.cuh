@@ -10,29 +10,35 @@
 // elements, and weight load, dequantization and MMA overlapped in one
 // pipeline without software synchronization in the hot loop).
 //
-// Structure (one CTA per SM, persistent, 12 warps):
-//   warp 0      producer: per k-block, a TMA 2-D load of the int8 activation
-//               tile (BN tokens x 128 k, 128-byte swizzle) and a 1-D bulk
-//               copy of the packed weight tile (128 n x 128 k, 8320 bytes)
-//               into a STAGES-deep shared-memory ring.
-//   warps 4-7   dequantizers: thread r of the warpgroup owns weight row r; it
-//               reads its 64 code bytes as four 16-byte vectors and turns
-//               every four codes into four int8 weights with
+// Structure (persistent CTAs; warp roles):
+//   producer    one thread: per k-block, a TMA 2-D load of the int8
+//               activation tile (BN tokens x 128 k, 128-byte swizzle) and a
+//               1-D bulk copy of the packed weight tile (128 n x 128 k, 8320
+//               bytes) into a STAGES-deep shared-memory ring.
+//   dequant     four warps (one per TMEM lane quarter): thread r owns weight
+//               row r; it reads its 64 code bytes as four 16-byte vectors and
+//               turns every four codes into four int8 weights with
 //               ((w & 0x0F0F0F0F) * s2 + (128 - z*s2) * 0x01010101) ^ 0x80808080
 //               (each byte stays in [8, 248] before the xor, so no carry
 //               crosses a byte), then writes the 128 int8 weights of its row
 //               straight into tensor memory with tcgen05.st. The dequantized
 //               weights never touch shared memory (the point of the "QUICK"
 //               abstract's interleaving, reached here through TMEM).
-//   warp 1      MMA issuer (one thread): tcgen05.mma.kind::i8 with A = the
-//               dequantized weights in TMEM (M = 128 rows = n), B = the
-//               activation tile in shared memory (N = BN tokens), K = 32 per
-//               instruction; int32 accumulators in TMEM (two buffers).
-//   warps 8-11  epilogue: tcgen05.ld of the accumulators (lane = n, column =
-//               token), scale, fp16 store; or, for a partial k-range,
-//               red.add into an int32 workspace and a ticket counter whose
-//               last arriver finishes the tile (nobody spins on another CTA).
-//   warp 2      owns the TMEM allocation.
+//   MMA         one thread: tcgen05.mma.kind::i8 with A = the dequantized
+//               weights in TMEM (M = 128 rows = n), B = the activation tile in
+//               shared memory (N = BN tokens), K = 32 per instruction; int32
+//               accumulators in TMEM.
+//   epilogue    four warps: tcgen05.ld of the accumulators (lane = n,
+//               column = token), scale, fp16 store; or, for a partial
+//               k-range, red.add into an int32 workspace and a ticket counter
+//               whose last arriver finishes the tile (nobody spins on another
+//               CTA).
+// Two layouts: "compact" (6 warps; the dequant warps also run the epilogue;
+// 128 TMEM columns and ~50 KB of shared memory, so several CTAs share an SM
+// and hide each other's issue latencies, which dominate when the MMA is thin
+// as in decode) and "full" (12 warps, one CTA per SM, a separate epilogue
+// group and two accumulator buffers so a tile's epilogue overlaps the next
+// tile's mainloop).
 // The roles synchronize only through mbarriers; every wait is bounded in
 // time and reports through the device error word.
 //
@@ -67,7 +73,7 @@ struct Seg {
 
 // The same deterministic schedule is replayed by every role of a CTA.
 struct Sched {
-  int64_t u, u_end;
+  int64_t u, u_end, u_begin;
   int tile_it, KB, num_tiles, stream_k;
   __device__ __forceinline__ void init(const GemmArgs& a) {
     KB = a.KB;
@@ -77,8 +83,25 @@ struct Sched {
       const int64_t U = static_cast<int64_t>(num_tiles) * KB;
       u = U * blockIdx.x / gridDim.x;
       u_end = U * (blockIdx.x + 1) / gridDim.x;
+      u_begin = u;
     } else {
       tile_it = blockIdx.x;
+    }
+  }
+  // Total k-blocks of this CTA, and the (tile, k-block) of its it-th one.
+  __device__ __forceinline__ int total() const {
+    if (stream_k) return static_cast<int>(u_end - u_begin);
+    const int mine = blockIdx.x < num_tiles ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+    return mine * KB;
+  }
+  __device__ __forceinline__ void at(int it, int& tile, int& kb) const {
+    if (stream_k) {
+      const int64_t uu = u_begin + it;
+      tile = static_cast<int>(uu / KB);
+      kb = static_cast<int>(uu - static_cast<int64_t>(tile) * KB);
+    } else {
+      tile = static_cast<int>(blockIdx.x) + (it / KB) * static_cast<int>(gridDim.x);
+      kb = it % KB;
     }
   }
   __device__ __forceinline__ bool next(Seg& s) {
@@ -100,20 +123,47 @@ struct Sched {
   }
 };
 
-template <int BN_, int STAGES_, int TA_, int NACC_>
+template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_>
 struct GemmCfg {
-  static constexpr int BN = BN_, STAGES = STAGES_, TA = TA_, NACC = NACC_;
-  static constexpr int kThreads = 384;
-  static constexpr int kA8Bytes = BN * 128;
-  static constexpr int kWBytes = kTileBytes;  // 8320
+  static constexpr int BN = BN_, KS = KS_, NS = NS_, NT = NT_, DQ = DQ_, NACC = NACC_;
+  // One CTA per SM, persistent. Work moves in chunks of up to KS k-blocks of
+  // one tile (one weight copy, one wait and one commit per chunk amortize the
+  // fixed latencies of the synchronization operations).
+  //   warp 0        weight producer (one thread) and TMEM owner
+  //   warp 1        MMA issuer (one thread)
+  //   warp 3        activation producer (one thread)
+  //   warps 4..     DQ dequantizer warpgroups, chunk c goes to group c % DQ
+  //   last 4 warps  epilogue
+  // Three rings: weight slots (NS, freed as soon as the dequantizers have
+  // read them), activation slots (NS, freed when the chunk's MMAs finish)
+  // and TMEM weight slots (NT, KS x 32 columns each, freed likewise).
+  static constexpr int kDqWarp0 = 4;
+  static constexpr int kEpWarp0 = 4 + 4 * DQ;
+  static constexpr int kThreads = 32 * (4 + 4 * DQ + 4);
+  static constexpr int kA8Bytes = BN * 128;        // one k-block of activations
+  static constexpr int kASlot = KS * kA8Bytes;
+  static constexpr int kWSlot = KS * kTileBytes;   // KS consecutive packed tiles
   static constexpr int kTmemCols = 512;
-  static constexpr int kTmemA = NACC * BN;  // first column of the weight ring
-  static_assert(NACC * BN + TA * 32 <= kTmemCols, "tensor memory budget");
+  static constexpr int kTmemA = NACC * BN;         // accumulators first, then the TMEM weight ring
+  static constexpr int kTSlotCols = KS * 32;
+  static_assert(kTmemA + NT * kTSlotCols <= kTmemCols, "tensor memory budget");
+  static_assert(NT > DQ, "every dequantizer group needs a TMEM slot of its own");
+  // The MMA issuer waits for chunk c + 1 before it commits chunk c, so both
+  // rings need a second slot.
+  static_assert(NS >= 2 && NT >= 2, "two slots per ring at least");
+  // Several dequantizer groups wait on the weight ring out of order; bounding
+  // them by the TMEM ring keeps every parity wait within one phase.
+  static_assert(NS >= NT, "weight ring at least as deep as the TMEM ring");
+  // With enough TMEM slots a group keeps a chunk's TMEM stores in flight
+  // while it loads its next chunk (it publishes chunk c only when it starts
+  // chunk c + DQ, which must not need a slot that chunk c + 1 still holds);
+  // otherwise it completes them within the chunk.
+  static constexpr bool kPipelinedStores = NT >= 2 * DQ && NT >= DQ + 2;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
-  static constexpr int kOffA8 = 0;
-  static constexpr int kOffW = STAGES * kA8Bytes;
-  static constexpr int kOffBar = (kOffW + STAGES * kWBytes + 15) / 16 * 16;
-  static constexpr int kNumBars = 2 * STAGES + 2 * TA + 2 * NACC + 1;
+  static constexpr int kOffA8 = 0;                 // 1024-aligned activation slots
+  static constexpr int kOffW = NS * kASlot;        // 16-aligned weight slots
+  static constexpr int kOffBar = (kOffW + NS * kWSlot + 15) / 16 * 16;
+  static constexpr int kNumBars = 4 * NS + 2 * NT + 2 * NACC + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -127,21 +177,147 @@ enum : int {
   kErrDrain = 5,
 };
 
+// Dequantizes this thread's row r of a 128 x 128 weight tile in shared
+// memory into 32 registers: register c holds the int8 weights of
+// k = 4c .. 4c+3 (byte j = k 4c+j), the column order of the TMEM A operand.
+__device__ __forceinline__ void dequant_tile_regs(const uint8_t* wt, int r, uint32_t (&out)[32]) {
+  const uint32_t meta = wt[kTileCodeBytes + r];
+  const uint32_t zq = meta & 15u, s2 = (meta >> 4) + 1u;
+  const uint32_t bias = (128u - zq * s2) * 0x01010101u;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 v = *reinterpret_cast<const uint4*>(wt + (c * kTileN + r) * 16);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      out[c * 8 + 2 * jj] = ((w[jj] & 0x0F0F0F0Fu) * s2 + bias) ^ 0x80808080u;
+      out[c * 8 + 2 * jj + 1] = (((w[jj] >> 4) & 0x0F0F0F0Fu) * s2 + bias) ^ 0x80808080u;
+    }
+  }
+}
+
+// Epilogue of one segment for the four warps of an epilogue group (128
+// threads, named barrier 1). `tacc` is this warp's lane quarter at the
+// first lane's accumulator; lane j's accumulator is `lane_stride * j`
+// columns further; bit j of `lanes_used` says whether lane j holds a partial
+// sum for this segment. Returns false if the group has to abort.
+template <int BN>
+__device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg& sg, bool ok_in, uint64_t* accfull,
+                                                 uint32_t bph, uint64_t* accempty, uint32_t tacc,
+                                                 uint32_t lane_stride, uint32_t lanes_used, int quarter, int lane,
+                                                 volatile int* abort_flag, volatile int* epi_fail,
+                                                 volatile int* last_flag, DevErr err) {
+  // the four warps take one decision, so every named barrier below is
+  // reached by all of them
+  bool ok = ok_in && mbar_wait(accfull, bph, abort_flag, err, kErrEpilogue);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && lane == 0) *epi_fail = 1;
+  named_bar_sync(1, 128);
+  if (*epi_fail) return false;
+  tc_fence_after();
+  const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
+  const int64_t N = args.N;
+  const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
+  const int m0 = m_tile * BN;
+  const bool whole = (sg.kb0 == 0 && sg.kb1 == args.KB);
+  const float s1f = __half2float(args.s1[n]);
+#pragma unroll 1
+  for (int c = 0; c < BN; c += 16) {
+    uint32_t v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = 0;
+#pragma unroll 1
+    for (uint32_t l = 0, used = lanes_used; used != 0; ++l, used >>= 1) {
+      if (used & 1u) {
+        uint32_t u[16];
+        tmem_ld_16(tacc + l * lane_stride + c, u);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] += u[j];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      const int m = m0 + c + j;
+      if (m < args.M) {
+        const int32_t acc = static_cast<int32_t>(v[j]);
+        const int64_t o = static_cast<int64_t>(m) * N + n;
+        if (!whole) {
+          red_add_s32(args.ws_acc + o, acc);
+        } else if (args.acc_out != nullptr) {
+          args.acc_out[o] = acc;
+        } else {
+          const float scale = __fmul_rn(__half2float(args.sA[m]), s1f);
+          args.Y[o] = __float2half_rn(__fmul_rn(__int2float_rn(acc), scale));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(accempty);
+  if (!whole) {
+    // Partial k-range: publish with red.add, then one thread releases the
+    // group's writes and takes a ticket (bar.sync orders the other threads'
+    // writes before its gpu-scope fence). The CTA whose ticket completes the
+    // tile's k-blocks finishes the tile and restores the workspace to zero.
+    named_bar_sync(1, 128);
+    if (quarter == 0 && lane == 0) {
+      const int add = sg.kb1 - sg.kb0;
+      fence_acq_rel_gpu();
+      const int old = atom_add_relaxed_gpu(args.ws_cnt + sg.tile, add);
+      fence_acq_rel_gpu();
+      *last_flag = (old + add == args.KB) ? 1 : 0;
+    }
+    named_bar_sync(1, 128);
+    if (*last_flag) {
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 16) {
+        int32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + c + j;
+          v[j] = m < args.M ? __ldcg(args.ws_acc + static_cast<int64_t>(m) * N + n) : 0;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int m = m0 + c + j;
+          if (m < args.M) {
+            const int64_t o = static_cast<int64_t>(m) * N + n;
+            __stcg(args.ws_acc + o, 0);
+            if (args.acc_out != nullptr) {
+              args.acc_out[o] = v[j];
+            } else {
+              const float scale = __fmul_rn(__half2float(args.sA[m]), s1f);
+              args.Y[o] = __float2half_rn(__fmul_rn(__int2float_rn(v[j]), scale));
+            }
+          }
+        }
+      }
+      if (quarter == 0 && lane == 0) args.ws_cnt[sg.tile] = 0;
+    }
+    named_bar_sync(1, 128);
+  }
+  return true;
+}
+
 template <class C>
-__global__ void __launch_bounds__(384, 1) w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                                                           const GemmArgs args) {
-  constexpr int BN = C::BN, STAGES = C::STAGES, TA = C::TA, NACC = C::NACC;
+__global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+                                                                    const GemmArgs args) {
+  constexpr int BN = C::BN, KS = C::KS, NS = C::NS, NT = C::NT, DQ = C::DQ, NACC = C::NACC;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA8 = smem + C::kOffA8;
   uint8_t* sW = smem + C::kOffW;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
-  uint64_t* tempty = tfull + TA;
-  uint64_t* accfull = tempty + TA;
-  uint64_t* accempty = accfull + NACC;
-  uint64_t* done = accempty + NACC;
+  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + C::kOffBar);  // weight slot loaded
+  uint64_t* wempty = wfull + NS;                                     // weight slot read by the dequantizers
+  uint64_t* afull = wempty + NS;                                     // activation slot loaded
+  uint64_t* aempty = afull + NS;                                     // activation slot's MMAs finished
+  uint64_t* tfull = aempty + NS;                                     // TMEM weight slot written
+  uint64_t* tempty = tfull + NT;                                     // TMEM weight slot's MMAs finished
+  uint64_t* accfull = tempty + NT;                                   // a segment's MMAs finished
+  uint64_t* accempty = accfull + NACC;                               // epilogue has read the accumulator
+  uint64_t* done = accempty + NACC;                                  // all MMAs finished
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 2);
@@ -151,11 +327,13 @@ __global__ void __launch_bounds__(384, 1) w4a8_gemm_kernel(const __grid_constant
   const DevErr err{args.err};
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < STAGES; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
+    for (int i = 0; i < NS; ++i) {
+      mbar_init(&wfull[i], 1);
+      mbar_init(&wempty[i], 4);
+      mbar_init(&afull[i], 1);
+      mbar_init(&aempty[i], 1);
     }
-    for (int i = 0; i < TA; ++i) {
+    for (int i = 0; i < NT; ++i) {
       mbar_init(&tfull[i], 4);
       mbar_init(&tempty[i], 1);
     }
@@ -170,11 +348,11 @@ __global__ void __launch_bounds__(384, 1) w4a8_gemm_kernel(const __grid_constant
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if (warp == 2) {
+  if (warp == 0) {
     tmem_alloc(&misc[0], C::kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_a);
+  if (warp == 3 && lane == 0) prefetch_tensormap(&tmap_a);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -185,198 +363,184 @@ __global__ void __launch_bounds__(384, 1) w4a8_gemm_kernel(const __grid_constant
   Seg sg;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ----------------------------------------------------- weight producer
+    // The weights do not come from the preceding kernel, so they start
+    // streaming before the dependency wait. One copy per chunk: the packed
+    // tiles of consecutive k-blocks of a tile are contiguous.
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
-      int it = 0;
+      int c = 0;
       bool ok = true;
       while (ok && sch.next(sg)) {
-        const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
-        const uint8_t* wsrc = args.tiles + static_cast<int64_t>(n_tile) * args.KB * kTileBytes;
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, err, kErrProducer)) {
+        const uint8_t* wsrc = args.tiles + static_cast<int64_t>(sg.tile / args.m_tiles) * args.KB * kTileBytes;
+        for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
+          const int cnt = min(KS, sg.kb1 - kb);
+          const int w = c % NS;
+          if (!mbar_wait(&wempty[w], ((c / NS) & 1) ^ 1, abort_flag, err, kErrProducer)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[s], C::kA8Bytes + C::kWBytes);
-          tma_load_2d(sA8 + s * C::kA8Bytes, &tmap_a, &full[s], kb * 128, m_tile * BN);
-          bulk_load(sW + s * C::kWBytes, wsrc + static_cast<int64_t>(kb) * kTileBytes, C::kWBytes, &full[s],
+          mbar_arrive_expect_tx(&wfull[w], cnt * kTileBytes);
+          bulk_load(sW + w * C::kWSlot, wsrc + static_cast<int64_t>(kb) * kTileBytes, cnt * kTileBytes, &wfull[w],
                     pol_w);
         }
       }
-      // Copies still in flight must land before the CTA may exit.
-      const int first = it - STAGES > 0 ? it - STAGES : 0;
-      for (int i = first; i < it; ++i) mbar_wait(&full[i % STAGES], (i / STAGES) & 1, nullptr, err, kErrDrain);
+      // copies still in flight must land before the CTA exits
+      const int first = c - NS > 0 ? c - NS : 0;
+      for (int i = first; i < c; ++i) mbar_wait(&wfull[i % NS], (i / NS) & 1, nullptr, err, kErrDrain);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
+  } else if (warp == 3) {
+    // ------------------------------------------------- activation producer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_i8(128, BN);
-      int it = 0, seg_i = 0;
+      grid_dependency_wait();  // the activation tiles come from the preceding kernel
+      int c = 0;
       bool ok = true;
       while (ok && sch.next(sg)) {
-        const int b = seg_i % NACC;
-        const uint32_t bph = (seg_i / NACC) & 1;
-        if (!mbar_wait(&accempty[b], bph ^ 1, abort_flag, err, kErrMma)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + b * BN;
-        for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
-          const int s = it % STAGES, a = it % TA;
-          const uint32_t ph = (it / STAGES) & 1, aph = (it / TA) & 1;
-          if (!mbar_wait(&full[s], ph, abort_flag, err, kErrMma) ||
-              !mbar_wait(&tfull[a], aph, abort_flag, err, kErrMma)) {
+        const int m0 = (sg.tile % args.m_tiles) * BN;
+        for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
+          const int cnt = min(KS, sg.kb1 - kb);
+          const int a = c % NS;
+          if (!mbar_wait(&aempty[a], ((c / NS) & 1) ^ 1, abort_flag, err, kErrProducer)) {
             ok = false;
             break;
           }
-          tc_fence_after();
-          const uint32_t a_tmem = tmem + C::kTmemA + a * 32;
-          const uint32_t b_addr = smem_u32(sA8 + s * C::kA8Bytes);
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            mma_i8_ts(d_tmem, a_tmem + kk * 8, smem_desc_k128_sw128(b_addr + kk * 32), idesc,
-                      (kb > sg.kb0 || kk > 0) ? 1u : 0u);
+          mbar_arrive_expect_tx(&afull[a], cnt * C::kA8Bytes);
+          for (int j = 0; j < cnt; ++j)
+            tma_load_2d(sA8 + a * C::kASlot + j * C::kA8Bytes, &tmap_a, &afull[a], (kb + j) * 128, m0);
+        }
+      }
+      const int first = c - NS > 0 ? c - NS : 0;
+      for (int i = first; i < c; ++i) mbar_wait(&afull[i % NS], (i / NS) & 1, nullptr, err, kErrDrain);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8(128, BN);
+      int c = 0, seg_i = 0;
+      bool ok = true;
+      while (ok && sch.next(sg)) {
+        const int b = seg_i % NACC;
+        if (!mbar_wait(&accempty[b], ((seg_i / NACC) & 1) ^ 1, abort_flag, err, kErrMma)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem + b * BN;
+        // The waits for chunk c + 1 are done while chunk c's last MMAs are
+        // still executing (the tensor core queue is shallow, so a wait done
+        // between chunks would leave it idle).
+        bool ready = mbar_wait(&tfull[c % NT], (c / NT) & 1, abort_flag, err, kErrMma) &&
+                     mbar_wait(&afull[c % NS], (c / NS) & 1, abort_flag, err, kErrMma);
+        for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
+          if (!ready) {
+            ok = false;
+            break;
           }
-          mma_commit(&empty[s]);
-          mma_commit(&tempty[a]);
+          const int cnt = min(KS, sg.kb1 - kb);
+          const int a = c % NS, t = c % NT;
+          const bool has_next = kb + KS < sg.kb1;
+          tc_fence_after();
+          const uint32_t a_tmem = tmem + C::kTmemA + t * C::kTSlotCols;
+          const uint32_t b_addr = smem_u32(sA8 + a * C::kASlot);
+          for (int j = 0; j < cnt; ++j) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              if (j == cnt - 1 && kk == 3 && has_next) {
+                ready = mbar_wait(&tfull[(c + 1) % NT], ((c + 1) / NT) & 1, abort_flag, err, kErrMma) &&
+                        mbar_wait(&afull[(c + 1) % NS], ((c + 1) / NS) & 1, abort_flag, err, kErrMma);
+              }
+              mma_i8_ts(d_tmem, a_tmem + j * 32 + kk * 8,
+                        smem_desc_k128_sw128(b_addr + j * C::kA8Bytes + kk * 32), idesc,
+                        (kb + j > sg.kb0 || kk > 0) ? 1u : 0u);
+            }
+          }
+          mma_commit(&aempty[a]);
+          mma_commit(&tempty[t]);
         }
         if (!ok) break;
         mma_commit(&accfull[b]);
         ++seg_i;
       }
+      // the next kernel in the stream may start its prologue now
+      grid_launch_dependents();
       // every issued MMA must finish before TMEM is released
       mma_commit(done);
       mbar_wait(done, 0, nullptr, err, kErrDrain);
     }
     __syncwarp();
-  } else if (warp >= 4 && warp < 8) {
-    // --------------------------------------------------------- dequantizer
-    const int qd = warp - 4;  // TMEM lane quarter
-    const int r = qd * 32 + lane;
-    const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
-    int it = 0;
+  } else if (warp >= C::kDqWarp0 && warp < C::kDqWarp0 + 4 * DQ) {
+    // --------------------------------------------------------- dequantizers
+    // Group g takes chunks c = g (mod DQ). The weight slot is released as
+    // soon as it has been read; the TMEM stores of a chunk stay in flight
+    // while the group loads and unpacks its next chunk.
+    const int g = (warp - C::kDqWarp0) >> 2;
+    const int quarter = warp & 3;  // TMEM lane quarter this warp may access
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    int c = 0, prev_t = -1;
     bool ok = true;
     while (ok && sch.next(sg)) {
-      for (int kb = sg.kb0; kb < sg.kb1; ++kb, ++it) {
-        const int s = it % STAGES, a = it % TA;
-        const uint32_t ph = (it / STAGES) & 1, aph = (it / TA) & 1;
-        bool w_ok = mbar_wait(&full[s], ph, abort_flag, err, kErrDequant) &&
-                    mbar_wait(&tempty[a], aph ^ 1, abort_flag, err, kErrDequant);
-        w_ok = __all_sync(0xffffffffu, w_ok);
-        if (!w_ok) {
+      for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
+        if (c % DQ != g) continue;
+        const int cnt = min(KS, sg.kb1 - kb);
+        const int w = c % NS, t = c % NT;
+        // TMEM slot first: once the MMAs of chunk c - NT are done, every
+        // chunk up to c - NT has been loaded, so (NS >= NT) the weight slot's
+        // barrier is at most one phase behind and its parity wait cannot
+        // alias an older phase, however far the other groups lag.
+        if (!__all_sync(0xffffffffu, mbar_wait(&tempty[t], ((c / NT) & 1) ^ 1, abort_flag, err, kErrDequant) &&
+                                         mbar_wait(&wfull[w], (c / NS) & 1, abort_flag, err, kErrDequant))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint8_t* wt = sW + s * C::kWBytes;
-        const uint32_t meta = wt[kTileCodeBytes + r];
-        const uint32_t zq = meta & 15u, s2 = (meta >> 4) + 1u;
-        const uint32_t bias = (128u - zq * s2) * 0x01010101u;
-        uint32_t out[32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 v = *reinterpret_cast<const uint4*>(wt + (c * kTileN + r) * 16);
-          const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            out[c * 8 + 2 * jj] = ((w[jj] & 0x0F0F0F0Fu) * s2 + bias) ^ 0x80808080u;
-            out[c * 8 + 2 * jj + 1] = (((w[jj] >> 4) & 0x0F0F0F0Fu) * s2 + bias) ^ 0x80808080u;
+        for (int j = 0; j < cnt; ++j) {
+          uint32_t out[32];
+          dequant_tile_regs(sW + w * C::kWSlot + j * kTileBytes, r, out);
+          if (C::kPipelinedStores && j == 0 && prev_t >= 0) {
+            // the previous chunk's stores are done once these ones may start
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tfull[prev_t]);
           }
+          tmem_st_32(tmem + C::kTmemA + t * C::kTSlotCols + j * 32 + lane_base, out);
         }
-        tmem_st_32(tmem + C::kTmemA + a * 32 + lane_base, out);
-        tmem_wait_st();
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&tfull[a]);
+        if (lane == 0) mbar_arrive(&wempty[w]);
+        if (C::kPipelinedStores) {
+          prev_t = t;
+        } else {
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tfull[t]);
+        }
       }
     }
-  } else if (warp >= 8) {
-    // ------------------------------------------------------------ epilogue
-    const int qe = warp - 8;
-    const uint32_t lane_base = static_cast<uint32_t>(qe * 32) << 16;
-    const int64_t N = args.N;
-    int seg_i = 0;
-    bool ok = true;
-    while (ok && sch.next(sg)) {
-      const int b = seg_i % NACC;
-      const uint32_t bph = (seg_i / NACC) & 1;
-      // the four epilogue warps take one decision, so their named barriers
-      // below are always reached by all of them
-      ok = __all_sync(0xffffffffu, mbar_wait(&accfull[b], bph, abort_flag, err, kErrEpilogue));
-      if (!ok && lane == 0) *epi_fail = 1;
-      named_bar_sync(1, 128);
-      ok = *epi_fail == 0;
-      if (!ok) break;
-      tc_fence_after();
-      const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
-      const int64_t n = static_cast<int64_t>(n_tile) * kTileN + qe * 32 + lane;
-      const int m0 = m_tile * BN;
-      const bool whole = (sg.kb0 == 0 && sg.kb1 == args.KB);
-      const float s1f = __half2float(args.s1[n]);
-      const uint32_t tb = tmem + b * BN + lane_base;
-#pragma unroll 1
-      for (int c = 0; c < BN; c += 16) {
-        uint32_t v[16];
-        tmem_ld_16(tb + c, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int m = m0 + c + j;
-          if (m < args.M) {
-            const int32_t acc = static_cast<int32_t>(v[j]);
-            const int64_t o = static_cast<int64_t>(m) * N + n;
-            if (!whole) {
-              red_add_s32(args.ws_acc + o, acc);
-            } else if (args.acc_out != nullptr) {
-              args.acc_out[o] = acc;
-            } else {
-              const float scale = __fmul_rn(__half2float(args.sA[m]), s1f);
-              args.Y[o] = __float2half_rn(__fmul_rn(__int2float_rn(acc), scale));
-            }
-          }
-        }
-      }
+    tmem_wait_st();
+    if (prev_t >= 0) {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[b]);
-      if (!whole) {
-        // partial k-range: publish, take a ticket; the CTA that completes the
-        // tile's k-blocks finishes it and restores the workspace to zero
-        __threadfence();
-        named_bar_sync(1, 128);
-        if (qe == 0 && lane == 0) {
-          const int add = sg.kb1 - sg.kb0;
-          const int old = atomicAdd(args.ws_cnt + sg.tile, add);
-          *last_flag = (old + add == args.KB) ? 1 : 0;
-        }
-        named_bar_sync(1, 128);
-        if (*last_flag) {
-          __threadfence();
-          const int mend = min(m0 + BN, args.M);
-          for (int m = m0; m < mend; ++m) {
-            const int64_t o = static_cast<int64_t>(m) * N + n;
-            const int32_t acc = __ldcg(args.ws_acc + o);
-            __stcg(args.ws_acc + o, 0);
-            if (args.acc_out != nullptr) {
-              args.acc_out[o] = acc;
-            } else {
-              const float scale = __fmul_rn(__half2float(args.sA[m]), s1f);
-              args.Y[o] = __float2half_rn(__fmul_rn(__int2float_rn(acc), scale));
-            }
-          }
-          if (qe == 0 && lane == 0) args.ws_cnt[sg.tile] = 0;
-        }
-        named_bar_sync(1, 128);
-      }
+      if (lane == 0) mbar_arrive(&tfull[prev_t]);
+    }
+  } else if (warp >= C::kEpWarp0 && warp < C::kEpWarp0 + 4) {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;
+    const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    int seg_i = 0;
+    while (sch.next(sg)) {
+      const int b = seg_i % NACC;
+      if (!epilogue_segment<BN>(args, sg, true, &accfull[b], (seg_i / NACC) & 1, &accempty[b],
+                                tmem + b * BN + lane_base, 0, 1u, quarter, lane, abort_flag, epi_fail, last_flag,
+                                err))
+        break;
       ++seg_i;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 2) {
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmemCols);
   }

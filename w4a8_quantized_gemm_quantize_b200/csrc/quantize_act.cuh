@@ -58,7 +58,12 @@ __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __r
                                                                 int8_t* __restrict__ A8, __half* __restrict__ sA,
                                                                 int32_t* __restrict__ rowsum) {
   __shared__ float fred[32];
-  __shared__ int ired[32];
+  __shared__ int ird[32];
+  // launched as a programmatic dependent: wait for the preceding kernel's
+  // writes, then let the next kernel (the GEMM) start its prologue
+  grid_dependency_wait();
+  grid_launch_dependents();
+  int* ired = ird;
   const int64_t m = blockIdx.x;
   const uint4* row = reinterpret_cast<const uint4*>(A + m * K);
   const int nvec = static_cast<int>(K >> 3);

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <utility>
 
 #include "gemm.cuh"
 #include "pack.cuh"
@@ -68,23 +69,53 @@ w4a8_status_t device_info(DeviceInfo** out) {
   return W4A8_OK;
 }
 
+// Launches with programmatic stream serialization: the kernel may start
+// while its predecessor in the stream finishes; it waits (griddepcontrol)
+// before touching anything the predecessor writes.
+template <typename... KArgs, typename... Args>
+w4a8_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                         Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cuda_status(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
+}
+
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int64_t packed_s1_offset(int64_t N, int64_t K) { return kHeaderBytes + (N / kTileN) * (K / kTileK) * kTileBytes; }
 
 // ------------------------------------------------------------------ GEMM
+// Resident CTAs per SM of a configuration (shared memory, threads and tensor
+// memory permitting), computed once per device.
 template <class C>
-w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs args, int grid,
-                              cudaStream_t stream) {
-  static bool attr_done[kMaxDevices] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!attr_done[dev]) {
+w4a8_status_t ctas_per_sm(int dev, int* out) {
+  static int cache[kMaxDevices] = {};
+  if (cache[dev] == 0) {
     if (cudaFuncSetAttribute(w4a8_gemm_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
       return launch_status();
-    attr_done[dev] = true;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, w4a8_gemm_kernel<C>, C::kThreads, C::kSmemBytes) !=
+        cudaSuccess)
+      return launch_status();
+    n = n < 512 / C::kTmemCols ? n : 512 / C::kTmemCols;  // every resident CTA must get its TMEM (one)
+    cache[dev] = n > 0 ? n : 1;
   }
+  *out = cache[dev];
+  return W4A8_OK;
+}
+
+template <class C>
+w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs args, int grid,
+                              cudaStream_t stream) {
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
@@ -94,16 +125,16 @@ w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs a
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return W4A8_ERR_CUDA;
-  w4a8_gemm_kernel<C><<<grid, C::kThreads, C::kSmemBytes, stream>>>(map, args);
-  return launch_status();
+  return launch_pdl(w4a8_gemm_kernel<C>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, map, args);
 }
 
-// Tile configurations: tokens per tile, shared-memory stages, TMEM weight
-// stages, accumulator buffers.
-using Cfg16 = GemmCfg<16, 12, 8, 2>;
-using Cfg32 = GemmCfg<32, 12, 8, 2>;
-using Cfg64 = GemmCfg<64, 10, 8, 2>;
-using Cfg128 = GemmCfg<128, 8, 8, 2>;
+// Tile configurations: tokens per tile, k-blocks per chunk, weight and
+// activation ring slots, TMEM ring slots, dequantizer groups, accumulator
+// buffers.
+using Cfg16 = GemmCfg<16, 4, 5, 3, 2, 2>;
+using Cfg32 = GemmCfg<32, 4, 4, 3, 2, 2>;
+using Cfg64 = GemmCfg<64, 2, 6, 6, 2, 2>;
+using Cfg128 = GemmCfg<128, 2, 4, 4, 2, 2>;
 
 size_t ws_counter_bytes(int64_t M, int64_t N) {
   const int64_t tiles = (N / kTileN) * ((M + 15) / 16);  // the most tiles any block_m gives
@@ -141,7 +172,17 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const void* packed, in
   if (num_tiles64 > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
   const int num_tiles = static_cast<int>(num_tiles64);
   const int KB = static_cast<int>(K / kTileK);
-  int max_ctas = dev->sms;
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  int per_sm = 1;
+  switch (bn) {
+    case 16: st = ctas_per_sm<Cfg16>(dev_id, &per_sm); break;
+    case 32: st = ctas_per_sm<Cfg32>(dev_id, &per_sm); break;
+    case 64: st = ctas_per_sm<Cfg64>(dev_id, &per_sm); break;
+    default: st = ctas_per_sm<Cfg128>(dev_id, &per_sm); break;
+  }
+  if (st != W4A8_OK) return st;
+  int max_ctas = dev->sms * per_sm;
   if (o.max_ctas > 0 && o.max_ctas < max_ctas) max_ctas = o.max_ctas;
 
   const size_t need_ws = ws_counter_bytes(M, N) + static_cast<size_t>(M) * N * 4;
@@ -217,17 +258,16 @@ w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, int8_t* A8,
   if (!aligned(A, 16) || !aligned(A8, 16) || !aligned(sA, 2) || !aligned(rowsum, 4)) return W4A8_ERR_MISALIGNED;
   const __half* a = static_cast<const __half*>(A);
   __half* s = static_cast<__half*>(sA);
-  const int grid = static_cast<int>(M);
+  const dim3 grid(static_cast<unsigned>(M));
   const int64_t nvec = K / 8;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (nvec <= 128) quantize_act_kernel<128, 1><<<grid, 128, 0, st>>>(a, K, A8, s, rowsum);
-  else if (nvec <= 256) quantize_act_kernel<256, 1><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
-  else if (nvec <= 512) quantize_act_kernel<256, 2><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
-  else if (nvec <= 1024) quantize_act_kernel<256, 4><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
-  else if (nvec <= 2048) quantize_act_kernel<256, 8><<<grid, 256, 0, st>>>(a, K, A8, s, rowsum);
-  else if (nvec <= 4096) quantize_act_kernel<512, 8><<<grid, 512, 0, st>>>(a, K, A8, s, rowsum);
-  else quantize_act_kernel<1024, 8><<<grid, 1024, 0, st>>>(a, K, A8, s, rowsum);
-  return launch_status();
+  if (nvec <= 128) return launch_pdl(quantize_act_kernel<128, 1>, grid, dim3(128), 0, st, a, K, A8, s, rowsum);
+  if (nvec <= 256) return launch_pdl(quantize_act_kernel<256, 1>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
+  if (nvec <= 512) return launch_pdl(quantize_act_kernel<256, 2>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
+  if (nvec <= 1024) return launch_pdl(quantize_act_kernel<256, 4>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
+  if (nvec <= 2048) return launch_pdl(quantize_act_kernel<256, 8>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
+  if (nvec <= 4096) return launch_pdl(quantize_act_kernel<512, 8>, grid, dim3(512), 0, st, a, K, A8, s, rowsum);
+  return launch_pdl(quantize_act_kernel<1024, 8>, grid, dim3(1024), 0, st, a, K, A8, s, rowsum);
 }
 
 w4a8_status_t w4a8_quantize_weights(const float* W, int64_t N, int64_t K, int32_t group, uint8_t* q, uint8_t* z,
