@@ -142,21 +142,29 @@ W4A8_API size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
  * Y = fp16(sA[m] * s1[n] * sum_k A8[m,k] * W8[n,k]), W8 decoded from the
  * packed blob in registers (see the top of this file).
  * A8: int8 [M, K] (from w4a8_quantize_act). sA: fp16 [M] (2-byte aligned).
+ * rowsum: int32 [M] (4-byte aligned), rowsum[m] = sum_k A8[m,k] as written
+ *   by w4a8_quantize_act. The kernel multiplies the weights in the biased
+ *   unsigned form W8 + 128 (no sign fix-up while dequantizing) and subtracts
+ *   128 * rowsum[m] exactly; a rowsum that does not match A8 gives wrong
+ *   results.
  * packed: the blob of w4a8_pack_weights for exactly this N and K.
  * Y: fp16 [M, N]. workspace: see w4a8_gemm_workspace_bytes; with too small a
  * workspace (including NULL / 0) the call uses a schedule that needs none.
  * Limits: M >= 0 (M == 0 is a no-op), N % 128 == 0, K % 128 == 0,
  * 0 < K <= 65536, M * N < 2^62.
  */
-W4A8_API w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
-                        void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream);
+W4A8_API w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed,
+                                 int64_t M, int64_t N, int64_t K, void* Y, void* workspace, size_t workspace_bytes,
+                                 w4a8_stream_t stream);
 
 /*
- * Debug entry point: the same GEMM, writing the raw int32 accumulators
- * acc[m,n] = sum_k A8[m,k] * W8[n,k] to `acc` [M, N] instead of Y.
+ * Debug entry point: the same GEMM, writing the int32 accumulators
+ * acc[m,n] = sum_k A8[m,k] * W8[n,k] to `acc` [M, N] instead of Y
+ * (rowsum as for w4a8_gemm).
  */
-W4A8_API w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const void* packed, int64_t M, int64_t N, int64_t K,
-                                  int32_t* acc, void* workspace, size_t workspace_bytes, w4a8_stream_t stream);
+W4A8_API w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const int32_t* rowsum, const void* packed, int64_t M,
+                                           int64_t N, int64_t K, int32_t* acc, void* workspace,
+                                           size_t workspace_bytes, w4a8_stream_t stream);
 
 /* Scheduling overrides for tests and tuning (zero = automatic). */
 typedef struct {
@@ -171,9 +179,9 @@ typedef struct {
  * accumulators) must be non-NULL; sA may be NULL when acc is given.
  * opts may be NULL (= all automatic).
  */
-W4A8_API w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
-                           void* Y, int32_t* acc, void* workspace, size_t workspace_bytes,
-                           const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
+W4A8_API w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed,
+                                    int64_t M, int64_t N, int64_t K, void* Y, int32_t* acc, void* workspace,
+                                    size_t workspace_bytes, const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
 
 /*
  * Allocation-free GEMM: the same computation and results as w4a8_gemm, for
@@ -203,8 +211,8 @@ W4A8_API w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const void
  * Arguments, layouts and the other limits are those of w4a8_gemm.
  */
 #define W4A8_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
-W4A8_API w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N,
-                                         int64_t K, void* Y, w4a8_stream_t stream);
+W4A8_API w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed,
+                                         int64_t M, int64_t N, int64_t K, void* Y, w4a8_stream_t stream);
 
 /*
  * Synchronizes `stream`, then stores the current device's error word in

@@ -111,15 +111,15 @@ def check_gemm(A, q, z, s2, s1, schedules=((0, 0, 0),)):
     M, K = A.shape
     N = q.shape[0]
     blob = gpu_path_from_codes(q, z, s2, s1)
-    A8, sA, _ = w4a8.quantize_act(dev(A))
+    A8, sA, rs = w4a8.quantize_act(dev(A))
     oA8, osA, _ = O.quantize_act(A)
     oacc = O.gemm_acc(oA8, O.dequant_weights(q, z, s2))
     oY = O.epilogue(oacc, osA, s1)
     ws = torch.zeros(w4a8.workspace_bytes(M, N, K), dtype=torch.uint8, device=DEV)
     for sched, bm, ctas in schedules:
-        acc = w4a8.gemm_ex(A8, None, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
+        acc = w4a8.gemm_ex(A8, None, rs, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
                            workspace=ws, schedule=sched, block_m=bm, max_ctas=ctas)
-        Y = w4a8.gemm_ex(A8, sA, blob, N, K, Y=torch.empty((M, N), dtype=torch.float16, device=DEV),
+        Y = w4a8.gemm_ex(A8, sA, rs, blob, N, K, Y=torch.empty((M, N), dtype=torch.float16, device=DEV),
                          workspace=ws, schedule=sched, block_m=bm, max_ctas=ctas)
         torch.cuda.synchronize()
         ha = host(acc)
@@ -181,7 +181,8 @@ def test_gemm_empty_m():
     blob = gpu_path_from_codes(q, z, s2, s1)
     A8 = torch.empty((0, K), dtype=torch.int8, device=DEV)
     sA = torch.empty((0,), dtype=torch.float16, device=DEV)
-    Y = w4a8.gemm(A8, sA, blob, N, K)
+    rs = torch.empty((0,), dtype=torch.int32, device=DEV)
+    Y = w4a8.gemm(A8, sA, rs, blob, N, K)
     assert Y.shape == (0, N)
 
 
@@ -190,9 +191,9 @@ def test_gemm_without_workspace_uses_whole_tiles():
     q, z, s2, s1 = I.uniform_codes(N, K, 9)
     A = I.activations(M, K, 10)
     blob = gpu_path_from_codes(q, z, s2, s1)
-    A8, sA, _ = w4a8.quantize_act(dev(A))
+    A8, sA, rs = w4a8.quantize_act(dev(A))
     empty_ws = torch.zeros(16, dtype=torch.uint8, device=DEV)
-    Y = w4a8.gemm(A8, sA, blob, N, K, workspace=empty_ws)
+    Y = w4a8.gemm(A8, sA, rs, blob, N, K, workspace=empty_ws)
     oA8, osA, _ = O.quantize_act(A)
     oY = O.w4a8_gemm(oA8, osA, q, z, s2, s1)
     torch.cuda.synchronize()
@@ -204,8 +205,9 @@ def test_gemm_split_k_requires_workspace():
     q, z, s2, s1 = I.uniform_codes(N, K, 11)
     blob = gpu_path_from_codes(q, z, s2, s1)
     A8 = torch.zeros((M, K), dtype=torch.int8, device=DEV)
+    rs = torch.zeros((M,), dtype=torch.int32, device=DEV)
     with pytest.raises(w4a8.W4A8Error, match="WORKSPACE"):
-        w4a8.gemm_ex(A8, None, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
+        w4a8.gemm_ex(A8, None, rs, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
                      workspace=torch.zeros(16, dtype=torch.uint8, device=DEV), schedule=2)
 
 
@@ -226,8 +228,8 @@ def _full_size_case(workload, lin, M, n_random_cols=64):
     del Wd
     A8, sA, rs = w4a8.quantize_act(dev(A))
     ws = torch.zeros(w4a8.workspace_bytes(M, N, K), dtype=torch.uint8, device=DEV)
-    Y = w4a8.gemm(A8, sA, blob, N, K, workspace=ws)
-    acc = w4a8.gemm_debug_acc(A8, blob, N, K, workspace=ws)
+    Y = w4a8.gemm(A8, sA, rs, blob, N, K, workspace=ws)
+    acc = w4a8.gemm_debug_acc(A8, rs, blob, N, K, workspace=ws)
     torch.cuda.synchronize()
     # activations: full comparison
     oA8, osA, ors = O.quantize_act(A)

@@ -97,22 +97,24 @@ def test_pack_validation(L):
 
 def test_gemm_validation(L):
     g = L.w4a8_gemm
-    assert g(FAKE, FAKE, FAKE, 4, 100, 256, FAKE, None, 0, None) == 2      # N % 128
-    assert g(FAKE, FAKE, FAKE, 4, 128, 200, FAKE, None, 0, None) == 2      # K % 128
-    assert g(FAKE, FAKE, FAKE, 4, 128, 65536 + 128, FAKE, None, 0, None) == 2
-    assert g(FAKE, FAKE, FAKE, -2, 128, 256, FAKE, None, 0, None) == 1
-    assert g(FAKE, FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1      # no Y
-    assert g(FAKE_ODD, FAKE, FAKE, 4, 128, 256, FAKE, None, 0, None) == 3
-    assert g(FAKE, FAKE, FAKE, 0, 128, 256, FAKE, None, 0, None) == 0      # M == 0: no-op
+    assert g(FAKE, FAKE, FAKE, FAKE, 4, 100, 256, FAKE, None, 0, None) == 2      # N % 128
+    assert g(FAKE, FAKE, FAKE, FAKE, 4, 128, 200, FAKE, None, 0, None) == 2      # K % 128
+    assert g(FAKE, FAKE, FAKE, FAKE, 4, 128, 65536 + 128, FAKE, None, 0, None) == 2
+    assert g(FAKE, FAKE, FAKE, FAKE, -2, 128, 256, FAKE, None, 0, None) == 1
+    assert g(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1      # no Y
+    assert g(FAKE, FAKE, None, FAKE, 4, 128, 256, FAKE, None, 0, None) == 1      # no rowsum
+    assert g(FAKE_ODD, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, 0, None) == 3
+    assert g(FAKE, FAKE, FAKE_ODD, FAKE, 4, 128, 256, FAKE, None, 0, None) == 3  # rowsum alignment
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 128, 256, FAKE, None, 0, None) == 0      # M == 0: no-op
     ex = L.w4a8_gemm_ex
-    bad = w4a8.GemmOpts(0, 48, 0, 0)                                       # block_m not supported
-    assert ex(FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
+    bad = w4a8.GemmOpts(0, 48, 0, 0)                                             # block_m not supported
+    assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
     bad = w4a8.GemmOpts(3, 0, 0, 0)
-    assert ex(FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
+    assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
     both = FAKE
-    assert ex(FAKE, FAKE, FAKE, 4, 128, 256, FAKE, both, None, 0, None, None) == 1  # Y and acc
-    assert L.w4a8_gemm_debug_acc(FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1  # no acc
-    assert ex(None, None, None, 0, 128, 256, None, None, None, 0, None, None) == 0   # M == 0
+    assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, both, None, 0, None, None) == 1  # Y and acc
+    assert L.w4a8_gemm_debug_acc(FAKE, FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1  # no acc
+    assert ex(None, None, None, None, 0, 128, 256, None, None, None, 0, None, None) == 0   # M == 0
 
 
 def test_python_binding_refuses_cpu_tensors(L):

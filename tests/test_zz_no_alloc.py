@@ -33,31 +33,31 @@ def _case(M, N, K, seed):
     q, z, s2, s1 = (torch.from_numpy(x).to(DEV) for x in I.uniform_codes(N, K, seed))
     blob = w4a8.pack_weights(q, z, s2, s1)
     A = torch.from_numpy(I.activations(M, K, seed + 1)).to(DEV)
-    A8, sA, _ = w4a8.quantize_act(A)
-    return A8, sA, blob
+    A8, sA, rs = w4a8.quantize_act(A)
+    return A8, sA, rs, blob
 
 
-def _noalloc(L, A8, sA, blob, M, N, K, Y):
+def _noalloc(L, A8, sA, rs, blob, M, N, K, Y):
     stream = ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream)
     return L.w4a8_gemm_noalloc(ctypes.c_void_p(A8.data_ptr()), ctypes.c_void_p(sA.data_ptr()),
-                               ctypes.c_void_p(blob.data_ptr()), M, N, K, ctypes.c_void_p(Y.data_ptr()), stream)
+                               ctypes.c_void_p(rs.data_ptr()), ctypes.c_void_p(blob.data_ptr()), M, N, K, ctypes.c_void_p(Y.data_ptr()), stream)
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 6144, 4096), (32, 4096, 14336), (33, 1024, 512)])
 def test_noalloc_matches_workspace_entry_point_twice(M, N, K):
     w4a8_build.build()
     L = w4a8.lib()
-    A8, sA, blob = _case(M, N, K, I.seed_of("noalloc", M, N, K))
+    A8, sA, rs, blob = _case(M, N, K, I.seed_of("noalloc", M, N, K))
     ws = torch.zeros(w4a8.workspace_bytes(M, N, K), dtype=torch.uint8, device=DEV)
     Y_ref = torch.empty((M, N), dtype=torch.float16, device=DEV)
     code = L.w4a8_gemm(ctypes.c_void_p(A8.data_ptr()), ctypes.c_void_p(sA.data_ptr()),
-                       ctypes.c_void_p(blob.data_ptr()), M, N, K, ctypes.c_void_p(Y_ref.data_ptr()),
+                       ctypes.c_void_p(rs.data_ptr()), ctypes.c_void_p(blob.data_ptr()), M, N, K, ctypes.c_void_p(Y_ref.data_ptr()),
                        ctypes.c_void_p(ws.data_ptr()), ws.numel(),
                        ctypes.c_void_p(torch.cuda.current_stream(DEV).cuda_stream))
     assert code == 0, w4a8.status_string(code)
     for _ in range(2):  # the second call finds the scratch array used by the first
         Y = torch.full((M, N), float("nan"), dtype=torch.float16, device=DEV)
-        code = _noalloc(L, A8, sA, blob, M, N, K, Y)
+        code = _noalloc(L, A8, sA, rs, blob, M, N, K, Y)
         assert code == 0, w4a8.status_string(code)
         torch.cuda.synchronize()
         assert max_ulp_fp16(Y.cpu().numpy(), Y_ref.cpu().numpy()) <= 1
@@ -71,9 +71,10 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     assert w4a8.workspace_bytes(M, N, K) > w4a8.NOALLOC_SCRATCH_BYTES
     A8 = torch.zeros((M, K), dtype=torch.int8, device=DEV)
     sA = torch.zeros((M,), dtype=torch.float16, device=DEV)
+    rs = torch.zeros((M,), dtype=torch.int32, device=DEV)
     blob = torch.zeros((w4a8.packed_bytes(N, K),), dtype=torch.uint8, device=DEV)
     Y = torch.zeros((M, N), dtype=torch.float16, device=DEV)
-    code = _noalloc(L, A8, sA, blob, M, N, K, Y)
+    code = _noalloc(L, A8, sA, rs, blob, M, N, K, Y)
     assert w4a8.status_string(code) == "W4A8_ERR_WORKSPACE"
     torch.cuda.synchronize()
     assert not Y.any()  # nothing was launched

@@ -8,7 +8,7 @@ library is missing or the tensors are not on a CUDA device, the calls raise.
     A8, sA, rowsum = quantize_act(A)             # fp16 [M,K] -> int8, fp16, int32
     q, z, s2, s1 = quantize_weights(W)           # fp32 [N,K] -> two-level codes
     blob = pack_weights(q, z, s2, s1)            # offline reordering
-    Y = gemm(A8, sA, blob, N, K)                 # fp16 [M,N]
+    Y = gemm(A8, sA, rowsum, blob, N, K)         # fp16 [M,N]
 """
 from __future__ import annotations
 
@@ -64,13 +64,13 @@ def lib() -> ctypes.CDLL:
         "w4a8_packed_bytes": (sz, [i64, i64, i32]),
         "w4a8_pack_weights": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i32, vp, sz, vp]),
         "w4a8_gemm_workspace_bytes": (sz, [i64, i64, i64]),
-        "w4a8_gemm": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
-        "w4a8_gemm_debug_acc": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
-        "w4a8_gemm_ex": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, vp, vp, vp, sz,
+        "w4a8_gemm": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "w4a8_gemm_debug_acc": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "w4a8_gemm_ex": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, sz,
                                         ctypes.POINTER(GemmOpts), vp]),
         "w4a8_get_device_error": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_int32)]),
         "w4a8_clear_device_error": (ctypes.c_int, [vp]),
-        "w4a8_gemm_noalloc": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, vp, vp]),
+        "w4a8_gemm_noalloc": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -200,9 +200,9 @@ def _workspace_for(device, M, N, K):
     return ws.get(M, N, K)
 
 
-def _gemm_common(A8, sA, blob, N, K, Y, acc, workspace, opts):
+def _gemm_common(A8, sA, rowsum, blob, N, K, Y, acc, workspace, opts):
     torch = _torch()
-    _require_cuda(A8, sA, blob, Y, acc, workspace)
+    _require_cuda(A8, sA, rowsum, blob, Y, acc, workspace)
     M = A8.shape[0]
     if A8.dtype != torch.int8 or A8.shape[1] != K:
         raise W4A8Error("A8 must be int8 [M, K]")
@@ -210,48 +210,49 @@ def _gemm_common(A8, sA, blob, N, K, Y, acc, workspace, opts):
         workspace = _workspace_for(A8.device, M, N, K)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     o = None if opts is None else ctypes.byref(GemmOpts(*opts))
-    code = lib().w4a8_gemm_ex(_ptr(A8), _ptr(sA), _ptr(blob), M, N, K, _ptr(Y), _ptr(acc), _ptr(workspace),
-                              ws_bytes, o, _stream(A8.device))
+    code = lib().w4a8_gemm_ex(_ptr(A8), _ptr(sA), _ptr(rowsum), _ptr(blob), M, N, K, _ptr(Y), _ptr(acc),
+                              _ptr(workspace), ws_bytes, o, _stream(A8.device))
     _check(code, "w4a8_gemm_ex")
 
 
-def gemm(A8, sA, blob, N: int, K: int, out=None, workspace=None, opts=None):
-    """Y fp16 [M, N] = fp16(sA * s1 * (A8 @ W8^T))."""
+def gemm(A8, sA, rowsum, blob, N: int, K: int, out=None, workspace=None, opts=None):
+    """Y fp16 [M, N] = fp16(sA * s1 * (A8 @ W8^T)); rowsum as from quantize_act."""
     torch = _torch()
     M = A8.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A8.device)
-    _gemm_common(A8, sA, blob, N, K, Y, None, workspace, opts)
+    _gemm_common(A8, sA, rowsum, blob, N, K, Y, None, workspace, opts)
     return Y
 
 
-def gemm_debug_acc(A8, blob, N: int, K: int, out=None, workspace=None, opts=None):
+def gemm_debug_acc(A8, rowsum, blob, N: int, K: int, out=None, workspace=None, opts=None):
     """int32 [M, N] accumulators sum_k A8[m,k] * W8[n,k]."""
     torch = _torch()
     M = A8.shape[0]
     acc = out if out is not None else torch.empty((M, N), dtype=torch.int32, device=A8.device)
-    _gemm_common(A8, None, blob, N, K, None, acc, workspace, opts)
+    _gemm_common(A8, None, rowsum, blob, N, K, None, acc, workspace, opts)
     return acc
 
 
-def gemm_ex(A8, sA, blob, N: int, K: int, Y=None, acc=None, workspace=None, schedule=0, block_m=0,
+def gemm_ex(A8, sA, rowsum, blob, N: int, K: int, Y=None, acc=None, workspace=None, schedule=0, block_m=0,
             max_ctas=0):
     """GEMM with explicit scheduling overrides (for tests and tuning)."""
-    _gemm_common(A8, sA, blob, N, K, Y, acc, workspace, (schedule, block_m, max_ctas, 0))
+    _gemm_common(A8, sA, rowsum, blob, N, K, Y, acc, workspace, (schedule, block_m, max_ctas, 0))
     return Y if Y is not None else acc
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
-def gemm_noalloc(A8, sA, blob, N: int, K: int, out=None):
+def gemm_noalloc(A8, sA, rowsum, blob, N: int, K: int, out=None):
     """The GEMM through the allocation-free entry point: the library's own
     built-in scratch array replaces the workspace (see w4a8_gemm_noalloc in
     include/w4a8.h), so no workspace is passed or allocated."""
     torch = _torch()
-    _require_cuda(A8, sA, blob, out)
+    _require_cuda(A8, sA, rowsum, blob, out)
     M = A8.shape[0]
     Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A8.device)
-    _check(lib().w4a8_gemm_noalloc(_ptr(A8), _ptr(sA), _ptr(blob), M, N, K, _ptr(Y), _stream(A8.device)),
+    _check(lib().w4a8_gemm_noalloc(_ptr(A8), _ptr(sA), _ptr(rowsum), _ptr(blob), M, N, K, _ptr(Y),
+                                   _stream(A8.device)),
            "w4a8_gemm_noalloc")
     return Y
 

@@ -57,6 +57,7 @@ struct GemmArgs {
   const uint8_t* tiles;  // packed weight tiles (blob + header)
   const __half* s1;      // per-output-channel scales (inside the blob)
   const __half* sA;      // per-token scales [M]
+  const int32_t* rowsum; // per-token sums of the int8 activation codes [M]
   __half* Y;             // [M, N] fp16 (unused when acc_out != nullptr)
   int32_t* acc_out;      // optional: raw int32 accumulators [M, N]
   int32_t* ws_acc;       // [M, N] int32 partial sums: zero on entry and exit
@@ -148,8 +149,6 @@ struct GemmCfg {
   static constexpr int kTSlotCols = KS * 32;
   static_assert(kTmemA + NT * kTSlotCols <= kTmemCols, "tensor memory budget");
   static_assert(NT > DQ, "every dequantizer group needs a TMEM slot of its own");
-  // The MMA issuer waits for chunk c + 1 before it commits chunk c, so both
-  // rings need a second slot.
   static_assert(NS >= 2 && NT >= 2, "two slots per ring at least");
   // Several dequantizer groups wait on the weight ring out of order; bounding
   // them by the TMEM ring keeps every parity wait within one phase.
@@ -178,8 +177,12 @@ enum : int {
 };
 
 // Dequantizes this thread's row r of a 128 x 128 weight tile in shared
-// memory into 32 registers: register c holds the int8 weights of
-// k = 4c .. 4c+3 (byte j = k 4c+j), the column order of the TMEM A operand.
+// memory into 32 registers: register c holds the weights of k = 4c .. 4c+3
+// (byte j = k 4c+j), the column order of the TMEM A operand, each as the
+// unsigned byte W8 + 128 = q*s2 + (128 - z*s2) in [8, 248]: two integer
+// operations per four weights (AND + IMAD; the high nibbles need one shift
+// more), and no carry crosses a byte. The MMA reads them as u8 against s8
+// activations; the epilogue removes the offset with 128 * rowsum.
 __device__ __forceinline__ void dequant_tile_regs(const uint8_t* wt, int r, uint32_t (&out)[32]) {
   const uint32_t meta = wt[kTileCodeBytes + r];
   const uint32_t zq = meta & 15u, s2 = (meta >> 4) + 1u;
@@ -190,8 +193,8 @@ __device__ __forceinline__ void dequant_tile_regs(const uint8_t* wt, int r, uint
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
-      out[c * 8 + 2 * jj] = ((w[jj] & 0x0F0F0F0Fu) * s2 + bias) ^ 0x80808080u;
-      out[c * 8 + 2 * jj + 1] = (((w[jj] >> 4) & 0x0F0F0F0Fu) * s2 + bias) ^ 0x80808080u;
+      out[c * 8 + 2 * jj] = (w[jj] & 0x0F0F0F0Fu) * s2 + bias;
+      out[c * 8 + 2 * jj + 1] = ((w[jj] >> 4) & 0x0F0F0F0Fu) * s2 + bias;
     }
   }
 }
@@ -240,11 +243,14 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
     for (int j = 0; j < 16; ++j) {
       const int m = m0 + c + j;
       if (m < args.M) {
-        const int32_t acc = static_cast<int32_t>(v[j]);
         const int64_t o = static_cast<int64_t>(m) * N + n;
         if (!whole) {
-          red_add_s32(args.ws_acc + o, acc);
-        } else if (args.acc_out != nullptr) {
+          red_add_s32(args.ws_acc + o, static_cast<int32_t>(v[j]));
+          continue;
+        }
+        // sum_k A8 * (W8 + 128) - 128 * sum_k A8 (exact in int32 for K <= 65536)
+        const int32_t acc = static_cast<int32_t>(v[j] - (static_cast<uint32_t>(__ldg(args.rowsum + m)) << 7));
+        if (args.acc_out != nullptr) {
           args.acc_out[o] = acc;
         } else {
           const float scale = __fmul_rn(__half2float(args.sA[m]), s1f);
@@ -277,7 +283,9 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = m0 + c + j;
-          v[j] = m < args.M ? __ldcg(args.ws_acc + static_cast<int64_t>(m) * N + n) : 0;
+          v[j] = m < args.M ? __ldcg(args.ws_acc + static_cast<int64_t>(m) * N + n) -
+                                  __ldg(args.rowsum + m) * 128
+                            : 0;
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -425,29 +433,20 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
         if (!mbar_wait(&accempty[b], ((seg_i / NACC) & 1) ^ 1, abort_flag, err, kErrMma)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem + b * BN;
-        // The waits for chunk c + 1 are done while chunk c's last MMAs are
-        // still executing (the tensor core queue is shallow, so a wait done
-        // between chunks would leave it idle).
-        bool ready = mbar_wait(&tfull[c % NT], (c / NT) & 1, abort_flag, err, kErrMma) &&
-                     mbar_wait(&afull[c % NS], (c / NS) & 1, abort_flag, err, kErrMma);
         for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
-          if (!ready) {
+          const int cnt = min(KS, sg.kb1 - kb);
+          const int a = c % NS, t = c % NT;
+          if (!mbar_wait(&tfull[t], (c / NT) & 1, abort_flag, err, kErrMma) ||
+              !mbar_wait(&afull[a], (c / NS) & 1, abort_flag, err, kErrMma)) {
             ok = false;
             break;
           }
-          const int cnt = min(KS, sg.kb1 - kb);
-          const int a = c % NS, t = c % NT;
-          const bool has_next = kb + KS < sg.kb1;
           tc_fence_after();
           const uint32_t a_tmem = tmem + C::kTmemA + t * C::kTSlotCols;
           const uint32_t b_addr = smem_u32(sA8 + a * C::kASlot);
           for (int j = 0; j < cnt; ++j) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
-              if (j == cnt - 1 && kk == 3 && has_next) {
-                ready = mbar_wait(&tfull[(c + 1) % NT], ((c + 1) / NT) & 1, abort_flag, err, kErrMma) &&
-                        mbar_wait(&afull[(c + 1) % NS], ((c + 1) / NS) & 1, abort_flag, err, kErrMma);
-              }
               mma_i8_ts(d_tmem, a_tmem + j * 32 + kk * 8,
                         smem_desc_k128_sw128(b_addr + j * C::kA8Bytes + kk * 32), idesc,
                         (kb + j > sg.kb0 || kk > 0) ? 1u : 0u);

@@ -184,11 +184,11 @@ __device__ __forceinline__ uint64_t smem_desc_k128_sw128(uint32_t saddr) {
   return d;
 }
 
-// Instruction descriptor: kind::i8, D = s32, A = B = s8, both K-major,
-// shape M x N (M = 128 here).
+// Instruction descriptor: kind::i8, D = s32, A = u8 (the biased weights),
+// B = s8 (the activations), both K-major, shape M x N (M = 128 here).
 __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
   return (2u << 4)                                     // D format: s32
-         | (1u << 7)                                   // A: signed 8-bit
+         | (0u << 7)                                   // A: unsigned 8-bit
          | (1u << 10)                                  // B: signed 8-bit
          | (static_cast<uint32_t>(n >> 3) << 17)       // N / 8
          | (static_cast<uint32_t>(m >> 4) << 24);      // M / 16

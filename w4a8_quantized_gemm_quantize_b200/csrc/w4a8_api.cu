@@ -131,8 +131,8 @@ w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs a
 // Tile configurations: tokens per tile, k-blocks per chunk, weight and
 // activation ring slots, TMEM ring slots, dequantizer groups, accumulator
 // buffers.
-using Cfg16 = GemmCfg<16, 4, 5, 3, 2, 2>;
-using Cfg32 = GemmCfg<32, 4, 4, 3, 2, 2>;
+using Cfg16 = GemmCfg<16, 4, 5, 3, 1, 2>;
+using Cfg32 = GemmCfg<32, 4, 4, 3, 1, 2>;
 using Cfg64 = GemmCfg<64, 2, 6, 6, 2, 2>;
 using Cfg128 = GemmCfg<128, 2, 4, 4, 2, 2>;
 
@@ -143,9 +143,9 @@ size_t ws_counter_bytes(int64_t M, int64_t N) {
 
 }  // namespace
 
-w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
-                        void* Y, int32_t* acc, void* ws, size_t ws_bytes, const w4a8_gemm_opts_t* opts,
-                        cudaStream_t stream) {
+w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+                        int64_t N, int64_t K, void* Y, int32_t* acc, void* ws, size_t ws_bytes,
+                        const w4a8_gemm_opts_t* opts, cudaStream_t stream) {
   w4a8_gemm_opts_t o = {0, 0, 0, 0};
   if (opts != nullptr) o = *opts;
   if (o.reserved != 0 || o.schedule < 0 || o.schedule > 2 || o.max_ctas < 0) return W4A8_ERR_INVALID_ARG;
@@ -156,9 +156,10 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const void* packed, in
   if (M > INT32_MAX || N > INT32_MAX || (N > 0 && M > (int64_t(1) << 62) / N)) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0 || N == 0) return W4A8_OK;
   if ((Y == nullptr) == (acc == nullptr)) return W4A8_ERR_INVALID_ARG;
-  if (A8 == nullptr || packed == nullptr || (acc == nullptr && sA == nullptr)) return W4A8_ERR_INVALID_ARG;
+  if (A8 == nullptr || packed == nullptr || rowsum == nullptr || (acc == nullptr && sA == nullptr))
+    return W4A8_ERR_INVALID_ARG;
   if (!aligned(A8, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(acc, 16) || !aligned(sA, 2) ||
-      !aligned(ws, 256))
+      !aligned(rowsum, 4) || !aligned(ws, 256))
     return W4A8_ERR_MISALIGNED;
   DeviceInfo* dev = nullptr;
   w4a8_status_t st = device_info(&dev);
@@ -209,6 +210,7 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const void* packed, in
   a.tiles = static_cast<const uint8_t*>(packed) + kHeaderBytes;
   a.s1 = reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + packed_s1_offset(N, K));
   a.sA = static_cast<const __half*>(sA);
+  a.rowsum = rowsum;
   a.Y = static_cast<__half*>(Y);
   a.acc_out = acc;
   a.ws_cnt = stream_k ? static_cast<int32_t*>(ws) : nullptr;
@@ -317,22 +319,23 @@ size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return ws_counter_bytes(M, N) + static_cast<size_t>(M) * N * 4;
 }
 
-w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
-                        void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
-  return gemm_impl(A8, sA, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
+w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+                        int64_t N, int64_t K, void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
+  return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
-w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const void* packed, int64_t M, int64_t N, int64_t K,
-                                  int32_t* acc, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
-  return gemm_impl(A8, nullptr, packed, M, N, K, nullptr, acc, workspace, workspace_bytes, nullptr,
+w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const int32_t* rowsum, const void* packed, int64_t M, int64_t N,
+                                  int64_t K, int32_t* acc, void* workspace, size_t workspace_bytes,
+                                  w4a8_stream_t stream) {
+  return gemm_impl(A8, nullptr, rowsum, packed, M, N, K, nullptr, acc, workspace, workspace_bytes, nullptr,
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
-w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N, int64_t K,
-                           void* Y, int32_t* acc, void* workspace, size_t workspace_bytes,
+w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+                           int64_t N, int64_t K, void* Y, int32_t* acc, void* workspace, size_t workspace_bytes,
                            const w4a8_gemm_opts_t* opts, w4a8_stream_t stream) {
-  return gemm_impl(A8, sA, packed, M, N, K, Y, acc, workspace, workspace_bytes, opts,
+  return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, acc, workspace, workspace_bytes, opts,
                    reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -363,10 +366,10 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[W4A8_NOALLOC_SCRATCH_
 static void* g_noalloc_addr[64] = {};
 static std::mutex g_noalloc_mu;
 
-w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const void* packed, int64_t M, int64_t N,
-                                int64_t K, void* Y, w4a8_stream_t stream) {
+w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed,
+                                int64_t M, int64_t N, int64_t K, void* Y, w4a8_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= 0 || N <= 0) return gemm_impl(A8, sA, packed, M, N, K, Y, nullptr, nullptr, 0, nullptr, st);
+  if (M <= 0 || N <= 0) return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, nullptr, nullptr, 0, nullptr, st);
   const size_t need = w4a8_gemm_workspace_bytes(M, N, K);
   if (need > W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
   int dev = 0;
@@ -384,7 +387,7 @@ w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const void* pa
   }
   // the split-k tickets and partial sums must start at zero
   if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return launch_status();
-  return gemm_impl(A8, sA, packed, M, N, K, Y, nullptr, scratch, need, nullptr, st);
+  return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, nullptr, scratch, need, nullptr, st);
 }
 
 }  // extern "C"
