@@ -124,14 +124,19 @@ struct Sched {
   }
 };
 
-template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_>
+template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_, int NMMA_>
 struct GemmCfg {
-  static constexpr int BN = BN_, KS = KS_, NS = NS_, NT = NT_, DQ = DQ_, NACC = NACC_;
+  static constexpr int BN = BN_, KS = KS_, NS = NS_, NT = NT_, DQ = DQ_, NACC = NACC_, NMMA = NMMA_;
   // One CTA per SM, persistent. Work moves in chunks of up to KS k-blocks of
   // one tile (one weight copy, one wait and one commit per chunk amortize the
   // fixed latencies of the synchronization operations).
   //   warp 0        weight producer (one thread) and TMEM owner
-  //   warp 1        MMA issuer (one thread)
+  //   warps 1..     NMMA MMA issuers (one thread each), chunk c goes to
+  //                 issuer c % NMMA, which accumulates into a partial
+  //                 accumulator of its own; the epilogue adds the partials.
+  //                 With two issuers one thread's barrier waits and commits
+  //                 overlap the other's MMAs, so the tensor pipe does not
+  //                 idle between chunks when the MMAs are thin (small BN).
   //   warp 3        activation producer (one thread)
   //   warps 4..     DQ dequantizer warpgroups, chunk c goes to group c % DQ
   //   last 4 warps  epilogue
@@ -145,7 +150,8 @@ struct GemmCfg {
   static constexpr int kASlot = KS * kA8Bytes;
   static constexpr int kWSlot = KS * kTileBytes;   // KS consecutive packed tiles
   static constexpr int kTmemCols = 512;
-  static constexpr int kTmemA = NACC * BN;         // accumulators first, then the TMEM weight ring
+  static_assert(NMMA == 1 || NMMA == 2, "one or two MMA issuers (warps 1 and 2)");
+  static constexpr int kTmemA = NACC * NMMA * BN;  // accumulators first, then the TMEM weight ring
   static constexpr int kTSlotCols = KS * 32;
   static_assert(kTmemA + NT * kTSlotCols <= kTmemCols, "tensor memory budget");
   static_assert(NT > DQ, "every dequantizer group needs a TMEM slot of its own");
@@ -312,7 +318,7 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                                                     const GemmArgs args) {
-  constexpr int BN = C::BN, KS = C::KS, NS = C::NS, NT = C::NT, DQ = C::DQ, NACC = C::NACC;
+  constexpr int BN = C::BN, KS = C::KS, NS = C::NS, NT = C::NT, DQ = C::DQ, NACC = C::NACC, NMMA = C::NMMA;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA8 = smem + C::kOffA8;
@@ -346,10 +352,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       mbar_init(&tempty[i], 1);
     }
     for (int i = 0; i < NACC; ++i) {
-      mbar_init(&accfull[i], 1);
+      mbar_init(&accfull[i], NMMA);
       mbar_init(&accempty[i], 4);
     }
-    mbar_init(done, 1);
+    mbar_init(done, NMMA);
     misc[1] = 0;
     misc[2] = 0;
     misc[3] = 0;
@@ -422,9 +428,13 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       for (int i = first; i < c; ++i) mbar_wait(&afull[i % NS], (i / NS) & 1, nullptr, err, kErrDrain);
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp >= 1 && warp < 1 + NMMA) {
+    // ----------------------------------------------------------- MMA issuers
+    // Issuer mi takes chunks c = mi (mod NMMA) into its partial accumulator
+    // (b * NMMA + mi) and commits every segment's accumulator barrier, with
+    // or without MMAs of its own in that segment.
     if (lane == 0) {
+      const int mi = warp - 1;
       constexpr uint32_t idesc = idesc_i8(128, BN);
       int c = 0, seg_i = 0;
       bool ok = true;
@@ -432,8 +442,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
         const int b = seg_i % NACC;
         if (!mbar_wait(&accempty[b], ((seg_i / NACC) & 1) ^ 1, abort_flag, err, kErrMma)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + b * BN;
+        const uint32_t d_tmem = tmem + (b * NMMA + mi) * BN;
+        bool first = true;
         for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
+          if (c % NMMA != mi) continue;
           const int cnt = min(KS, sg.kb1 - kb);
           const int a = c % NS, t = c % NT;
           if (!mbar_wait(&tfull[t], (c / NT) & 1, abort_flag, err, kErrMma) ||
@@ -449,9 +461,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
             for (int kk = 0; kk < 4; ++kk) {
               mma_i8_ts(d_tmem, a_tmem + j * 32 + kk * 8,
                         smem_desc_k128_sw128(b_addr + j * C::kA8Bytes + kk * 32), idesc,
-                        (kb + j > sg.kb0 || kk > 0) ? 1u : 0u);
+                        (!first || j > 0 || kk > 0) ? 1u : 0u);
             }
           }
+          first = false;
           mma_commit(&aempty[a]);
           mma_commit(&tempty[t]);
         }
@@ -526,13 +539,17 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     // ------------------------------------------------------------ epilogue
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-    int seg_i = 0;
+    int seg_i = 0, c0 = 0;
     while (sch.next(sg)) {
       const int b = seg_i % NACC;
+      // issuer mi wrote partial mi iff the segment has a chunk c = mi (mod NMMA)
+      const int nch = (sg.kb1 - sg.kb0 + KS - 1) / KS;
+      const uint32_t used = NMMA == 1 ? 1u : (nch >= 2 ? 3u : (1u << (c0 % 2)));
       if (!epilogue_segment<BN>(args, sg, true, &accfull[b], (seg_i / NACC) & 1, &accempty[b],
-                                tmem + b * BN + lane_base, 0, 1u, quarter, lane, abort_flag, epi_fail, last_flag,
-                                err))
+                                tmem + b * NMMA * BN + lane_base, BN, used, quarter, lane, abort_flag, epi_fail,
+                                last_flag, err))
         break;
+      c0 += nch;
       ++seg_i;
     }
   }
