@@ -131,7 +131,8 @@ W4A8_API w4a8_status_t w4a8_pack_weights(const uint8_t* q, const uint8_t* z, con
 /*
  * Workspace for w4a8_gemm / w4a8_gemm_debug_acc / w4a8_gemm_ex: int32
  * partial sums and per-tile tickets used when one output tile's k-range is
- * split across CTAs (the decode regime). The caller zero-fills it ONCE before
+ * split across CTAs that are not in one cluster (the decode regime with
+ * more tiles than fit one cluster each; the cluster split needs none). The caller zero-fills it ONCE before
  * first use; every call that completes without a device error leaves it
  * zero-filled again. Calls that share a workspace must not overlap in time.
  * A workspace of the returned size serves every M' <= M, N' <= N.
@@ -168,7 +169,11 @@ W4A8_API w4a8_status_t w4a8_gemm_debug_acc(const int8_t* A8, const int32_t* rows
 
 /* Scheduling overrides for tests and tuning (zero = automatic). */
 typedef struct {
-  int32_t schedule;  /* 0 auto, 1 whole tiles per CTA, 2 split k-ranges (needs workspace) */
+  int32_t schedule;  /* 0 auto, 1 whole tiles per CTA, 2 split k-ranges (needs workspace),
+                        3 cluster split (block_m <= 32: each tile's k-range split over the
+                        2..4 CTAs of one thread-block cluster, reduced on chip; needs no
+                        workspace; W4A8_ERR_UNSUPPORTED_SHAPE if the tiles do not fit
+                        one cluster each) */
   int32_t block_m;   /* tokens per tile: 0 auto, or 16, 32, 64, 128 */
   int32_t max_ctas;  /* 0 auto (one CTA per SM), else an upper bound on the grid */
   int32_t reserved;  /* must be 0 */

@@ -130,7 +130,12 @@ def check_gemm(A, q, z, s2, s1, schedules=((0, 0, 0),)):
     return oY
 
 
-ALL_SCHEDULES = [(0, 0, 0)] + [(s, bm, c) for s in (1, 2) for bm in (16, 32, 64, 128) for c in (0, 7)]
+# (schedule, block_m, max_ctas); auto with a small grid mixes stream-K
+# remainder tiles with whole tiles
+ALL_SCHEDULES = ([(0, 0, 0), (0, 16, 4), (0, 16, 5), (0, 32, 3)] +
+                 [(s, bm, c) for s in (1, 2) for bm in (16, 32, 64, 128) for c in (0, 7)] +
+                 [(3, 16, 0), (3, 32, 0)])
+CLUSTER = [(3, 16, 0), (3, 32, 0)]  # cluster split-K: needs few enough tiles
 
 
 @pytest.mark.parametrize("M", [1, 16, 33])
@@ -148,7 +153,31 @@ def test_gemm_tiny_config_all_schedules(M):
 def test_gemm_ragged_shapes(M, N, K):
     q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-g", N, K))
     A = I.activations(M, K, I.seed_of("t-a", M, K))
-    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (1, 0, 0), (2, 0, 0), (2, 16, 5), (1, 128, 3)])
+    scheds = [(0, 0, 0), (1, 0, 0), (2, 0, 0), (2, 16, 5), (1, 128, 3), (0, 16, 5), (0, 64, 3)]
+    if (N // 128) * -(-M // 16) <= 32:  # one cluster per tile fits
+        scheds += CLUSTER
+    check_gemm(A, q, z, s2, s1, scheds)
+
+
+@pytest.mark.parametrize("K", [256, 384, 512, 4096])
+def test_gemm_cluster_split_sizes(K):
+    """Cluster split-K with every split size the k-block count allows
+    (2, 3, 4 CTAs per tile), through the automatic choice and forced."""
+    N, M = 512, 5
+    q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-cl", N, K))
+    A = I.activations(M, K, I.seed_of("t-cla", M, K))
+    check_gemm(A, q, z, s2, s1, [(0, 0, 0)] + CLUSTER)
+
+
+def test_gemm_cluster_split_needs_two_k_blocks():
+    N, K, M = 256, 128, 4
+    q, z, s2, s1 = I.uniform_codes(N, K, 12)
+    blob = gpu_path_from_codes(q, z, s2, s1)
+    A8 = torch.zeros((M, K), dtype=torch.int8, device=DEV)
+    rs = torch.zeros((M,), dtype=torch.int32, device=DEV)
+    with pytest.raises(w4a8.W4A8Error, match="UNSUPPORTED"):
+        w4a8.gemm_ex(A8, None, rs, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
+                     schedule=3)
 
 
 def test_gemm_extreme_codes():
@@ -163,7 +192,7 @@ def test_gemm_extreme_codes():
     s1 = np.full(N, 1e-3, np.float16)
     A = np.full((M, K), 1.0, np.float16)
     A[1] = -1.0
-    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (2, 0, 0)])
+    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (2, 0, 0), (3, 16, 0)])
 
 
 def test_gemm_zero_rows_and_columns():
@@ -172,7 +201,7 @@ def test_gemm_zero_rows_and_columns():
     q[5] = np.repeat(z[5], 128)      # a weight row that dequantizes to 0
     A = I.activations(M, K, 78)
     A[4] = 0                         # a zero token: sA = 0
-    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (2, 16, 0)])
+    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (2, 16, 0), (3, 32, 0)])
 
 
 def test_gemm_empty_m():

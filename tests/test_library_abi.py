@@ -109,7 +109,7 @@ def test_gemm_validation(L):
     ex = L.w4a8_gemm_ex
     bad = w4a8.GemmOpts(0, 48, 0, 0)                                             # block_m not supported
     assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
-    bad = w4a8.GemmOpts(3, 0, 0, 0)
+    bad = w4a8.GemmOpts(4, 0, 0, 0)
     assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
     both = FAKE
     assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, both, None, 0, None, None) == 1  # Y and acc

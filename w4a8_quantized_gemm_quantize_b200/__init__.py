@@ -31,7 +31,7 @@ EXPORTED_SYMBOLS = (
     "w4a8_gemm_noalloc",
 )
 
-SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K = 0, 1, 2
+SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
 
 
 class W4A8Error(RuntimeError):

@@ -10,43 +10,36 @@
 // elements, and weight load, dequantization and MMA overlapped in one
 // pipeline without software synchronization in the hot loop).
 //
-// Structure (persistent CTAs; warp roles):
-//   producer    one thread: per k-block, a TMA 2-D load of the int8
-//               activation tile (BN tokens x 128 k, 128-byte swizzle) and a
-//               1-D bulk copy of the packed weight tile (128 n x 128 k, 8320
-//               bytes) into a STAGES-deep shared-memory ring.
-//   dequant     four warps (one per TMEM lane quarter): thread r owns weight
-//               row r; it reads its 64 code bytes as four 16-byte vectors and
-//               turns every four codes into four int8 weights with
-//               ((w & 0x0F0F0F0F) * s2 + (128 - z*s2) * 0x01010101) ^ 0x80808080
-//               (each byte stays in [8, 248] before the xor, so no carry
-//               crosses a byte), then writes the 128 int8 weights of its row
-//               straight into tensor memory with tcgen05.st. The dequantized
-//               weights never touch shared memory (the point of the "QUICK"
-//               abstract's interleaving, reached here through TMEM).
-//   MMA         one thread: tcgen05.mma.kind::i8 with A = the dequantized
-//               weights in TMEM (M = 128 rows = n), B = the activation tile in
-//               shared memory (N = BN tokens), K = 32 per instruction; int32
-//               accumulators in TMEM.
-//   epilogue    four warps: tcgen05.ld of the accumulators (lane = n,
-//               column = token), scale, fp16 store; or, for a partial
-//               k-range, red.add into an int32 workspace and a ticket counter
-//               whose last arriver finishes the tile (nobody spins on another
-//               CTA).
-// Two layouts: "compact" (6 warps; the dequant warps also run the epilogue;
-// 128 TMEM columns and ~50 KB of shared memory, so several CTAs share an SM
-// and hide each other's issue latencies, which dominate when the MMA is thin
-// as in decode) and "full" (12 warps, one CTA per SM, a separate epilogue
-// group and two accumulator buffers so a tile's epilogue overlaps the next
-// tile's mainloop).
-// The roles synchronize only through mbarriers; every wait is bounded in
-// time and reports through the device error word.
+// Structure: one persistent CTA per SM; warp-specialized roles that
+// synchronize only through mbarriers (every wait bounded in time, reported
+// through the device error word):
+//   weight producer      one thread: per chunk of up to KS k-blocks of a
+//                        tile, one 1-D bulk copy of the contiguous packed
+//                        tiles (KS x 8320 bytes) into a weight ring slot;
+//                        it starts before the dependency wait because the
+//                        weights do not come from the preceding kernel.
+//   activation producer  one thread: TMA 2-D loads of the int8 activation
+//                        tiles (BN tokens x 128 k, 128-byte swizzle), after
+//                        the programmatic-launch dependency wait.
+//   dequantizers         DQ warpgroups; thread r owns weight row r of a tile:
+//                        it reads its 64 code bytes as four 16-byte vectors
+//                        and turns every four codes into four unsigned bytes
+//                        W8 + 128 = q * s2 + (128 - z * s2) in [8, 248] with
+//                        one AND and one IMAD (no carry crosses a byte), then
+//                        writes them straight into tensor memory
+//                        (tcgen05.st). The dequantized weights never touch
+//                        shared memory (the point of the "QUICK" abstract's
+//                        interleaving, reached here through TMEM).
+//   MMA issuers          NMMA threads, alternate chunks:
+//                        tcgen05.mma.kind::i8 with A = the dequantized
+//                        weights in TMEM (u8, M = 128 rows = n), B = the
+//                        activation tile in shared memory (s8, N = BN
+//                        tokens), K = 32 per instruction; int32 accumulators
+//                        in TMEM, one partial accumulator per issuer.
+//   epilogue             four warps: tcgen05.ld of the partial accumulators,
+//                        sum, minus 128 * rowsum[m] (undoes the weight bias
+//                        exactly), scale, fp16 store.
 //
-// Work split: tiles are (token block of BN) x (128 output channels), each
-// with K/128 k-blocks. Either whole tiles round-robin over the CTAs, or
-// ("stream-K") each CTA takes one contiguous range of the flattened
-// (tile, k-block) sequence, which balances small-M problems whose tile count
-// is below the SM count.
 #pragma once
 #include "pack.cuh"
 #include "ptx.cuh"
@@ -65,49 +58,56 @@ struct GemmArgs {
   int* err;              // device error word
   int M, N, KB;
   int m_tiles, num_tiles;
-  int stream_k;
+  int sk_tiles;          // the first sk_tiles tiles are split stream-K over all CTAs
+  int split;             // > 1: cluster split-K, `split` CTAs (one cluster) per tile
 };
 
 struct Seg {
   int tile, kb0, kb1;
 };
 
-// The same deterministic schedule is replayed by every role of a CTA.
+// The same deterministic schedule is replayed by every role of a CTA. Two
+// kinds of work:
+//   stream-K     the first sk_tiles tiles, flattened to (tile, k-block)
+//                units: CTA i takes the i-th of grid equal ranges (its first
+//                and last tiles are usually partial, reduced through the
+//                global workspace);
+//   whole tiles  the remaining tiles round robin, all k-blocks each.
+// A CTA does its stream-K range first, so that the reduction of partial
+// tiles overlaps the mainloop of its whole tiles and the last epilogue is a
+// direct one. With cluster split-K instead, tile t is split into `split`
+// k-ranges taken by the CTAs of cluster t (CTA rank r takes k-blocks
+// [KB r / split, KB (r + 1) / split)) and reduced on chip.
 struct Sched {
-  int64_t u, u_end, u_begin;
-  int tile_it, KB, num_tiles, stream_k;
+  int64_t u, u_end;
+  int tile_it, KB, num_tiles, split;
   __device__ __forceinline__ void init(const GemmArgs& a) {
     KB = a.KB;
     num_tiles = a.num_tiles;
-    stream_k = a.stream_k;
-    if (stream_k) {
-      const int64_t U = static_cast<int64_t>(num_tiles) * KB;
+    split = a.split;
+    u = u_end = 0;
+    if (split > 1) {
+      tile_it = static_cast<int>(blockIdx.x) / split;
+      return;
+    }
+    if (a.sk_tiles > 0) {
+      const int64_t U = static_cast<int64_t>(a.sk_tiles) * KB;
       u = U * blockIdx.x / gridDim.x;
       u_end = U * (blockIdx.x + 1) / gridDim.x;
-      u_begin = u;
-    } else {
-      tile_it = blockIdx.x;
     }
-  }
-  // Total k-blocks of this CTA, and the (tile, k-block) of its it-th one.
-  __device__ __forceinline__ int total() const {
-    if (stream_k) return static_cast<int>(u_end - u_begin);
-    const int mine = blockIdx.x < num_tiles ? (num_tiles - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
-    return mine * KB;
-  }
-  __device__ __forceinline__ void at(int it, int& tile, int& kb) const {
-    if (stream_k) {
-      const int64_t uu = u_begin + it;
-      tile = static_cast<int>(uu / KB);
-      kb = static_cast<int>(uu - static_cast<int64_t>(tile) * KB);
-    } else {
-      tile = static_cast<int>(blockIdx.x) + (it / KB) * static_cast<int>(gridDim.x);
-      kb = it % KB;
-    }
+    tile_it = a.sk_tiles + static_cast<int>(blockIdx.x);
   }
   __device__ __forceinline__ bool next(Seg& s) {
-    if (stream_k) {
-      if (u >= u_end) return false;
+    if (split > 1) {
+      if (tile_it < 0 || tile_it >= num_tiles) return false;
+      const int r = static_cast<int>(blockIdx.x) % split;
+      s.tile = tile_it;
+      s.kb0 = KB * r / split;
+      s.kb1 = KB * (r + 1) / split;
+      tile_it = -1;
+      return true;
+    }
+    if (u < u_end) {
       s.tile = static_cast<int>(u / KB);
       s.kb0 = static_cast<int>(u - static_cast<int64_t>(s.tile) * KB);
       const int64_t left = u_end - u;
@@ -165,10 +165,19 @@ struct GemmCfg {
   // otherwise it completes them within the chunk.
   static constexpr bool kPipelinedStores = NT >= 2 * DQ && NT >= DQ + 2;
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
+  // Cluster split-K (small BN only): up to kMaxSplit CTAs per tile. The
+  // owner of TMEM lane quarter q is cluster rank q % split; it receives the
+  // other ranks' 32 x BN partial sums of that quarter into kRecvSlots slots
+  // of 32 x BN int32 (column-major: word j * 32 + row), at most 4 of them
+  // for any split <= 4 (split 3: rank 0 owns two quarters, two senders each).
+  static constexpr int kMaxSplit = BN <= 32 ? 4 : 1;
+  static constexpr int kRecvSlots = kMaxSplit > 1 ? 4 : 0;
+  static constexpr int kRecvSlotBytes = 32 * BN * 4;
   static constexpr int kOffA8 = 0;                 // 1024-aligned activation slots
   static constexpr int kOffW = NS * kASlot;        // 16-aligned weight slots
-  static constexpr int kOffBar = (kOffW + NS * kWSlot + 15) / 16 * 16;
-  static constexpr int kNumBars = 4 * NS + 2 * NT + 2 * NACC + 1;
+  static constexpr int kOffRecv = kOffW + NS * kWSlot;
+  static constexpr int kOffBar = (kOffRecv + kRecvSlots * kRecvSlotBytes + 15) / 16 * 16;
+  static constexpr int kNumBars = 4 * NS + 2 * NT + 2 * NACC + 1 + 4;  // + one receive barrier per lane quarter
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -205,6 +214,44 @@ __device__ __forceinline__ void dequant_tile_regs(const uint8_t* wt, int r, uint
   }
 }
 
+// Per-token operands of the epilogue, one row per lane for a block of 32
+// rows starting at token mb (fetched ahead of use and broadcast with
+// shuffles, so no global load sits between the accumulator and the store).
+//
+// Loads under a guard read an in-bounds address (the row is clamped, M >= 1)
+// and let the guard only select the value. sA may be null (the accumulator
+// output needs no scales): it is read with a plain load, never with the fp16
+// __ldg overload, which is a side-effect-free asm statement that the compiler
+// is free to evaluate ahead of the null test.
+struct RowOperands {
+  int32_t rowsum;
+  float sa;
+  __device__ __forceinline__ void fetch(const GemmArgs& a, int mb, int lane) {
+    const int m = mb + lane;
+    const int mc = m < a.M ? m : a.M - 1;
+    const int32_t r = __ldg(a.rowsum + mc);
+    float s = 0.0f;
+    if (a.sA != nullptr) s = __half2float(a.sA[mc]);
+    rowsum = m < a.M ? r : 0;
+    sa = m < a.M ? s : 0.0f;
+  }
+  __device__ __forceinline__ int32_t rowsum_of(int row) const { return __shfl_sync(0xffffffffu, rowsum, row & 31); }
+  __device__ __forceinline__ float sa_of(int row) const { return __shfl_sync(0xffffffffu, sa, row & 31); }
+};
+
+// Stores one output element: acc = biased sum - 128 * rowsum (exact in
+// int32 for K <= 65536), then either the raw accumulator or
+// fp16(acc * (sA * s1)).
+__device__ __forceinline__ void store_output(const GemmArgs& a, int64_t o, uint32_t biased, int32_t rowsum, float sa,
+                                             float s1f) {
+  const int32_t acc = static_cast<int32_t>(biased - (static_cast<uint32_t>(rowsum) << 7));
+  if (a.acc_out != nullptr) {
+    a.acc_out[o] = acc;
+  } else {
+    a.Y[o] = __float2half_rn(__fmul_rn(__int2float_rn(acc), __fmul_rn(sa, s1f)));
+  }
+}
+
 // Epilogue of one segment for the four warps of an epilogue group (128
 // threads, named barrier 1). `tacc` is this warp's lane quarter at the
 // first lane's accumulator; lane j's accumulator is `lane_stride * j`
@@ -216,6 +263,14 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
                                                  uint32_t lane_stride, uint32_t lanes_used, int quarter, int lane,
                                                  volatile int* abort_flag, volatile int* epi_fail,
                                                  volatile int* last_flag, DevErr err) {
+  const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
+  const int64_t N = args.N;
+  const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
+  const int m0 = m_tile * BN;
+  const bool whole = (sg.kb0 == 0 && sg.kb1 == args.KB);
+  const float s1f = __half2float(args.s1[n]);
+  RowOperands rows;
+  if (whole) rows.fetch(args, m0, lane);  // in flight while the MMAs finish
   // the four warps take one decision, so every named barrier below is
   // reached by all of them
   bool ok = ok_in && mbar_wait(accfull, bph, abort_flag, err, kErrEpilogue);
@@ -224,14 +279,9 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
   named_bar_sync(1, 128);
   if (*epi_fail) return false;
   tc_fence_after();
-  const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
-  const int64_t N = args.N;
-  const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
-  const int m0 = m_tile * BN;
-  const bool whole = (sg.kb0 == 0 && sg.kb1 == args.KB);
-  const float s1f = __half2float(args.s1[n]);
 #pragma unroll 1
   for (int c = 0; c < BN; c += 16) {
+    if (whole && c > 0 && (c & 31) == 0) rows.fetch(args, m0 + c, lane);
     uint32_t v[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = 0;
@@ -239,8 +289,7 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
     for (uint32_t l = 0, used = lanes_used; used != 0; ++l, used >>= 1) {
       if (used & 1u) {
         uint32_t u[16];
-        tmem_ld_16(tacc + l * lane_stride + c, u);
-        tmem_wait_ld();
+        tmem_ld_16_wait(tacc + l * lane_stride + c, u);
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] += u[j];
       }
@@ -248,21 +297,14 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const int m = m0 + c + j;
-      if (m < args.M) {
-        const int64_t o = static_cast<int64_t>(m) * N + n;
-        if (!whole) {
-          red_add_s32(args.ws_acc + o, static_cast<int32_t>(v[j]));
-          continue;
-        }
-        // sum_k A8 * (W8 + 128) - 128 * sum_k A8 (exact in int32 for K <= 65536)
-        const int32_t acc = static_cast<int32_t>(v[j] - (static_cast<uint32_t>(__ldg(args.rowsum + m)) << 7));
-        if (args.acc_out != nullptr) {
-          args.acc_out[o] = acc;
-        } else {
-          const float scale = __fmul_rn(__half2float(args.sA[m]), s1f);
-          args.Y[o] = __float2half_rn(__fmul_rn(__int2float_rn(acc), scale));
-        }
+      const int64_t o = static_cast<int64_t>(m) * N + n;
+      if (!whole) {
+        if (m < args.M) red_add_s32(args.ws_acc + o, static_cast<int32_t>(v[j]));
+        continue;
       }
+      const int32_t rs = rows.rowsum_of(c + j);
+      const float sa = rows.sa_of(c + j);
+      if (m < args.M) store_output(args, o, v[j], rs, sa, s1f);
     }
   }
   tc_fence_before();
@@ -285,32 +327,105 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
     if (*last_flag) {
 #pragma unroll 1
       for (int c = 0; c < BN; c += 16) {
-        int32_t v[16];
+        if ((c & 31) == 0) rows.fetch(args, m0 + c, lane);
+        uint32_t v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = m0 + c + j;
-          v[j] = m < args.M ? __ldcg(args.ws_acc + static_cast<int64_t>(m) * N + n) -
-                                  __ldg(args.rowsum + m) * 128
-                            : 0;
+          const int mc = m < args.M ? m : args.M - 1;
+          const uint32_t x = static_cast<uint32_t>(__ldcg(args.ws_acc + static_cast<int64_t>(mc) * N + n));
+          v[j] = m < args.M ? x : 0u;
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = m0 + c + j;
+          const int32_t rs = rows.rowsum_of(c + j);
+          const float sa = rows.sa_of(c + j);
           if (m < args.M) {
             const int64_t o = static_cast<int64_t>(m) * N + n;
             __stcg(args.ws_acc + o, 0);
-            if (args.acc_out != nullptr) {
-              args.acc_out[o] = v[j];
-            } else {
-              const float scale = __fmul_rn(__half2float(args.sA[m]), s1f);
-              args.Y[o] = __float2half_rn(__fmul_rn(__int2float_rn(v[j]), scale));
-            }
+            store_output(args, o, v[j], rs, sa, s1f);
           }
         }
       }
       if (quarter == 0 && lane == 0) args.ws_cnt[sg.tile] = 0;
     }
     named_bar_sync(1, 128);
+  }
+  return true;
+}
+
+// Epilogue of a cluster split-K tile for the four warps of the epilogue
+// group: every CTA of the cluster holds the partial sums of its k-range; the
+// owner of lane quarter q (rank q % split) receives the other ranks' 32 x BN
+// partials of that quarter through distributed shared memory (st.async,
+// counted by the owner's receive barrier), adds them and writes the rows.
+template <class C>
+__device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg& sg, uint64_t* accfull,
+                                                 uint64_t* accempty, uint32_t tacc, uint32_t lanes_used,
+                                                 int quarter, int lane, uint32_t* recv, uint64_t* recvbar,
+                                                 volatile int* abort_flag, volatile int* epi_fail, DevErr err) {
+  constexpr int BN = C::BN;
+  static_assert(BN <= 32, "one row block of per-token operands");
+  const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
+  const int64_t N = args.N;
+  const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
+  const int m0 = m_tile * BN;
+  const float s1f = __half2float(args.s1[n]);
+  RowOperands rows;
+  rows.fetch(args, m0, lane);  // in flight while the MMAs finish
+  cluster_wait();              // every receive barrier of the cluster is armed
+  bool ok = mbar_wait(accfull, 0, abort_flag, err, kErrEpilogue);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok && lane == 0) *epi_fail = 1;
+  named_bar_sync(1, 128);
+  if (*epi_fail) return false;
+  tc_fence_after();
+  uint32_t v[BN];
+#pragma unroll
+  for (int c = 0; c < BN; c += 16) {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[c + j] = 0;
+#pragma unroll 1
+    for (uint32_t l = 0, used = lanes_used; used != 0; ++l, used >>= 1) {
+      if (used & 1u) {
+        uint32_t u[16];
+        tmem_ld_16_wait(tacc + l * BN + c, u);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[c + j] += u[j];
+      }
+    }
+  }
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(accempty);
+
+  const int S = args.split;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int owner = quarter % S;
+  const int slot0 = (quarter / S) * (S - 1);  // this quarter's first receive slot at its owner
+  if (owner != rank) {
+    const int slot = slot0 + (rank < owner ? rank : rank - 1);
+    const uint32_t dst = mapa_shared(smem_u32(recv) + slot * C::kRecvSlotBytes + lane * 4, owner);
+    const uint32_t bar = mapa_shared(smem_u32(&recvbar[quarter]), owner);
+#pragma unroll
+    for (int j = 0; j < BN; ++j) st_async_b32(dst + j * 128, v[j], bar);
+    return true;
+  }
+  ok = mbar_wait(&recvbar[quarter], 0, abort_flag, err, kErrEpilogue);
+  if (!__all_sync(0xffffffffu, ok)) return false;
+#pragma unroll 1
+  for (int sidx = 0; sidx < S - 1; ++sidx) {
+    const uint32_t* src = recv + (slot0 + sidx) * (C::kRecvSlotBytes / 4) + lane;
+#pragma unroll
+    for (int j = 0; j < BN; ++j) v[j] += src[j * 32];
+  }
+#pragma unroll
+  for (int j = 0; j < BN; ++j) {
+    const int m = m0 + j;
+    const int32_t rs = rows.rowsum_of(j);
+    const float sa = rows.sa_of(j);
+    if (m < args.M) store_output(args, static_cast<int64_t>(m) * N + n, v[j], rs, sa, s1f);
   }
   return true;
 }
@@ -332,6 +447,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
   uint64_t* accfull = tempty + NT;                                   // a segment's MMAs finished
   uint64_t* accempty = accfull + NACC;                               // epilogue has read the accumulator
   uint64_t* done = accempty + NACC;                                  // all MMAs finished
+  uint64_t* recvbar = done + 1;                                      // cluster partials received, per quarter
+  uint32_t* recv = reinterpret_cast<uint32_t*>(smem + C::kOffRecv);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 2);
@@ -356,6 +473,12 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       mbar_init(&accempty[i], 4);
     }
     mbar_init(done, NMMA);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(&recvbar[q], 1);
+      // armed once: completes when the other ranks' partials of quarter q land
+      if (C::kMaxSplit > 1 && args.split > 1 && q % args.split == static_cast<int>(cluster_ctarank()))
+        mbar_arrive_expect_tx(&recvbar[q], (args.split - 1) * C::kRecvSlotBytes);
+    }
     misc[1] = 0;
     misc[2] = 0;
     misc[3] = 0;
@@ -371,10 +494,14 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
+  // cluster split-K: the receive barriers are initialized before any CTA of
+  // the cluster may store into this one (the epilogue waits on this phase)
+  if (C::kMaxSplit > 1 && args.split > 1) cluster_arrive();
 
   Sched sch;
   sch.init(args);
   Seg sg;
+  bool cluster_waited = false;
 
   if (warp == 0) {
     // ----------------------------------------------------- weight producer
@@ -537,6 +664,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     }
   } else if (warp >= C::kEpWarp0 && warp < C::kEpWarp0 + 4) {
     // ------------------------------------------------------------ epilogue
+    // sA and rowsum come from the preceding kernel (the activation quantizer)
+    grid_dependency_wait();
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     int seg_i = 0, c0 = 0;
@@ -545,6 +674,15 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       // issuer mi wrote partial mi iff the segment has a chunk c = mi (mod NMMA)
       const int nch = (sg.kb1 - sg.kb0 + KS - 1) / KS;
       const uint32_t used = NMMA == 1 ? 1u : (nch >= 2 ? 3u : (1u << (c0 % 2)));
+      if constexpr (C::kMaxSplit > 1) {
+        if (args.split > 1) {
+          // the single segment of a cluster split-K CTA
+          cluster_waited = true;
+          epilogue_cluster<C>(args, sg, &accfull[b], &accempty[b], tmem + b * NMMA * BN + lane_base, used,
+                              quarter, lane, recv, recvbar, abort_flag, epi_fail, err);
+          break;
+        }
+      }
       if (!epilogue_segment<BN>(args, sg, true, &accfull[b], (seg_i / NACC) & 1, &accempty[b],
                                 tmem + b * NMMA * BN + lane_base, BN, used, quarter, lane, abort_flag, epi_fail,
                                 last_flag, err))
@@ -554,6 +692,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     }
   }
 
+  // every thread of a cluster split-K launch waits on the cluster barrier
+  // phase it arrived on (the epilogue group already has, unless it failed
+  // before reaching it)
+  __syncwarp();
+  if (C::kMaxSplit > 1 && args.split > 1 && !__all_sync(0xffffffffu, cluster_waited)) cluster_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {

@@ -72,8 +72,10 @@ __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __r
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int idx = threadIdx.x + i * THREADS;
+    // streamed once; the address is clamped into the row because the
+    // compiler may issue this load ahead of the bounds test
+    v[i] = __ldcs(row + (idx < nvec ? idx : nvec - 1));
     if (idx < nvec) {
-      v[i] = __ldcs(row + idx);  // streamed once
       const __half2* h = reinterpret_cast<const __half2*>(&v[i]);
 #pragma unroll
       for (int j = 0; j < 4; ++j) {

@@ -72,19 +72,29 @@ w4a8_status_t device_info(DeviceInfo** out) {
 // Launches with programmatic stream serialization: the kernel may start
 // while its predecessor in the stream finishes; it waits (griddepcontrol)
 // before touching anything the predecessor writes.
+// A cluster size above 1 launches thread-block clusters of that many CTAs
+// along x.
 template <typename... KArgs, typename... Args>
 w4a8_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                         Args&&... args) {
+                         int cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  int n = 1;
+  if (cluster > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(cluster);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    n = 2;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = n;
   return cuda_status(cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...));
 }
 
@@ -113,9 +123,46 @@ w4a8_status_t ctas_per_sm(int dev, int* out) {
   return W4A8_OK;
 }
 
+// Clusters of `split` CTAs of a configuration that can be resident at once
+// (0 when a cluster of that size cannot be scheduled), computed once per
+// device and size.
+template <class C>
+w4a8_status_t max_clusters(int dev, int split, int* out) {
+  static int cache[kMaxDevices][C::kMaxSplit + 1] = {};
+  if (split < 2 || split > C::kMaxSplit) {
+    *out = 0;
+    return W4A8_OK;
+  }
+  if (cache[dev][split] == 0) {
+    int dummy = 0;
+    w4a8_status_t st = ctas_per_sm<C>(dev, &dummy);  // sets the shared-memory attribute
+    if (st != W4A8_OK) return st;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(split);
+    cfg.blockDim = dim3(C::kThreads);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(split);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, w4a8_gemm_kernel<C>, &cfg) != cudaSuccess) {
+      (void)cudaGetLastError();
+      n = 0;
+    }
+    cache[dev][split] = n > 0 ? n : -1;
+  }
+  *out = cache[dev][split] > 0 ? cache[dev][split] : 0;
+  return W4A8_OK;
+}
+
 template <class C>
 w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs args, int grid,
                               cudaStream_t stream) {
+  if (args.split > C::kMaxSplit) return W4A8_ERR_INVALID_ARG;
   CUtensorMap map;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
@@ -125,7 +172,8 @@ w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs a
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return W4A8_ERR_CUDA;
-  return launch_pdl(w4a8_gemm_kernel<C>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, map, args);
+  return launch_pdl(w4a8_gemm_kernel<C>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, args.split, map,
+                    args);
 }
 
 // Tile configurations: tokens per tile, k-blocks per chunk, weight and
@@ -148,7 +196,7 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum,
                         const w4a8_gemm_opts_t* opts, cudaStream_t stream) {
   w4a8_gemm_opts_t o = {0, 0, 0, 0};
   if (opts != nullptr) o = *opts;
-  if (o.reserved != 0 || o.schedule < 0 || o.schedule > 2 || o.max_ctas < 0) return W4A8_ERR_INVALID_ARG;
+  if (o.reserved != 0 || o.schedule < 0 || o.schedule > 3 || o.max_ctas < 0) return W4A8_ERR_INVALID_ARG;
   if (!(o.block_m == 0 || o.block_m == 16 || o.block_m == 32 || o.block_m == 64 || o.block_m == 128))
     return W4A8_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
@@ -186,20 +234,39 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum,
   int max_ctas = dev->sms * per_sm;
   if (o.max_ctas > 0 && o.max_ctas < max_ctas) max_ctas = o.max_ctas;
 
+  // Cluster split: the largest split (<= 4, <= KB) whose clusters can all
+  // be resident with one tile each. Chosen automatically when the tiles
+  // fill at most half of the SMs (each tile then gets two or more CTAs).
+  int split = 1;
+  if (bn <= 32 && (o.schedule == 3 || (o.schedule == 0 && o.max_ctas == 0 && 2 * num_tiles <= dev->sms))) {
+    for (int S = 4; S >= 2 && split == 1; --S) {
+      if (S > KB) continue;
+      int nclu = 0;
+      st = bn == 16 ? max_clusters<Cfg16>(dev_id, S, &nclu) : max_clusters<Cfg32>(dev_id, S, &nclu);
+      if (st != W4A8_OK) return st;
+      if (num_tiles <= nclu) split = S;
+    }
+  }
+  if (o.schedule == 3 && split == 1) return W4A8_ERR_UNSUPPORTED_SHAPE;
+
   const size_t need_ws = ws_counter_bytes(M, N) + static_cast<size_t>(M) * N * 4;
   const bool ws_ok = ws != nullptr && ws_bytes >= need_ws;
-  int stream_k;
-  if (o.schedule == 2) {
+  // Tiles split stream-K (the rest go whole, round robin): everything when
+  // the tiles do not fill one wave, else the tiles beyond the full waves, so
+  // that every CTA gets the same number of k-blocks.
+  int sk_tiles = 0;
+  if (split > 1) {
+    sk_tiles = 0;
+  } else if (o.schedule == 2) {
     if (!ws_ok) return W4A8_ERR_WORKSPACE;
-    stream_k = 1;
-  } else if (o.schedule == 1) {
-    stream_k = 0;
-  } else {
-    // whole tiles once there are enough of them to fill the machine twice
-    stream_k = (ws_ok && num_tiles < 2 * max_ctas) ? 1 : 0;
+    sk_tiles = num_tiles;
+  } else if (o.schedule == 0 && ws_ok) {
+    sk_tiles = num_tiles < max_ctas ? num_tiles : num_tiles % max_ctas;
   }
   int grid;
-  if (stream_k) {
+  if (split > 1) {
+    grid = num_tiles * split;
+  } else if (sk_tiles == num_tiles) {
     const int64_t units = static_cast<int64_t>(num_tiles) * KB;
     grid = static_cast<int>(units < max_ctas ? units : max_ctas);
   } else {
@@ -213,15 +280,16 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum,
   a.rowsum = rowsum;
   a.Y = static_cast<__half*>(Y);
   a.acc_out = acc;
-  a.ws_cnt = stream_k ? static_cast<int32_t*>(ws) : nullptr;
-  a.ws_acc = stream_k ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_counter_bytes(M, N)) : nullptr;
+  a.ws_cnt = sk_tiles > 0 ? static_cast<int32_t*>(ws) : nullptr;
+  a.ws_acc = sk_tiles > 0 ? reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + ws_counter_bytes(M, N)) : nullptr;
   a.err = dev->err;
   a.M = static_cast<int>(M);
   a.N = static_cast<int>(N);
   a.KB = KB;
   a.m_tiles = m_tiles;
   a.num_tiles = num_tiles;
-  a.stream_k = stream_k;
+  a.sk_tiles = sk_tiles;
+  a.split = split;
   switch (bn) {
     case 16: return launch_gemm_cfg<Cfg16>(A8, M, K, a, grid, stream);
     case 32: return launch_gemm_cfg<Cfg32>(A8, M, K, a, grid, stream);
@@ -263,13 +331,13 @@ w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, int8_t* A8,
   const dim3 grid(static_cast<unsigned>(M));
   const int64_t nvec = K / 8;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (nvec <= 128) return launch_pdl(quantize_act_kernel<128, 1>, grid, dim3(128), 0, st, a, K, A8, s, rowsum);
-  if (nvec <= 256) return launch_pdl(quantize_act_kernel<256, 1>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
-  if (nvec <= 512) return launch_pdl(quantize_act_kernel<256, 2>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
-  if (nvec <= 1024) return launch_pdl(quantize_act_kernel<256, 4>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
-  if (nvec <= 2048) return launch_pdl(quantize_act_kernel<256, 8>, grid, dim3(256), 0, st, a, K, A8, s, rowsum);
-  if (nvec <= 4096) return launch_pdl(quantize_act_kernel<512, 8>, grid, dim3(512), 0, st, a, K, A8, s, rowsum);
-  return launch_pdl(quantize_act_kernel<1024, 8>, grid, dim3(1024), 0, st, a, K, A8, s, rowsum);
+  if (nvec <= 128) return launch_pdl(quantize_act_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, A8, s, rowsum);
+  if (nvec <= 256) return launch_pdl(quantize_act_kernel<256, 1>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
+  if (nvec <= 512) return launch_pdl(quantize_act_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
+  if (nvec <= 1024) return launch_pdl(quantize_act_kernel<256, 4>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
+  if (nvec <= 2048) return launch_pdl(quantize_act_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
+  if (nvec <= 4096) return launch_pdl(quantize_act_kernel<512, 8>, grid, dim3(512), 0, st, 1, a, K, A8, s, rowsum);
+  return launch_pdl(quantize_act_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, A8, s, rowsum);
 }
 
 w4a8_status_t w4a8_quantize_weights(const float* W, int64_t N, int64_t K, int32_t group, uint8_t* q, uint8_t* z,
