@@ -72,9 +72,17 @@ def gemm_ops(M, N, K):
     return 2 * M * N * K
 
 
-def cases_of(workload):
+def cases_of(workload, only=None):
+    """The workload's (M, layer, N, K) cases; `only` ("16:gate_up,1:o")
+    keeps a subset (for profiling single shapes)."""
     wl = I.WORKLOADS[workload]
-    return [(M, name, N, K) for M in wl.ms for (name, N, K) in wl.linears]
+    cases = [(M, name, N, K) for M in wl.ms for (name, N, K) in wl.linears]
+    if only:
+        keep = {(int(x.split(":")[0]), x.split(":")[1]) for x in only.split(",")}
+        cases = [c for c in cases if (c[0], c[1]) in keep]
+        if not cases:
+            raise SystemExit(f"--cases {only!r} selects nothing from workload {workload!r}")
+    return cases
 
 
 def load_peaks():
@@ -265,7 +273,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     wl = I.WORKLOADS[args.workload]
-    cases = cases_of(args.workload)
+    cases = cases_of(args.workload, args.cases)
     n_copies = len(wl.ms)  # one weight copy per M value: no GEMM reuses L2-resident weights
 
     # ---- offline: quantize + pack the weights (untimed), one copy per M
@@ -310,6 +318,15 @@ def run_gpu(args, world, rank, local):
                 events[i][1].record()
             if d2h is not None:
                 d2h[(M, name)].copy_(Y, non_blocking=True)
+
+    if args.profile:
+        # for an external profiler: eager steps only, no timing, no JSON line
+        for _ in range(args.profile):
+            step()
+        torch.cuda.synchronize()
+        assert w4a8.get_device_error(dev) == 0
+        print(f"profile: {args.profile} eager steps of {len(cases)} cases done")
+        return None
 
     for _ in range(args.warmup):
         step()
@@ -412,6 +429,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cases", default=None,
+                    help="subset of the workload's cases, e.g. 16:gate_up,1:o (profiling)")
+    ap.add_argument("--profile", type=int, default=0,
+                    help="run this many eager steps for an external profiler and exit (no timing)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -427,6 +448,8 @@ def main():
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
 
     r = run_gpu(args, world, rank, local)
+    if r is None:  # --profile
+        return 0
     cases = r["cases"]
     peaks = load_peaks()
     wbytes = sum(weight_bytes(N, K) for (M, _, N, K) in cases)

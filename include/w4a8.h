@@ -64,6 +64,7 @@ typedef enum {
 #define W4A8_DEVERR_DEQUANT_WAIT 3
 #define W4A8_DEVERR_EPILOGUE_WAIT 4
 #define W4A8_DEVERR_DRAIN_WAIT 5
+#define W4A8_DEVERR_SELFTEST_WAIT 6
 
 /* Human-readable name of a status code (static string, never NULL). */
 W4A8_API const char* w4a8_status_string(int status);
@@ -228,6 +229,18 @@ W4A8_API w4a8_status_t w4a8_get_device_error(w4a8_stream_t stream, int32_t* code
 
 /* Resets the current device's error word to 0 (stream-ordered). */
 W4A8_API w4a8_status_t w4a8_clear_device_error(w4a8_stream_t stream);
+
+/*
+ * Failure-path self-test (no counterpart in the papers; it exercises the
+ * library's own failure detection). Launches one warp that waits on an
+ * mbarrier nothing ever completes, with the same bounded wait every kernel of
+ * the library uses but a limit of `limit_ns` (clamped to [1 us, 2 s]). The
+ * wait gives up, records W4A8_DEVERR_SELFTEST_WAIT in the device error word
+ * (unless it already holds a code) and the kernel returns: no fault, no hang,
+ * and the context stays usable. Read the result with w4a8_get_device_error
+ * and reset it with w4a8_clear_device_error.
+ */
+W4A8_API w4a8_status_t w4a8_selftest_bounded_wait(int64_t limit_ns, w4a8_stream_t stream);
 
 #ifdef __cplusplus
 }

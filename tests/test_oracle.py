@@ -187,6 +187,32 @@ def test_dequant_full_domain_bytewise():
         assert lanes == ref
 
 
+def test_unsigned_biased_accumulation_identity():
+    """The GEMM may multiply the biased unsigned bytes B = W8 + 128 =
+    q*s2 + (128 - z*s2) in [8, 248] against the int8 activations and subtract
+    128 * sum_k A8 afterwards: sum_k A8 (W8 + 128) - 128 sum_k A8 equals the
+    oracle's accumulator exactly, and the biased sum stays inside int32 for
+    every K <= 65536 (|sum| <= 127 * 248 * 65536 < 2^31)."""
+    assert 127 * 248 * 65536 < 2 ** 31
+    rng = np.random.default_rng(17)
+    for K in (128, 384, 1024):
+        M, N = 3, 5
+        q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+        z = rng.integers(0, 16, (N, K // 128)).astype(np.uint8)
+        s2 = rng.integers(1, 9, (N, K // 128)).astype(np.uint8)
+        A8 = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        ref = O.gemm_acc(A8, O.dequant_weights(q, z, s2))
+        zz = np.repeat(z.astype(np.int64), 128, axis=1)
+        ss = np.repeat(s2.astype(np.int64), 128, axis=1)
+        biased = q.astype(np.int64) * ss + (128 - zz * ss)
+        assert biased.min() >= 8 and biased.max() <= 248
+        for m in range(M):
+            rowsum = int(A8[m].astype(np.int64).sum())
+            for n in range(N):
+                s = sum(int(a) * int(b) for a, b in zip(A8[m].tolist(), biased[n].tolist()))
+                assert s - 128 * rowsum == int(ref[m, n])
+
+
 def test_quantize_weights_exact_group():
     """A row whose groups are exactly representable: s1 = 2^-6 (the largest
     group range is 120 * 2^-6), group 0 holds t in {-56, 0, 64}

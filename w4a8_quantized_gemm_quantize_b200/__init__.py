@@ -19,6 +19,7 @@ __all__ = [
     "W4A8Error", "lib", "library_path", "EXPORTED_SYMBOLS", "status_string", "quantize_act",
     "quantize_weights", "packed_bytes", "pack_weights", "workspace_bytes", "Workspace", "gemm",
     "gemm_debug_acc", "gemm_ex", "gemm_noalloc", "get_device_error", "clear_device_error",
+    "selftest_bounded_wait",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -28,7 +29,7 @@ EXPORTED_SYMBOLS = (
     "w4a8_status_string", "w4a8_version", "w4a8_quantize_act", "w4a8_quantize_weights",
     "w4a8_packed_bytes", "w4a8_pack_weights", "w4a8_gemm_workspace_bytes", "w4a8_gemm",
     "w4a8_gemm_debug_acc", "w4a8_gemm_ex", "w4a8_get_device_error", "w4a8_clear_device_error",
-    "w4a8_gemm_noalloc",
+    "w4a8_gemm_noalloc", "w4a8_selftest_bounded_wait",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
@@ -71,6 +72,7 @@ def lib() -> ctypes.CDLL:
         "w4a8_get_device_error": (ctypes.c_int, [vp, ctypes.POINTER(ctypes.c_int32)]),
         "w4a8_clear_device_error": (ctypes.c_int, [vp]),
         "w4a8_gemm_noalloc": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp]),
+        "w4a8_selftest_bounded_wait": (ctypes.c_int, [i64, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -265,3 +267,12 @@ def get_device_error(device=None) -> int:
 
 def clear_device_error(device=None):
     _check(lib().w4a8_clear_device_error(_stream(device)), "w4a8_clear_device_error")
+
+
+DEVERR_SELFTEST_WAIT = 6
+
+
+def selftest_bounded_wait(limit_ns: int, device=None):
+    """Launches the failure-path self-test (a bounded wait that must give up
+    after `limit_ns`); its code shows in get_device_error()."""
+    _check(lib().w4a8_selftest_bounded_wait(int(limit_ns), _stream(device)), "w4a8_selftest_bounded_wait")

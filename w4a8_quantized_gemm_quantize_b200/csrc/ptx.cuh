@@ -59,11 +59,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Waits for the phase with the given parity to complete. Returns false if
-// the CTA's abort flag (when given) is set, or once the time limit passes;
-// then it sets the flag (when given) and records `code` in the device error
-// word. Without an abort flag the wait only ends by completion or time.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          DevErr err, int code) {
+// the CTA's abort flag (when given) is set, or once `limit_ns` passes; then it
+// sets the flag (when given) and records `code` in the device error word.
+// Without an abort flag the wait only ends by completion or time.
+__device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                                DevErr err, int code, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = global_timer_ns();
@@ -71,13 +71,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 31u) == 0) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         if (abort_flag != nullptr) *abort_flag = 1;
         atomicCAS(err.word, 0, code);
         return false;
       }
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          DevErr err, int code) {
+  return mbar_wait_limit(bar, parity, abort_flag, err, code, kWaitLimitNs);
 }
 
 // ------------------------------------------------------ TMA / bulk copies

@@ -11,6 +11,7 @@
 #include "pack.cuh"
 #include "quantize_act.cuh"
 #include "quantize_weights.cuh"
+#include "selftest.cuh"
 #include "w4a8.h"
 
 namespace w4a8 {
@@ -424,6 +425,17 @@ w4a8_status_t w4a8_clear_device_error(w4a8_stream_t stream) {
   w4a8_status_t st = device_info(&dev);
   if (st != W4A8_OK) return st;
   return cuda_status(cudaMemsetAsync(dev->err, 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+w4a8_status_t w4a8_selftest_bounded_wait(int64_t limit_ns, w4a8_stream_t stream) {
+  DeviceInfo* dev = nullptr;
+  w4a8_status_t st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+  const int64_t lo = 1000, hi = static_cast<int64_t>(kWaitLimitNs);
+  const int64_t lim = limit_ns < lo ? lo : limit_ns > hi ? hi : limit_ns;
+  bounded_wait_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      dev->err, static_cast<uint64_t>(lim), W4A8_DEVERR_SELFTEST_WAIT);
+  return launch_status();
 }
 
 // ------------------------------------------------- allocation-free GEMM
