@@ -179,7 +179,12 @@ struct GemmCfg {
   static constexpr int kOffBar = (kOffRecv + kRecvSlots * kRecvSlotBytes + 15) / 16 * 16;
   static constexpr int kNumBars = 4 * NS + 2 * NT + 2 * NACC + 1 + 4;  // + one receive barrier per lane quarter
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  // epilogue per-token operands (128 int32 + 128 float), then the store
+  // transpose (1 KB per epilogue warp, read as 16-byte vectors: 16-aligned)
+  static constexpr int kOffRows = (kOffMisc + 64 + 15) / 16 * 16;
+  static constexpr int kOffYStage = kOffRows + 1024;
+  static_assert(kOffYStage % 16 == 0, "16-byte aligned store stage");
+  static constexpr int kSmemBytes = kOffYStage + 4096 + 1024;  // + alignment slack
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -214,29 +219,31 @@ __device__ __forceinline__ void dequant_tile_regs(const uint8_t* wt, int r, uint
   }
 }
 
-// Per-token operands of the epilogue, one row per lane for a block of 32
-// rows starting at token mb (fetched ahead of use and broadcast with
-// shuffles, so no global load sits between the accumulator and the store).
+// Per-token operands of the epilogue, staged in shared memory per segment:
+// thread t of the epilogue group loads token m0 + t before the group waits
+// for the accumulator (one global load per thread, hidden behind the
+// mainloop), and the store loops read them back as broadcast shared loads,
+// so no global load sits between the accumulator and the output stores.
 //
 // Loads under a guard read an in-bounds address (the row is clamped, M >= 1)
 // and let the guard only select the value. sA may be null (the accumulator
 // output needs no scales): it is read with a plain load, never with the fp16
 // __ldg overload, which is a side-effect-free asm statement that the compiler
 // is free to evaluate ahead of the null test.
-struct RowOperands {
-  int32_t rowsum;
-  float sa;
-  __device__ __forceinline__ void fetch(const GemmArgs& a, int mb, int lane) {
-    const int m = mb + lane;
-    const int mc = m < a.M ? m : a.M - 1;
-    const int32_t r = __ldg(a.rowsum + mc);
-    float s = 0.0f;
-    if (a.sA != nullptr) s = __half2float(a.sA[mc]);
-    rowsum = m < a.M ? r : 0;
-    sa = m < a.M ? s : 0.0f;
+struct RowStage {
+  int32_t* rowsum;  // [128]
+  float* sa;        // [128]
+  __device__ __forceinline__ void load(const GemmArgs& a, int m0, int t, int rows) {
+    if (t < rows) {
+      const int m = m0 + t;
+      const int mc = m < a.M ? m : a.M - 1;
+      const int32_t r = __ldg(a.rowsum + mc);
+      float s = 0.0f;
+      if (a.sA != nullptr) s = __half2float(a.sA[mc]);
+      rowsum[t] = m < a.M ? r : 0;
+      sa[t] = m < a.M ? s : 0.0f;
+    }
   }
-  __device__ __forceinline__ int32_t rowsum_of(int row) const { return __shfl_sync(0xffffffffu, rowsum, row & 31); }
-  __device__ __forceinline__ float sa_of(int row) const { return __shfl_sync(0xffffffffu, sa, row & 31); }
 };
 
 // Stores one output element: acc = biased sum - 128 * rowsum (exact in
@@ -252,6 +259,32 @@ __device__ __forceinline__ void store_output(const GemmArgs& a, int64_t o, uint3
   }
 }
 
+// fp16 output of one element (no store): fp16(acc * (sA * s1)) with
+// acc = biased sum - 128 * rowsum.
+__device__ __forceinline__ __half output_half(uint32_t biased, int32_t rowsum, float sa, float s1f) {
+  const int32_t acc = static_cast<int32_t>(biased - (static_cast<uint32_t>(rowsum) << 7));
+  return __float2half_rn(__fmul_rn(__int2float_rn(acc), __fmul_rn(sa, s1f)));
+}
+
+// Stores a warp's 16 rows x 32 channels of fp16 output (lane = channel
+// n_base + lane, h[j] = row m_start + j) with 16-byte stores: the block is
+// transposed through the warp's 1 KB shared-memory stage so that each
+// instruction writes 8 whole 64-byte row pieces instead of 2 bytes a lane.
+__device__ __forceinline__ void store_y_rows16(const GemmArgs& a, __half* stage, const __half (&h)[16], int m_start,
+                                               int64_t n_base, int lane) {
+#pragma unroll
+  for (int j = 0; j < 16; ++j) stage[j * 32 + lane] = h[j];
+  __syncwarp();
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int r = pass * 8 + (lane >> 2), q = lane & 3;
+    const uint4 v = *reinterpret_cast<const uint4*>(stage + r * 32 + q * 8);
+    const int m = m_start + r;
+    if (m < a.M) *reinterpret_cast<uint4*>(a.Y + static_cast<int64_t>(m) * a.N + n_base + q * 8) = v;
+  }
+  __syncwarp();  // the stage is reused by the next block
+}
+
 // Epilogue of one segment for the four warps of an epilogue group (128
 // threads, named barrier 1). `tacc` is this warp's lane quarter at the
 // first lane's accumulator; lane j's accumulator is `lane_stride * j`
@@ -261,16 +294,16 @@ template <int BN>
 __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg& sg, bool ok_in, uint64_t* accfull,
                                                  uint32_t bph, uint64_t* accempty, uint32_t tacc,
                                                  uint32_t lane_stride, uint32_t lanes_used, int quarter, int lane,
-                                                 volatile int* abort_flag, volatile int* epi_fail,
-                                                 volatile int* last_flag, DevErr err) {
+                                                 RowStage rows, __half* ystage, volatile int* abort_flag,
+                                                 volatile int* epi_fail, volatile int* last_flag, DevErr err) {
   const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
   const int64_t N = args.N;
   const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
   const int m0 = m_tile * BN;
   const bool whole = (sg.kb0 == 0 && sg.kb1 == args.KB);
   const float s1f = __half2float(args.s1[n]);
-  RowOperands rows;
-  if (whole) rows.fetch(args, m0, lane);  // in flight while the MMAs finish
+  named_bar_sync(1, 128);  // the previous segment's reads of the stage are done
+  rows.load(args, m0, quarter * 32 + lane, BN);
   // the four warps take one decision, so every named barrier below is
   // reached by all of them
   bool ok = ok_in && mbar_wait(accfull, bph, abort_flag, err, kErrEpilogue);
@@ -281,7 +314,6 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
   tc_fence_after();
 #pragma unroll 1
   for (int c = 0; c < BN; c += 16) {
-    if (whole && c > 0 && (c & 31) == 0) rows.fetch(args, m0 + c, lane);
     uint32_t v[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) v[j] = 0;
@@ -294,17 +326,30 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
         for (int j = 0; j < 16; ++j) v[j] += u[j];
       }
     }
+    int32_t rsv[16];
+    float sav[16];
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
-      const int m = m0 + c + j;
-      const int64_t o = static_cast<int64_t>(m) * N + n;
-      if (!whole) {
-        if (m < args.M) red_add_s32(args.ws_acc + o, static_cast<int32_t>(v[j]));
-        continue;
+      rsv[j] = rows.rowsum[c + j];
+      sav[j] = rows.sa[c + j];
+    }
+    if (!whole) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int m = m0 + c + j;
+        if (m < args.M) red_add_s32(args.ws_acc + static_cast<int64_t>(m) * N + n, static_cast<int32_t>(v[j]));
       }
-      const int32_t rs = rows.rowsum_of(c + j);
-      const float sa = rows.sa_of(c + j);
-      if (m < args.M) store_output(args, o, v[j], rs, sa, s1f);
+    } else if (args.acc_out != nullptr) {
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int m = m0 + c + j;
+        if (m < args.M) store_output(args, static_cast<int64_t>(m) * N + n, v[j], rsv[j], sav[j], s1f);
+      }
+    } else {
+      __half h[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) h[j] = output_half(v[j], rsv[j], sav[j], s1f);
+      store_y_rows16(args, ystage, h, m0 + c, n - lane, lane);
     }
   }
   tc_fence_before();
@@ -327,7 +372,6 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
     if (*last_flag) {
 #pragma unroll 1
       for (int c = 0; c < BN; c += 16) {
-        if ((c & 31) == 0) rows.fetch(args, m0 + c, lane);
         uint32_t v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
@@ -339,12 +383,10 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           const int m = m0 + c + j;
-          const int32_t rs = rows.rowsum_of(c + j);
-          const float sa = rows.sa_of(c + j);
           if (m < args.M) {
             const int64_t o = static_cast<int64_t>(m) * N + n;
             __stcg(args.ws_acc + o, 0);
-            store_output(args, o, v[j], rs, sa, s1f);
+            store_output(args, o, v[j], rows.rowsum[c + j], rows.sa[c + j], s1f);
           }
         }
       }
@@ -364,7 +406,8 @@ template <class C>
 __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg& sg, uint64_t* accfull,
                                                  uint64_t* accempty, uint32_t tacc, uint32_t lanes_used,
                                                  int quarter, int lane, uint32_t* recv, uint64_t* recvbar,
-                                                 volatile int* abort_flag, volatile int* epi_fail, DevErr err) {
+                                                 RowStage rows, __half* ystage, volatile int* abort_flag,
+                                                 volatile int* epi_fail, DevErr err) {
   constexpr int BN = C::BN;
   static_assert(BN <= 32, "one row block of per-token operands");
   const int m_tile = sg.tile % args.m_tiles, n_tile = sg.tile / args.m_tiles;
@@ -372,9 +415,8 @@ __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg
   const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
   const int m0 = m_tile * BN;
   const float s1f = __half2float(args.s1[n]);
-  RowOperands rows;
-  rows.fetch(args, m0, lane);  // in flight while the MMAs finish
-  cluster_wait();              // every receive barrier of the cluster is armed
+  rows.load(args, m0, quarter * 32 + lane, BN);  // made visible by the barrier after the accumulator wait
+  cluster_wait();                                // every receive barrier of the cluster is armed
   bool ok = mbar_wait(accfull, 0, abort_flag, err, kErrEpilogue);
   ok = __all_sync(0xffffffffu, ok);
   if (!ok && lane == 0) *epi_fail = 1;
@@ -420,12 +462,20 @@ __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg
 #pragma unroll
     for (int j = 0; j < BN; ++j) v[j] += src[j * 32];
   }
+  if (args.acc_out != nullptr) {
 #pragma unroll
-  for (int j = 0; j < BN; ++j) {
-    const int m = m0 + j;
-    const int32_t rs = rows.rowsum_of(j);
-    const float sa = rows.sa_of(j);
-    if (m < args.M) store_output(args, static_cast<int64_t>(m) * N + n, v[j], rs, sa, s1f);
+    for (int j = 0; j < BN; ++j) {
+      const int m = m0 + j;
+      if (m < args.M) store_output(args, static_cast<int64_t>(m) * N + n, v[j], rows.rowsum[j], rows.sa[j], s1f);
+    }
+    return true;
+  }
+#pragma unroll
+  for (int c = 0; c < BN; c += 16) {
+    __half h[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) h[j] = output_half(v[c + j], rows.rowsum[c + j], rows.sa[c + j], s1f);
+    store_y_rows16(args, ystage, h, m0 + c, n - lane, lane);
   }
   return true;
 }
@@ -668,6 +718,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     grid_dependency_wait();
     const int quarter = warp & 3;
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+    RowStage rows{reinterpret_cast<int32_t*>(smem + C::kOffRows), reinterpret_cast<float*>(smem + C::kOffRows + 512)};
+    __half* ystage = reinterpret_cast<__half*>(smem + C::kOffYStage + quarter * 1024);
     int seg_i = 0, c0 = 0;
     while (sch.next(sg)) {
       const int b = seg_i % NACC;
@@ -679,13 +731,13 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
           // the single segment of a cluster split-K CTA
           cluster_waited = true;
           epilogue_cluster<C>(args, sg, &accfull[b], &accempty[b], tmem + b * NMMA * BN + lane_base, used,
-                              quarter, lane, recv, recvbar, abort_flag, epi_fail, err);
+                              quarter, lane, recv, recvbar, rows, ystage, abort_flag, epi_fail, err);
           break;
         }
       }
       if (!epilogue_segment<BN>(args, sg, true, &accfull[b], (seg_i / NACC) & 1, &accempty[b],
-                                tmem + b * NMMA * BN + lane_base, BN, used, quarter, lane, abort_flag, epi_fail,
-                                last_flag, err))
+                                tmem + b * NMMA * BN + lane_base, BN, used, quarter, lane, rows, ystage,
+                                abort_flag, epi_fail, last_flag, err))
         break;
       c0 += nch;
       ++seg_i;
