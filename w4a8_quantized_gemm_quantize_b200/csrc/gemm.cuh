@@ -35,10 +35,12 @@
 //                        weights in TMEM (u8, M = 128 rows = n), B = the
 //                        activation tile in shared memory (s8, N = BN
 //                        tokens), K = 32 per instruction; int32 accumulators
-//                        in TMEM, one partial accumulator per issuer.
-//   epilogue             four warps: tcgen05.ld of the partial accumulators,
-//                        sum, minus 128 * rowsum[m] (undoes the weight bias
-//                        exactly), scale, fp16 store.
+//                        in TMEM; both issuers accumulate into the same
+//                        buffer (exact integer sums do not depend on order).
+//   epilogue             four warps: tcgen05.ld of the accumulator, which it
+//                        zeroes for its next use, minus 128 * rowsum[m]
+//                        (undoes the weight bias exactly), scale, fp16 store
+//                        (16-byte stores through a shared-memory transpose).
 //
 #pragma once
 #include "pack.cuh"
@@ -151,7 +153,7 @@ struct GemmCfg {
   static constexpr int kWSlot = KS * kTileBytes;   // KS consecutive packed tiles
   static constexpr int kTmemCols = 512;
   static_assert(NMMA == 1 || NMMA == 2, "one or two MMA issuers (warps 1 and 2)");
-  static constexpr int kTmemA = NACC * NMMA * BN;  // accumulators first, then the TMEM weight ring
+  static constexpr int kTmemA = NACC * BN;  // accumulators first, then the TMEM weight ring
   static constexpr int kTSlotCols = KS * 32;
   static_assert(kTmemA + NT * kTSlotCols <= kTmemCols, "tensor memory budget");
   static_assert(NT > DQ, "every dequantizer group needs a TMEM slot of its own");
@@ -326,6 +328,7 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
         for (int j = 0; j < 16; ++j) v[j] += u[j];
       }
     }
+    tmem_zero_16(tacc + c);  // every MMA accumulates: the buffer starts the next segment at zero
     int32_t rsv[16];
     float sav[16];
 #pragma unroll
@@ -352,6 +355,7 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
       store_y_rows16(args, ystage, h, m0 + c, n - lane, lane);
     }
   }
+  tmem_wait_st();
   tc_fence_before();
   __syncwarp();
   if (lane == 0) mbar_arrive(accempty);
@@ -607,9 +611,12 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     __syncwarp();
   } else if (warp >= 1 && warp < 1 + NMMA) {
     // ----------------------------------------------------------- MMA issuers
-    // Issuer mi takes chunks c = mi (mod NMMA) into its partial accumulator
-    // (b * NMMA + mi) and commits every segment's accumulator barrier, with
-    // or without MMAs of its own in that segment.
+    // Issuer mi takes chunks c = mi (mod NMMA). Both issuers accumulate into
+    // the segment's one accumulator buffer b: every MMA accumulates (the
+    // epilogue hands the buffer back zeroed), so the order in which the tensor
+    // pipe runs the two threads' MMAs does not change the exact int32 sums.
+    // Each issuer commits every segment's accumulator barrier, with or without
+    // MMAs of its own in that segment.
     if (lane == 0) {
       const int mi = warp - 1;
       constexpr uint32_t idesc = idesc_i8(128, BN);
@@ -617,10 +624,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       bool ok = true;
       while (ok && sch.next(sg)) {
         const int b = seg_i % NACC;
-        if (!mbar_wait(&accempty[b], ((seg_i / NACC) & 1) ^ 1, abort_flag, err, kErrMma)) break;
+        if (!mbar_wait(&accempty[b], (seg_i / NACC) & 1, abort_flag, err, kErrMma)) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem + (b * NMMA + mi) * BN;
-        bool first = true;
+        const uint32_t d_tmem = tmem + b * BN;
         for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
           if (c % NMMA != mi) continue;
           const int cnt = min(KS, sg.kb1 - kb);
@@ -638,10 +644,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
             for (int kk = 0; kk < 4; ++kk) {
               mma_i8_ts(d_tmem, a_tmem + j * 32 + kk * 8,
                         smem_desc_k128_sw128(b_addr + j * C::kA8Bytes + kk * 32), idesc,
-                        (!first || j > 0 || kk > 0) ? 1u : 0u);
+                        1u);
             }
           }
-          first = false;
           mma_commit(&aempty[a]);
           mma_commit(&tempty[t]);
         }
@@ -720,26 +725,31 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
     RowStage rows{reinterpret_cast<int32_t*>(smem + C::kOffRows), reinterpret_cast<float*>(smem + C::kOffRows + 512)};
     __half* ystage = reinterpret_cast<__half*>(smem + C::kOffYStage + quarter * 1024);
-    int seg_i = 0, c0 = 0;
+    // every MMA accumulates: the accumulator buffers start at zero
+    for (int b = 0; b < NACC; ++b)
+      for (int c = 0; c < BN; c += 16) tmem_zero_16(tmem + b * BN + c + lane_base);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0)
+      for (int b = 0; b < NACC; ++b) mbar_arrive(&accempty[b]);
+    int seg_i = 0;
     while (sch.next(sg)) {
       const int b = seg_i % NACC;
-      // issuer mi wrote partial mi iff the segment has a chunk c = mi (mod NMMA)
-      const int nch = (sg.kb1 - sg.kb0 + KS - 1) / KS;
-      const uint32_t used = NMMA == 1 ? 1u : (nch >= 2 ? 3u : (1u << (c0 % 2)));
+      const uint32_t used = 1u;  // one accumulator per buffer
       if constexpr (C::kMaxSplit > 1) {
         if (args.split > 1) {
           // the single segment of a cluster split-K CTA
           cluster_waited = true;
-          epilogue_cluster<C>(args, sg, &accfull[b], &accempty[b], tmem + b * NMMA * BN + lane_base, used,
+          epilogue_cluster<C>(args, sg, &accfull[b], &accempty[b], tmem + b * BN + lane_base, used,
                               quarter, lane, recv, recvbar, rows, ystage, abort_flag, epi_fail, err);
           break;
         }
       }
       if (!epilogue_segment<BN>(args, sg, true, &accfull[b], (seg_i / NACC) & 1, &accempty[b],
-                                tmem + b * NMMA * BN + lane_base, BN, used, quarter, lane, rows, ystage,
+                                tmem + b * BN + lane_base, BN, used, quarter, lane, rows, ystage,
                                 abort_flag, epi_fail, last_flag, err))
         break;
-      c0 += nch;
       ++seg_i;
     }
   }

@@ -152,6 +152,14 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Zeroes 16 consecutive columns of this thread's lane.
+__device__ __forceinline__ void tmem_zero_16(uint32_t taddr) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1};" ::"r"(taddr),
+      "r"(0u)
+      : "memory");
+}
 // 32 lanes x 32 bits, 32 consecutive columns: register i -> column taddr+i of
 // this thread's lane.
 __device__ __forceinline__ void tmem_st_32(uint32_t taddr, const uint32_t (&r)[32]) {
