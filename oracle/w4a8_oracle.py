@@ -83,6 +83,31 @@ def quantize_act(A: np.ndarray):
     return A8, sA, rowsum
 
 
+def quantize_act_static(A: np.ndarray, s: np.float16):
+    """Per-tensor static symmetric int8 quantization of fp16 activations.
+
+    One fp16 scale s for the whole tensor, fixed offline by calibration
+    instead of measured per token at run time ("PrefixQuant: Static
+    Quantization Beats Dynamic through Prefixed Outliers in LLMs",
+    Methodology and Key Findings: per-tensor static quantization once the
+    outlier tokens are prefixed). Rounding and range as quantize_act:
+    A8 = clamp(rint(A / float(s)), -127, 127) with an fp32 divide (rint: half
+    to even); s == 0 gives all-zero codes. sA[m] = s for every token, so the
+    GEMM's per-token epilogue applies the tensor scale unchanged;
+    rowsum[m] = sum_k A8[m,k] (int32).
+
+    Returns (A8 int8 [M,K], sA fp16 [M], rowsum int32 [M]).
+    """
+    assert A.dtype == np.float16 and A.ndim == 2
+    sf = np.float32(np.float16(s))
+    A8 = np.zeros(A.shape, dtype=np.int8)
+    if sf != 0:
+        A8 = np.clip(np.rint(A.astype(np.float32) / sf), -127, 127).astype(np.int8)
+    sA = np.full(A.shape[0], np.float16(s), dtype=np.float16)
+    rowsum = A8.astype(np.int64).sum(axis=1).astype(np.int32)
+    return A8, sA, rowsum
+
+
 # ---------------------------------------------------------------------------
 # Progressive (two-level) weight quantization
 # ---------------------------------------------------------------------------

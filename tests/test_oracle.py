@@ -152,6 +152,59 @@ def test_quantize_codes_exact_rational():
     assert n_checked > 1000
 
 
+# ------------------------------------------------- static activation scale
+def test_static_quantize_codes_exact_rational():
+    """Static per-tensor codes: the integer nearest to A / s in exact
+    arithmetic (ties to even), clamped to [-127, 127] (so tokens with
+    |A| > 127.5 s saturate), except where A / s lies so close to a
+    half-integer that the fp32 quotient may round across it; sA repeats s
+    and rowsum sums the codes."""
+    A = _rand_act(5, 256, 14)
+    A[2] *= 40  # an outlier token: many codes saturate under the tensor scale
+    s = np.float16(0.0123)
+    A8, sA, rs = O.quantize_act_static(A, s)
+    assert (sA.view(np.uint16) == np.uint16(s.view(np.uint16))).all()
+    assert (rs == A8.astype(np.int64).sum(1)).all()
+    S = Fraction(float(s))
+    n_checked = n_clamped = 0
+    for m in range(A.shape[0]):
+        for k in range(A.shape[1]):
+            x = Fraction(float(A[m, k])) / S
+            frac = x - (x.numerator // x.denominator)
+            if abs(frac - Fraction(1, 2)) < Fraction(1, 10 ** 5):
+                continue
+            want = max(-127, min(127, _nearest_even(x)))
+            n_clamped += abs(want) == 127 and abs(x) > Fraction(255, 2)
+            assert int(A8[m, k]) == want, (m, k)
+            n_checked += 1
+    assert n_checked > 1200 and n_clamped > 50
+
+
+def test_static_quantize_reduces_to_dynamic_per_row():
+    """With the tensor scale set to a token's own dynamic scale, that
+    token's static codes are its dynamic codes (same rounding and range)."""
+    A = _rand_act(6, 512, 15)
+    A8d, sAd, rsd = O.quantize_act(A)
+    for m in range(A.shape[0]):
+        A8s, sAs, rss = O.quantize_act_static(A[m:m + 1], sAd[m])
+        assert (A8s[0] == A8d[m]).all() and rss[0] == rsd[m]
+        assert sAs[0].view(np.uint16) == sAd[m].view(np.uint16)
+
+
+def test_static_quantize_zero_scale_and_symmetry():
+    A = _rand_act(3, 128, 16)
+    A8, sA, rs = O.quantize_act_static(A, np.float16(0))
+    assert not A8.any() and not rs.any() and not sA.astype(np.float32).any()
+    s = np.float16(0.02)
+    A8p, _, rsp = O.quantize_act_static(A, s)
+    A8n, _, rsn = O.quantize_act_static(-A, s)
+    assert (A8n == -A8p).all() and (rsn == -rsp).all()  # rint is odd, the clamp symmetric
+    # power-of-two rescaling of both A and s leaves every code unchanged
+    s4 = np.float16(np.float32(s) * 4)  # exact: a power-of-two rescaling of an fp16 normal
+    A8q, _, _ = O.quantize_act_static((A.astype(np.float32) * 4).astype(np.float16), s4)
+    assert (A8q == A8p).all()
+
+
 # ------------------------------------------------------------- weights
 def test_dequant_full_domain_bytewise():
     """All 16*16*8 (q, z, s2): the oracle's W8 lies in [-120, 120] and equals
