@@ -302,6 +302,11 @@ def run_gpu(args, world, rank, local):
                            torch.empty((M,), dtype=torch.int32, device=dev),
                            torch.empty((M, N), dtype=torch.float16, device=dev))
     copy_of = {M: i for i, M in enumerate(wl.ms)}
+    static_scales = None
+    if args.act == "static":
+        # offline calibration: one scale per activation tensor, from its range
+        static_scales = {key: (A.float().abs().max() / 127).to(torch.float16).reshape(1)
+                         for key, A in acts.items()}
 
     def step(events=None, h2d=None, d2h=None, gemm_only=False):
         for i, (M, name, N, K) in enumerate(cases):
@@ -310,7 +315,10 @@ def run_gpu(args, world, rank, local):
                 A.copy_(h2d[(M, name)], non_blocking=True)
             A8, sA, rs, Y = outs[(M, name)]
             if not gemm_only:
-                w4a8.quantize_act(A, out=(A8, sA, rs))
+                if static_scales is not None:
+                    w4a8.quantize_act_static(A, static_scales[(M, name)], out=(A8, sA, rs))
+                else:
+                    w4a8.quantize_act(A, out=(A8, sA, rs))
             if events is not None:
                 events[i][0].record()
             w4a8.gemm(A8, sA, rs, blobs[(name, copy_of[M])], N, K, out=Y, workspace=ws)
@@ -431,6 +439,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cases", default=None,
                     help="subset of the workload's cases, e.g. 16:gate_up,1:o (profiling)")
+    ap.add_argument("--act", default="dynamic", choices=["dynamic", "static"],
+                    help="activation scales: per-token dynamic (w4a8_quantize_act), or one per-tensor static "
+                         "scale calibrated once before timing (w4a8_quantize_act_static)")
     ap.add_argument("--profile", type=int, default=0,
                     help="run this many eager steps for an external profiler and exit (no timing)")
     args = ap.parse_args()
@@ -494,7 +505,7 @@ def main():
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": args.workload, "cases": len(cases),
+        "config": {"workload": args.workload, "activation_scales": args.act, "cases": len(cases),
                    "shapes": [f"M={M} {n} {N}x{K}" for (M, n, N, K) in cases][:: max(1, len(cases) // 16)],
                    "group": 128, "weights_per_step_MB": round(wbytes / 1e6, 1),
                    "l2": f"inputs larger than L2: {r['n_copies']} weight copies, {wbytes / 1e6:.0f} MB per step",

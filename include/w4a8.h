@@ -90,6 +90,23 @@ W4A8_API w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, in
                                 w4a8_stream_t stream);
 
 /*
+ * Per-tensor static symmetric int8 quantization: one fp16 scale for the
+ * whole activation tensor, calibrated offline ("PrefixQuant: Static
+ * Quantization Beats Dynamic through Prefixed Outliers in LLMs",
+ * Methodology and Key Findings: per-tensor static quantization once the
+ * outlier tokens are prefixed). No amax pass:
+ *   A8[m,k] = clamp(rint(A[m,k] / float(s)), -127, 127)
+ *                                     (IEEE fp32 divide, ties to even)
+ *   s == 0 gives all-zero codes; rowsum[m] = sum_k A8[m,k]; sA[m] = s, so
+ *   the result feeds w4a8_gemm unchanged.
+ * s: device pointer to ONE fp16 value (read on the device, so a captured
+ * graph picks up a changed scale). Other arguments and limits as for
+ * w4a8_quantize_act.
+ */
+W4A8_API w4a8_status_t w4a8_quantize_act_static(const void* A, int64_t M, int64_t K, const void* s, int8_t* A8,
+                                                void* sA, int32_t* rowsum, w4a8_stream_t stream);
+
+/*
  * Offline two-level weight quantization (the "progressive quantization" of
  * the QServe/QoQ abstract), fp32 W [N, K] -> (q, z, s2, s1):
  *   level 1 (row n): r_g = max(max W_g, 0) - min(min W_g, 0) over each

@@ -68,6 +68,40 @@ def test_quantize_act_bit_exact(M, K):
     assert (host(rs) == ors).all()
 
 
+@pytest.mark.parametrize("M,K", [(1, 512), (3, 4096), (17, 14336), (5, 65536), (300, 1024), (2, 8)])
+@pytest.mark.parametrize("s", [0.0123, 1e-4, 0.0])
+def test_quantize_act_static_bit_exact(M, K, s):
+    """Per-tensor static quantization (outlier tokens saturate at +-127)."""
+    A = I.activations(M, K, I.seed_of("t-qas", M, K))
+    if K >= 8:
+        A = np.concatenate([A, special_rows(K)], axis=0)
+    sd = torch.tensor([s], dtype=torch.float16, device=DEV)
+    A8, sA, rs = w4a8.quantize_act_static(dev(A), sd)
+    torch.cuda.synchronize()
+    oA8, osA, ors = O.quantize_act_static(A, np.float16(s))
+    assert (host(A8) == oA8).all()
+    assert (host(sA).view(np.uint16) == osA.view(np.uint16)).all()
+    assert (host(rs) == ors).all()
+
+
+def test_static_quantization_through_the_gemm():
+    """Static activation codes feed the unchanged GEMM: bit-exact int32
+    accumulators and Y within 1 ulp of the oracle's static path."""
+    M, N, K = 20, 512, 1024
+    q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-sg", N, K))
+    A = I.activations(M, K, I.seed_of("t-sga", M, K))
+    s = np.float16(float(np.abs(A.astype(np.float32)).max()) / 127 / 4)  # a quarter of the tensor range: saturation
+    blob = gpu_path_from_codes(q, z, s2, s1)
+    A8, sA, rs = w4a8.quantize_act_static(dev(A), torch.tensor([float(s)], dtype=torch.float16, device=DEV))
+    acc = w4a8.gemm_debug_acc(A8, rs, blob, N, K)
+    Y = w4a8.gemm(A8, sA, rs, blob, N, K)
+    torch.cuda.synchronize()
+    oA8, osA, _ = O.quantize_act_static(A, s)
+    oacc = O.gemm_acc(oA8, O.dequant_weights(q, z, s2))
+    assert (host(acc) == oacc).all()
+    assert max_ulp_fp16(host(Y), O.epilogue(oacc, osA, s1)) <= 1
+
+
 def test_quantize_act_empty():
     A = torch.empty((0, 256), dtype=torch.float16, device=DEV)
     A8, sA, rs = w4a8.quantize_act(A)

@@ -79,6 +79,15 @@ def test_quantize_act_validation(L):
     assert f(FAKE, 0, 128, None, None, None, None) == 0      # M == 0: no-op
 
 
+def test_quantize_act_static_validation(L):
+    f = L.w4a8_quantize_act_static
+    assert f(FAKE, 4, 7, FAKE, FAKE, FAKE, None, None) == 2        # K % 8
+    assert f(FAKE, 4, 128, None, FAKE, FAKE, None, None) == 1      # no scale
+    assert f(FAKE, 4, 128, FAKE_ODD, FAKE, FAKE, None, None) == 3  # scale alignment
+    assert f(FAKE_ODD, 4, 128, FAKE, FAKE, FAKE, None, None) == 3
+    assert f(FAKE, 0, 128, None, None, None, None, None) == 0      # M == 0: no-op
+
+
 def test_quantize_weights_validation(L):
     f = L.w4a8_quantize_weights
     assert f(FAKE, 128, 100, 128, FAKE, FAKE, FAKE, FAKE, None) == 2

@@ -19,7 +19,7 @@ __all__ = [
     "W4A8Error", "lib", "library_path", "EXPORTED_SYMBOLS", "status_string", "quantize_act",
     "quantize_weights", "packed_bytes", "pack_weights", "workspace_bytes", "Workspace", "gemm",
     "gemm_debug_acc", "gemm_ex", "gemm_noalloc", "get_device_error", "clear_device_error",
-    "selftest_bounded_wait",
+    "selftest_bounded_wait", "quantize_act_static",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +29,7 @@ EXPORTED_SYMBOLS = (
     "w4a8_status_string", "w4a8_version", "w4a8_quantize_act", "w4a8_quantize_weights",
     "w4a8_packed_bytes", "w4a8_pack_weights", "w4a8_gemm_workspace_bytes", "w4a8_gemm",
     "w4a8_gemm_debug_acc", "w4a8_gemm_ex", "w4a8_get_device_error", "w4a8_clear_device_error",
-    "w4a8_gemm_noalloc", "w4a8_selftest_bounded_wait",
+    "w4a8_gemm_noalloc", "w4a8_selftest_bounded_wait", "w4a8_quantize_act_static",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
         "w4a8_clear_device_error": (ctypes.c_int, [vp]),
         "w4a8_gemm_noalloc": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp]),
         "w4a8_selftest_bounded_wait": (ctypes.c_int, [i64, vp]),
+        "w4a8_quantize_act_static": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -132,6 +133,26 @@ def quantize_act(A, out=None):
         _require_cuda(A8, sA, rowsum)
     _check(lib().w4a8_quantize_act(_ptr(A), M, K, _ptr(A8), _ptr(sA), _ptr(rowsum), _stream(A.device)),
            "w4a8_quantize_act")
+    return A8, sA, rowsum
+
+
+def quantize_act_static(A, s, out=None):
+    """Per-tensor static quantization with the fp16 scale `s` (a 1-element
+    CUDA tensor): fp16 [M, K] -> (A8 int8 [M, K], sA fp16 [M] = s, rowsum int32 [M])."""
+    torch = _torch()
+    _require_cuda(A, s)
+    if A.dtype != torch.float16 or A.dim() != 2 or s.dtype != torch.float16 or s.numel() != 1:
+        raise W4A8Error("A must be a 2-D fp16 tensor and s a 1-element fp16 tensor")
+    M, K = A.shape
+    if out is None:
+        A8 = torch.empty((M, K), dtype=torch.int8, device=A.device)
+        sA = torch.empty((M,), dtype=torch.float16, device=A.device)
+        rowsum = torch.empty((M,), dtype=torch.int32, device=A.device)
+    else:
+        A8, sA, rowsum = out
+        _require_cuda(A8, sA, rowsum)
+    _check(lib().w4a8_quantize_act_static(_ptr(A), M, K, _ptr(s), _ptr(A8), _ptr(sA), _ptr(rowsum),
+                                          _stream(A.device)), "w4a8_quantize_act_static")
     return A8, sA, rowsum
 
 

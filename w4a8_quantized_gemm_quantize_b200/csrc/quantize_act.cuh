@@ -115,4 +115,56 @@ __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __r
   if (threadIdx.x == 0) sA[m] = s_h;
 }
 
+// Per-tensor static int8 quantization: one fp16 scale s for the whole tensor,
+// fixed offline by calibration ("PrefixQuant: Static Quantization Beats
+// Dynamic through Prefixed Outliers in LLMs", Methodology: per-tensor static
+// quantization once outlier tokens are prefixed). No amax pass: one read of
+// A, A8 = clamp(rint(A / float(s)), -127, 127) (IEEE fp32 divide, ties to
+// even; s == 0 gives zero codes), rowsum, and sA[m] = s so that the GEMM's
+// per-token epilogue applies the tensor scale. One CTA per token.
+template <int THREADS, int VPT>
+__global__ void __launch_bounds__(THREADS) quantize_act_static_kernel(const __half* __restrict__ A, int64_t K,
+                                                                       const __half* __restrict__ s,
+                                                                       int8_t* __restrict__ A8,
+                                                                       __half* __restrict__ sA,
+                                                                       int32_t* __restrict__ rowsum) {
+  __shared__ int ird[32];
+  grid_dependency_wait();  // A (and s) may come from the preceding kernel
+  grid_launch_dependents();
+  const int64_t m = blockIdx.x;
+  const __half s_h = *s;
+  const float sf = __half2float(s_h);
+  const uint4* row = reinterpret_cast<const uint4*>(A + m * K);
+  uint2* out = reinterpret_cast<uint2*>(A8 + m * K);
+  const int nvec = static_cast<int>(K >> 3);
+  int local = 0;
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int idx = threadIdx.x + i * THREADS;
+    // the address is clamped into the row: the load may be issued ahead of
+    // the bounds test
+    const uint4 v = __ldcs(row + (idx < nvec ? idx : nvec - 1));
+    if (idx < nvec) {
+      const __half2* h = reinterpret_cast<const __half2*>(&v);
+      uint32_t packed[2] = {0u, 0u};
+      if (sf != 0.0f) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float2 f = __half22float2(h[j]);
+          const int q0 = quant_one(f.x, sf), q1 = quant_one(f.y, sf);
+          local += q0 + q1;
+          packed[j >> 1] |= ((static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8))
+                            << ((j & 1) * 16);
+        }
+      }
+      out[idx] = make_uint2(packed[0], packed[1]);
+    }
+  }
+  if (rowsum != nullptr) {
+    const int total = block_sum<THREADS>(local, ird);
+    if (threadIdx.x == 0) rowsum[m] = total;
+  }
+  if (threadIdx.x == 0) sA[m] = s_h;
+}
+
 }  // namespace w4a8

@@ -341,6 +341,29 @@ w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, int8_t* A8,
   return launch_pdl(quantize_act_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, A8, s, rowsum);
 }
 
+w4a8_status_t w4a8_quantize_act_static(const void* A, int64_t M, int64_t K, const void* s, int8_t* A8, void* sA,
+                                       int32_t* rowsum, w4a8_stream_t stream) {
+  if (M < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if (K == 0 || K % 8 != 0 || K > kMaxK || M > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return W4A8_OK;
+  if (A == nullptr || s == nullptr || A8 == nullptr || sA == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(A8, 16) || !aligned(s, 2) || !aligned(sA, 2) || !aligned(rowsum, 4))
+    return W4A8_ERR_MISALIGNED;
+  const __half* a = static_cast<const __half*>(A);
+  const __half* sc = static_cast<const __half*>(s);
+  __half* so = static_cast<__half*>(sA);
+  const dim3 grid(static_cast<unsigned>(M));
+  const int64_t nvec = K / 8;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (nvec <= 128)
+    return launch_pdl(quantize_act_static_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, sc, A8, so, rowsum);
+  if (nvec <= 512)
+    return launch_pdl(quantize_act_static_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum);
+  if (nvec <= 2048)
+    return launch_pdl(quantize_act_static_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum);
+  return launch_pdl(quantize_act_static_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, sc, A8, so, rowsum);
+}
+
 w4a8_status_t w4a8_quantize_weights(const float* W, int64_t N, int64_t K, int32_t group, uint8_t* q, uint8_t* z,
                                     uint8_t* s2, void* s1, w4a8_stream_t stream) {
   if (N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
