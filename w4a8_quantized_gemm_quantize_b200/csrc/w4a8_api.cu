@@ -180,8 +180,8 @@ w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs a
 // Tile configurations: tokens per tile, k-blocks per chunk, weight and
 // activation ring slots, TMEM ring slots, dequantizer groups, accumulator
 // buffers, MMA issuers.
-using Cfg16 = GemmCfg<16, 4, 5, 3, 1, 2, 2>;
-using Cfg32 = GemmCfg<32, 4, 4, 3, 1, 2, 2>;
+using Cfg16 = GemmCfg<16, 4, 5, 3, 2, 2, 2>;
+using Cfg32 = GemmCfg<32, 4, 4, 3, 2, 2, 2>;
 using Cfg64 = GemmCfg<64, 2, 6, 6, 2, 2, 2>;
 using Cfg128 = GemmCfg<128, 4, 2, 2, 1, 2, 2>;
 
