@@ -27,6 +27,14 @@
  *    thereby clearing) the CUDA runtime's last error.
  *  - Data pointers must be 16-byte aligned unless stated otherwise.
  *  - Matrices are row-major and dense (leading dimension = row length).
+ *  - The activation quantizers and the GEMM launch as programmatic
+ *    dependents of the preceding kernel in the stream: they may start while
+ *    it still runs and wait for it to complete before they read or write
+ *    anything of it, with one exception: the GEMM starts reading the packed
+ *    weight blob at once. The blob must therefore be complete before the
+ *    kernel just ahead of the GEMM in the stream starts (w4a8_pack_weights
+ *    and any ordinary kernel or copy satisfy this; only a kernel that itself
+ *    releases its dependents early could break it, by writing the blob).
  */
 #ifndef W4A8_H_
 #define W4A8_H_

@@ -93,9 +93,17 @@ struct Sched {
       return;
     }
     if (a.sk_tiles > 0) {
-      const int64_t U = static_cast<int64_t>(a.sk_tiles) * KB;
-      u = U * blockIdx.x / gridDim.x;
-      u_end = U * (blockIdx.x + 1) / gridDim.x;
+      // 32-bit divisions when the products fit (64-bit division is a long
+      // software sequence on the critical start-up path)
+      const uint64_t U = static_cast<uint64_t>(a.sk_tiles) * static_cast<uint64_t>(KB);
+      const uint64_t lo = U * blockIdx.x, hi = U * (blockIdx.x + 1);
+      if (hi <= 0xFFFFFFFFull) {
+        u = static_cast<uint32_t>(lo) / gridDim.x;
+        u_end = static_cast<uint32_t>(hi) / gridDim.x;
+      } else {
+        u = static_cast<int64_t>(lo / gridDim.x);
+        u_end = static_cast<int64_t>(hi / gridDim.x);
+      }
     }
     tile_it = a.sk_tiles + static_cast<int>(blockIdx.x);
   }
@@ -110,7 +118,8 @@ struct Sched {
       return true;
     }
     if (u < u_end) {
-      s.tile = static_cast<int>(u / KB);
+      s.tile = u <= 0xFFFFFFFFll ? static_cast<int>(static_cast<uint32_t>(u) / static_cast<uint32_t>(KB))
+                                 : static_cast<int>(u / KB);
       s.kb0 = static_cast<int>(u - static_cast<int64_t>(s.tile) * KB);
       const int64_t left = u_end - u;
       s.kb1 = left < static_cast<int64_t>(KB - s.kb0) ? s.kb0 + static_cast<int>(left) : KB;
@@ -134,11 +143,13 @@ struct GemmCfg {
   // fixed latencies of the synchronization operations).
   //   warp 0        weight producer (one thread) and TMEM owner
   //   warps 1..     NMMA MMA issuers (one thread each), chunk c goes to
-  //                 issuer c % NMMA, which accumulates into a partial
-  //                 accumulator of its own; the epilogue adds the partials.
-  //                 With two issuers one thread's barrier waits and commits
-  //                 overlap the other's MMAs, so the tensor pipe does not
-  //                 idle between chunks when the MMAs are thin (small BN).
+  //                 issuer c % NMMA; both accumulate into the segment's one
+  //                 accumulator buffer. With two issuers one thread's
+  //                 barrier waits and commits overlap the other's MMAs, so
+  //                 the tensor pipe does not idle between chunks when the
+  //                 MMAs are thin (small BN).
+  //   warp 1 lane 0 also issues the first kStartChunks weight copies at
+  //                 kernel entry, before the rest of the set-up
   //   warp 3        activation producer (one thread)
   //   warps 4..     DQ dequantizer warpgroups, chunk c goes to group c % DQ
   //   last 4 warps  epilogue
@@ -151,10 +162,16 @@ struct GemmCfg {
   static constexpr int kA8Bytes = BN * 128;        // one k-block of activations
   static constexpr int kASlot = KS * kA8Bytes;
   static constexpr int kWSlot = KS * kTileBytes;   // KS consecutive packed tiles
-  static constexpr int kTmemCols = 512;
   static_assert(NMMA == 1 || NMMA == 2, "one or two MMA issuers (warps 1 and 2)");
+  // Weight chunks requested at kernel entry. Two, not the whole ring: when
+  // every CTA of a launch requests its whole ring at once, the first chunk of
+  // each waits behind everyone's burst in the memory queues (measured: a
+  // full-ring start delayed the first weight bytes by ~1 us per launch).
+  static constexpr int kStartChunks = NS < 2 ? NS : 2;
   static constexpr int kTmemA = NACC * BN;  // accumulators first, then the TMEM weight ring
   static constexpr int kTSlotCols = KS * 32;
+  // tensor memory columns allocated (a power of two >= 32)
+  static constexpr int kTmemCols = kTmemA + NT * kTSlotCols <= 256 ? 256 : 512;
   static_assert(kTmemA + NT * kTSlotCols <= kTmemCols, "tensor memory budget");
   static_assert(NT > DQ, "every dequantizer group needs a TMEM slot of its own");
   static_assert(NS >= 2 && NT >= 2, "two slots per ring at least");
@@ -511,10 +528,37 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const DevErr err{args.err};
 
+  if (warp == 1) {
+    // Weight starter: the weights do not come from the preceding kernel, so
+    // the first kStartChunks chunks' copies go out before the rest of the
+    // set-up (barriers, tensor memory, the CTA barrier). The weight producer
+    // skips these chunks.
+    if (lane == 0) {
+      for (int i = 0; i < NS; ++i) {
+        mbar_init(&wfull[i], 1);
+        mbar_init(&wempty[i], 4);
+      }
+      fence_barrier_init();
+      fence_proxy_async_smem();
+      const uint64_t pol_w = l2_policy_evict_first();
+      Sched s0;
+      s0.init(args);
+      Seg g0;
+      int c = 0;
+      while (c < C::kStartChunks && s0.next(g0)) {
+        const uint8_t* wsrc = args.tiles + static_cast<int64_t>(g0.tile / args.m_tiles) * args.KB * kTileBytes;
+        for (int kb = g0.kb0; kb < g0.kb1 && c < C::kStartChunks; kb += KS, ++c) {
+          const int cnt = min(KS, g0.kb1 - kb);
+          mbar_arrive_expect_tx(&wfull[c], cnt * kTileBytes);
+          bulk_load(sW + c * C::kWSlot, wsrc + static_cast<int64_t>(kb) * kTileBytes, cnt * kTileBytes, &wfull[c],
+                    pol_w);
+        }
+      }
+    }
+    __syncwarp();
+  }
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
-      mbar_init(&wfull[i], 1);
-      mbar_init(&wempty[i], 4);
       mbar_init(&afull[i], 1);
       mbar_init(&aempty[i], 1);
     }
@@ -559,9 +603,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
 
   if (warp == 0) {
     // ----------------------------------------------------- weight producer
-    // The weights do not come from the preceding kernel, so they start
-    // streaming before the dependency wait. One copy per chunk: the packed
-    // tiles of consecutive k-blocks of a tile are contiguous.
+    // The weights do not come from the preceding kernel, so they stream
+    // without the dependency wait. One copy per chunk: the packed tiles of
+    // consecutive k-blocks of a tile are contiguous. The first kStartChunks
+    // chunks were issued by the weight starter at kernel entry.
     if (lane == 0) {
       const uint64_t pol_w = l2_policy_evict_first();
       int c = 0;
@@ -569,6 +614,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       while (ok && sch.next(sg)) {
         const uint8_t* wsrc = args.tiles + static_cast<int64_t>(sg.tile / args.m_tiles) * args.KB * kTileBytes;
         for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
+          if (c < C::kStartChunks) continue;
           const int cnt = min(KS, sg.kb1 - kb);
           const int w = c % NS;
           if (!mbar_wait(&wempty[w], ((c / NS) & 1) ^ 1, abort_flag, err, kErrProducer)) {
@@ -580,6 +626,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
                     pol_w);
         }
       }
+      // Every weight byte of this CTA is requested: the next kernel in the
+      // stream may launch and start its own weight stream on the SMs this
+      // grid frees (it waits for this grid to complete before it touches
+      // anything this grid reads or writes).
+      grid_launch_dependents();
       // copies still in flight must land before the CTA exits
       const int first = c - NS > 0 ? c - NS : 0;
       for (int i = first; i < c; ++i) mbar_wait(&wfull[i % NS], (i / NS) & 1, nullptr, err, kErrDrain);
@@ -654,8 +705,6 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
         mma_commit(&accfull[b]);
         ++seg_i;
       }
-      // the next kernel in the stream may start its prologue now
-      grid_launch_dependents();
       // every issued MMA must finish before TMEM is released
       mma_commit(done);
       mbar_wait(done, 0, nullptr, err, kErrDrain);
@@ -664,8 +713,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
   } else if (warp >= C::kDqWarp0 && warp < C::kDqWarp0 + 4 * DQ) {
     // --------------------------------------------------------- dequantizers
     // Group g takes chunks c = g (mod DQ). The weight slot is released as
-    // soon as it has been read; the TMEM stores of a chunk stay in flight
-    // while the group loads and unpacks its next chunk.
+    // soon as it has been read; with pipelined stores the TMEM stores of a
+    // chunk stay in flight while the group loads and unpacks its next chunk.
     const int g = (warp - C::kDqWarp0) >> 2;
     const int quarter = warp & 3;  // TMEM lane quarter this warp may access
     const int r = quarter * 32 + lane;

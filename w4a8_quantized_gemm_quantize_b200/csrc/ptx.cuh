@@ -66,12 +66,18 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, 
                                                 DevErr err, int code, uint64_t limit_ns) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 31u) == 0) {
       if (abort_flag != nullptr && *abort_flag) return false;
-      if (global_timer_ns() - t0 > limit_ns) {
+      const uint64_t now = global_timer_ns();
+      // The global timer is not guaranteed monotonic (the driver may step
+      // it): after a backward step the unsigned difference would wrap to a
+      // huge value and end a healthy wait at once, so restart the interval.
+      if (now < t0) {
+        t0 = now;
+      } else if (now - t0 > limit_ns) {
         if (abort_flag != nullptr) *abort_flag = 1;
         atomicCAS(err.word, 0, code);
         return false;

@@ -59,10 +59,12 @@ __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __r
                                                                 int32_t* __restrict__ rowsum) {
   __shared__ float fred[32];
   __shared__ int ird[32];
-  // launched as a programmatic dependent: wait for the preceding kernel's
-  // writes, then let the next kernel (the GEMM) start its prologue
-  grid_dependency_wait();
+  // launched as a programmatic dependent: the next kernel (the GEMM) may
+  // launch right away and stream its weights while this grid runs (it waits
+  // for this grid to complete before it reads the codes); this grid waits
+  // for the preceding kernel's writes before it reads A
   grid_launch_dependents();
+  grid_dependency_wait();
   int* ired = ird;
   const int64_t m = blockIdx.x;
   const uint4* row = reinterpret_cast<const uint4*>(A + m * K);
@@ -129,8 +131,8 @@ __global__ void __launch_bounds__(THREADS) quantize_act_static_kernel(const __ha
                                                                        __half* __restrict__ sA,
                                                                        int32_t* __restrict__ rowsum) {
   __shared__ int ird[32];
-  grid_dependency_wait();  // A (and s) may come from the preceding kernel
-  grid_launch_dependents();
+  grid_launch_dependents();  // as in quantize_act_kernel
+  grid_dependency_wait();    // A (and s) may come from the preceding kernel
   const int64_t m = blockIdx.x;
   const __half s_h = *s;
   const float sf = __half2float(s_h);

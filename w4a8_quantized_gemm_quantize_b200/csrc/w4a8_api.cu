@@ -117,7 +117,7 @@ w4a8_status_t ctas_per_sm(int dev, int* out) {
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, w4a8_gemm_kernel<C>, C::kThreads, C::kSmemBytes) !=
         cudaSuccess)
       return launch_status();
-    n = n < 512 / C::kTmemCols ? n : 512 / C::kTmemCols;  // every resident CTA must get its TMEM (one)
+    n = n < 512 / C::kTmemCols ? n : 512 / C::kTmemCols;  // every resident CTA must get its TMEM
     cache[dev] = n > 0 ? n : 1;
   }
   *out = cache[dev];
@@ -245,7 +245,7 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum,
       int nclu = 0;
       st = bn == 16 ? max_clusters<Cfg16>(dev_id, S, &nclu) : max_clusters<Cfg32>(dev_id, S, &nclu);
       if (st != W4A8_OK) return st;
-      if (num_tiles <= nclu) split = S;
+      if (num_tiles <= nclu && num_tiles * S <= max_ctas) split = S;
     }
   }
   if (o.schedule == 3 && split == 1) return W4A8_ERR_UNSUPPORTED_SHAPE;
