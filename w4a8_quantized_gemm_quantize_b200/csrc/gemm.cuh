@@ -93,17 +93,9 @@ struct Sched {
       return;
     }
     if (a.sk_tiles > 0) {
-      // 32-bit divisions when the products fit (64-bit division is a long
-      // software sequence on the critical start-up path)
-      const uint64_t U = static_cast<uint64_t>(a.sk_tiles) * static_cast<uint64_t>(KB);
-      const uint64_t lo = U * blockIdx.x, hi = U * (blockIdx.x + 1);
-      if (hi <= 0xFFFFFFFFull) {
-        u = static_cast<uint32_t>(lo) / gridDim.x;
-        u_end = static_cast<uint32_t>(hi) / gridDim.x;
-      } else {
-        u = static_cast<int64_t>(lo / gridDim.x);
-        u_end = static_cast<int64_t>(hi / gridDim.x);
-      }
+      const int64_t U = static_cast<int64_t>(a.sk_tiles) * KB;
+      u = U * blockIdx.x / gridDim.x;
+      u_end = U * (blockIdx.x + 1) / gridDim.x;
     }
     tile_it = a.sk_tiles + static_cast<int>(blockIdx.x);
   }
@@ -118,8 +110,7 @@ struct Sched {
       return true;
     }
     if (u < u_end) {
-      s.tile = u <= 0xFFFFFFFFll ? static_cast<int>(static_cast<uint32_t>(u) / static_cast<uint32_t>(KB))
-                                 : static_cast<int>(u / KB);
+      s.tile = static_cast<int>(u / KB);
       s.kb0 = static_cast<int>(u - static_cast<int64_t>(s.tile) * KB);
       const int64_t left = u_end - u;
       s.kb1 = left < static_cast<int64_t>(KB - s.kb0) ? s.kb0 + static_cast<int>(left) : KB;
@@ -163,11 +154,19 @@ struct GemmCfg {
   static constexpr int kASlot = KS * kA8Bytes;
   static constexpr int kWSlot = KS * kTileBytes;   // KS consecutive packed tiles
   static_assert(NMMA == 1 || NMMA == 2, "one or two MMA issuers (warps 1 and 2)");
+  // Launch overlap for the small-token (decode) configurations, whose
+  // launches are short enough for start-up and hand-over latency to matter:
+  // the first weight chunks are requested at kernel entry, and the next
+  // kernel in the stream is released as soon as every weight byte of the
+  // grid has been requested. The large-token configurations release it after
+  // their last MMA and start the weight stream after the set-up (measured
+  // faster for their long launches).
+  static constexpr bool kEarlyStart = BN <= 32;
   // Weight chunks requested at kernel entry. Two, not the whole ring: when
   // every CTA of a launch requests its whole ring at once, the first chunk of
   // each waits behind everyone's burst in the memory queues (measured: a
   // full-ring start delayed the first weight bytes by ~1 us per launch).
-  static constexpr int kStartChunks = NS < 2 ? NS : 2;
+  static constexpr int kStartChunks = kEarlyStart ? (NS < 2 ? NS : 2) : 0;
   static constexpr int kTmemA = NACC * BN;  // accumulators first, then the TMEM weight ring
   static constexpr int kTSlotCols = KS * 32;
   // tensor memory columns allocated (a power of two >= 32)
@@ -524,9 +523,10 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   volatile int* last_flag = reinterpret_cast<volatile int*>(misc + 2);
   volatile int* epi_fail = reinterpret_cast<volatile int*>(misc + 3);
+  volatile int* dep_done = reinterpret_cast<volatile int*>(misc + 4);  // dependency wait passed
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const DevErr err{args.err};
+  const DevErr err{args.err, dep_done};
 
   if (warp == 1) {
     // Weight starter: the weights do not come from the preceding kernel, so
@@ -580,6 +580,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     misc[1] = 0;
     misc[2] = 0;
     misc[3] = 0;
+    misc[4] = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
@@ -630,7 +631,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       // stream may launch and start its own weight stream on the SMs this
       // grid frees (it waits for this grid to complete before it touches
       // anything this grid reads or writes).
-      grid_launch_dependents();
+      if (C::kEarlyStart) grid_launch_dependents();
       // copies still in flight must land before the CTA exits
       const int first = c - NS > 0 ? c - NS : 0;
       for (int i = first; i < c; ++i) mbar_wait(&wfull[i % NS], (i / NS) & 1, nullptr, err, kErrDrain);
@@ -640,6 +641,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     // ------------------------------------------------- activation producer
     if (lane == 0) {
       grid_dependency_wait();  // the activation tiles come from the preceding kernel
+      *dep_done = 1;           // the time limits of the CTA's waits start counting
       int c = 0;
       bool ok = true;
       while (ok && sch.next(sg)) {
@@ -705,6 +707,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
         mma_commit(&accfull[b]);
         ++seg_i;
       }
+      // the next kernel in the stream may start its prologue now
+      if (!C::kEarlyStart) grid_launch_dependents();
       // every issued MMA must finish before TMEM is released
       mma_commit(done);
       mbar_wait(done, 0, nullptr, err, kErrDrain);

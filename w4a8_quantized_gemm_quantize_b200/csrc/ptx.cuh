@@ -10,9 +10,15 @@
 namespace w4a8 {
 
 // Device-side error word: 0 = fine; otherwise the code of the first wait that
-// gave up (see the W4A8_DEVERR_* values in the public header).
+// gave up (see the W4A8_DEVERR_* values in the public header). `armed`
+// (shared memory, optional) holds 0 until the CTA has passed its
+// programmatic-dependency wait: until then a wait may legitimately last as
+// long as the preceding kernel runs (every wait of a GEMM CTA depends, through
+// the pipeline, on the activations that kernel writes), so its time limit
+// only starts counting once the flag is set.
 struct DevErr {
   int* word;
+  const volatile int* armed = nullptr;
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -59,8 +65,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Waits for the phase with the given parity to complete. Returns false if
-// the CTA's abort flag (when given) is set, or once `limit_ns` passes; then it
-// sets the flag (when given) and records `code` in the device error word.
+// the CTA's abort flag (when given) is set, or once `limit_ns` passes (counted
+// from when the CTA is armed, see DevErr); then it sets the flag (when given)
+// and records `code` in the device error word.
 // Without an abort flag the wait only ends by completion or time.
 __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                 DevErr err, int code, uint64_t limit_ns) {
@@ -72,10 +79,10 @@ __device__ __forceinline__ bool mbar_wait_limit(uint64_t* bar, uint32_t parity, 
     if ((it & 31u) == 0) {
       if (abort_flag != nullptr && *abort_flag) return false;
       const uint64_t now = global_timer_ns();
-      // The global timer is not guaranteed monotonic (the driver may step
-      // it): after a backward step the unsigned difference would wrap to a
-      // huge value and end a healthy wait at once, so restart the interval.
-      if (now < t0) {
+      // The interval restarts while the CTA is not armed yet, and after a
+      // backward step of the global timer (not guaranteed monotonic: the
+      // unsigned difference would wrap and end a healthy wait at once).
+      if (now < t0 || (err.armed != nullptr && *err.armed == 0)) {
         t0 = now;
       } else if (now - t0 > limit_ns) {
         if (abort_flag != nullptr) *abort_flag = 1;

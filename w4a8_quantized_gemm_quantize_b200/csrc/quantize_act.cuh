@@ -56,15 +56,18 @@ __device__ __forceinline__ int quant_one(float x, float sf) {
 template <int THREADS, int VPT>
 __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __restrict__ A, int64_t K,
                                                                 int8_t* __restrict__ A8, __half* __restrict__ sA,
-                                                                int32_t* __restrict__ rowsum) {
+                                                                int32_t* __restrict__ rowsum, int early_release) {
   __shared__ float fred[32];
   __shared__ int ird[32];
-  // launched as a programmatic dependent: the next kernel (the GEMM) may
-  // launch right away and stream its weights while this grid runs (it waits
-  // for this grid to complete before it reads the codes); this grid waits
-  // for the preceding kernel's writes before it reads A
-  grid_launch_dependents();
+  // Launched as a programmatic dependent: this grid waits for the preceding
+  // kernel's writes before it reads A. With early_release (few tokens, a
+  // grid of a few CTAs) the next kernel (the GEMM) may launch right away and
+  // stream its weights while this grid runs; it waits for this grid to
+  // complete before it reads the codes. A grid of thousands of rows releases
+  // it after its wait instead, so that its CTAs do not hold SM slots early.
+  if (early_release) grid_launch_dependents();
   grid_dependency_wait();
+  if (!early_release) grid_launch_dependents();
   int* ired = ird;
   const int64_t m = blockIdx.x;
   const uint4* row = reinterpret_cast<const uint4*>(A + m * K);
@@ -129,10 +132,12 @@ __global__ void __launch_bounds__(THREADS) quantize_act_static_kernel(const __ha
                                                                        const __half* __restrict__ s,
                                                                        int8_t* __restrict__ A8,
                                                                        __half* __restrict__ sA,
-                                                                       int32_t* __restrict__ rowsum) {
+                                                                       int32_t* __restrict__ rowsum,
+                                                                       int early_release) {
   __shared__ int ird[32];
-  grid_launch_dependents();  // as in quantize_act_kernel
-  grid_dependency_wait();    // A (and s) may come from the preceding kernel
+  if (early_release) grid_launch_dependents();  // as in quantize_act_kernel
+  grid_dependency_wait();                       // A (and s) may come from the preceding kernel
+  if (!early_release) grid_launch_dependents();
   const int64_t m = blockIdx.x;
   const __half s_h = *s;
   const float sf = __half2float(s_h);

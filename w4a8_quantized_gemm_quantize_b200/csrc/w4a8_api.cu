@@ -22,6 +22,9 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 constexpr int64_t kMaxK = 65536;
+// Activation quantizers with at most this many rows (one CTA per row) release
+// the next kernel before their dependency wait (see quantize_act.cuh).
+constexpr int64_t kEarlyReleaseRows = 64;
 
 struct DeviceInfo {
   bool ready = false;
@@ -330,15 +333,16 @@ w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, int8_t* A8,
   const __half* a = static_cast<const __half*>(A);
   __half* s = static_cast<__half*>(sA);
   const dim3 grid(static_cast<unsigned>(M));
+  const int early = M <= kEarlyReleaseRows ? 1 : 0;
   const int64_t nvec = K / 8;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (nvec <= 128) return launch_pdl(quantize_act_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, A8, s, rowsum);
-  if (nvec <= 256) return launch_pdl(quantize_act_kernel<256, 1>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
-  if (nvec <= 512) return launch_pdl(quantize_act_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
-  if (nvec <= 1024) return launch_pdl(quantize_act_kernel<256, 4>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
-  if (nvec <= 2048) return launch_pdl(quantize_act_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum);
-  if (nvec <= 4096) return launch_pdl(quantize_act_kernel<512, 8>, grid, dim3(512), 0, st, 1, a, K, A8, s, rowsum);
-  return launch_pdl(quantize_act_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, A8, s, rowsum);
+  if (nvec <= 128) return launch_pdl(quantize_act_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, A8, s, rowsum, early);
+  if (nvec <= 256) return launch_pdl(quantize_act_kernel<256, 1>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
+  if (nvec <= 512) return launch_pdl(quantize_act_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
+  if (nvec <= 1024) return launch_pdl(quantize_act_kernel<256, 4>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
+  if (nvec <= 2048) return launch_pdl(quantize_act_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
+  if (nvec <= 4096) return launch_pdl(quantize_act_kernel<512, 8>, grid, dim3(512), 0, st, 1, a, K, A8, s, rowsum, early);
+  return launch_pdl(quantize_act_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, A8, s, rowsum, early);
 }
 
 w4a8_status_t w4a8_quantize_act_static(const void* A, int64_t M, int64_t K, const void* s, int8_t* A8, void* sA,
@@ -353,15 +357,16 @@ w4a8_status_t w4a8_quantize_act_static(const void* A, int64_t M, int64_t K, cons
   const __half* sc = static_cast<const __half*>(s);
   __half* so = static_cast<__half*>(sA);
   const dim3 grid(static_cast<unsigned>(M));
+  const int early = M <= kEarlyReleaseRows ? 1 : 0;
   const int64_t nvec = K / 8;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   if (nvec <= 128)
-    return launch_pdl(quantize_act_static_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, sc, A8, so, rowsum);
+    return launch_pdl(quantize_act_static_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, sc, A8, so, rowsum, early);
   if (nvec <= 512)
-    return launch_pdl(quantize_act_static_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum);
+    return launch_pdl(quantize_act_static_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum, early);
   if (nvec <= 2048)
-    return launch_pdl(quantize_act_static_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum);
-  return launch_pdl(quantize_act_static_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, sc, A8, so, rowsum);
+    return launch_pdl(quantize_act_static_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum, early);
+  return launch_pdl(quantize_act_static_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, sc, A8, so, rowsum, early);
 }
 
 w4a8_status_t w4a8_quantize_weights(const float* W, int64_t N, int64_t K, int32_t group, uint8_t* q, uint8_t* z,
