@@ -26,6 +26,9 @@ What the pages fix and what this file reads into them
 * Activations: 8-bit, per-token symmetric with a dynamic scale (the dynamic
   per-token baseline that "PrefixQuant: Static Quantization Beats Dynamic
   through Prefixed Outliers in LLMs" compares against, Key Findings).
+* 4-bit activations (W4A4): the W4A4KV4 models of "PrefixQuant ..." (Key
+  Findings) with per-tensor static scales; readings of the 4-bit code range,
+  rounding and nibble order are stated at `quantize_act4`.
 * Offline weight reordering ("QServe/QoQ" abstract: compute-aware weight
   reordering; "QUICK: Quantization-aware Interleaving and Conflict-free
   Kernel ...", abstract: offline interleaving; "Fast Matrix Multiplications
@@ -106,6 +109,80 @@ def quantize_act_static(A: np.ndarray, s: np.float16):
     sA = np.full(A.shape[0], np.float16(s), dtype=np.float16)
     rowsum = A8.astype(np.int64).sum(axis=1).astype(np.int32)
     return A8, sA, rowsum
+
+
+# ---------------------------------------------------------------------------
+# 4-bit activations (W4A4)
+# ---------------------------------------------------------------------------
+# "PrefixQuant: Static Quantization Beats Dynamic through Prefixed Outliers
+# in LLMs" (Key Findings) runs W4A4KV4 models: 4-bit weights against 4-bit
+# activations, with per-tensor static activation scales once the outlier
+# tokens are prefixed. The pages fix no code range, rounding or storage for
+# the 4-bit activations; the readings here are the 8-bit scheme's with the
+# symmetric 4-bit range: codes in [-7, 7] (-8 never occurs), rint half to even
+# of A / float(s) with an fp32 divide, per-tensor static s (the pages'
+# scheme) or a per-token dynamic s = fp16_rn(amax / 7); two codes per byte,
+# code k = 2j in the low nibble and k = 2j + 1 in the high nibble of byte j of
+# the row, each as a 4-bit two's complement value.
+A4_MAX = 7
+
+
+def quantize_act4(A: np.ndarray):
+    """Per-token symmetric 4-bit quantization of fp16 activations.
+
+    For each row m: amax = max_k |A[m,k]|; sA = fp16_rn(amax / 7) with an fp32
+    divide; A4 = clamp(rint(A / float(sA)), -7, 7) with an fp32 divide (rint:
+    half to even); sA == 0 gives all-zero codes; rowsum[m] = sum_k A4[m,k].
+
+    Returns (A4 int8 [M,K] with values in [-7, 7], sA fp16 [M], rowsum int32 [M]).
+    """
+    assert A.dtype == np.float16 and A.ndim == 2
+    Af = A.astype(np.float32)
+    amax = np.max(np.abs(Af), axis=1) if A.shape[1] else np.zeros(A.shape[0], np.float32)
+    sA = (amax / np.float32(A4_MAX)).astype(np.float16)
+    sf = sA.astype(np.float32)
+    A4 = np.zeros(A.shape, dtype=np.int8)
+    nz = sf != 0
+    if np.any(nz):
+        A4[nz] = np.clip(np.rint(Af[nz] / sf[nz][:, None]), -A4_MAX, A4_MAX).astype(np.int8)
+    rowsum = A4.astype(np.int64).sum(axis=1).astype(np.int32)
+    return A4, sA, rowsum
+
+
+def quantize_act4_static(A: np.ndarray, s: np.float16):
+    """Per-tensor static symmetric 4-bit quantization (the PrefixQuant scheme):
+    A4 = clamp(rint(A / float(s)), -7, 7) with an fp32 divide (rint: half to
+    even); s == 0 gives all-zero codes; sA[m] = s; rowsum[m] = sum_k A4[m,k].
+
+    Returns (A4 int8 [M,K], sA fp16 [M], rowsum int32 [M]).
+    """
+    assert A.dtype == np.float16 and A.ndim == 2
+    sf = np.float32(np.float16(s))
+    A4 = np.zeros(A.shape, dtype=np.int8)
+    if sf != 0:
+        A4 = np.clip(np.rint(A.astype(np.float32) / sf), -A4_MAX, A4_MAX).astype(np.int8)
+    sA = np.full(A.shape[0], np.float16(s), dtype=np.float16)
+    rowsum = A4.astype(np.int64).sum(axis=1).astype(np.int32)
+    return A4, sA, rowsum
+
+
+def pack_act4(A4: np.ndarray) -> np.ndarray:
+    """[M, K] codes in [-8, 7] -> [M, K/2] bytes: byte j of a row holds code
+    2j in bits 0-3 and code 2j+1 in bits 4-7 (4-bit two's complement)."""
+    assert A4.ndim == 2 and A4.shape[1] % 2 == 0
+    nib = (A4.astype(np.int16) & 0xF).astype(np.uint8)
+    return (nib[:, 0::2] | (nib[:, 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_act4(P: np.ndarray) -> np.ndarray:
+    """Inverse of `pack_act4`: [M, K/2] bytes -> [M, K] int8 codes."""
+    assert P.dtype == np.uint8 and P.ndim == 2
+    lo = (P & 0xF).astype(np.int16)
+    hi = (P >> 4).astype(np.int16)
+    out = np.empty((P.shape[0], 2 * P.shape[1]), dtype=np.int16)
+    out[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    out[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return out.astype(np.int8)
 
 
 # ---------------------------------------------------------------------------
@@ -290,3 +367,10 @@ def w4a8_gemm(A8, sA, q, z, s2, s1, group: int = GROUP) -> np.ndarray:
 def w4a8_gemm_packed(A8, sA, blob) -> np.ndarray:
     q, z, s2, s1, N, K = unpack_weights(blob)
     return w4a8_gemm(A8, sA, q, z, s2, s1)
+
+
+def w4a4_gemm(A4_packed, sA, q, z, s2, s1, group: int = GROUP) -> np.ndarray:
+    """W4A4: Y = fp16(sA[m] * s1[n] * sum_k A4[m,k] * (q[n,k] - z) * s2) with the
+    4-bit activation codes A4 = unpack_act4(A4_packed); the same int32 sum and
+    fp32 epilogue as the 8-bit GEMM."""
+    return epilogue(gemm_acc(unpack_act4(A4_packed), dequant_weights(q, z, s2, group)), sA, s1)

@@ -452,3 +452,105 @@ def test_pack_roundtrip():
     for jj in range(4):
         vals += lo[4 * jj:4 * jj + 4] + hi[4 * jj:4 * jj + 4]
     assert vals == q[r, ks].tolist()
+
+
+# ------------------------------------------------------- 4-bit activations
+def test_act4_codes_exact_rational():
+    """Dynamic 4-bit codes: sA = fp16(fp32(amax) / 7) and each code is the
+    integer nearest to A / sA in exact arithmetic (ties to even), clamped to
+    [-7, 7], except where A / sA lies so close to a half-integer that the fp32
+    quotient may round across it; rowsum sums the codes."""
+    A = _rand_act(5, 256, 21)
+    A4, sA, rs = O.quantize_act4(A)
+    assert A4.min() >= -7 and A4.max() <= 7 and (rs == A4.astype(np.int64).sum(1)).all()
+    n_checked = 0
+    for m in range(A.shape[0]):
+        amax = max(abs(Fraction(float(v))) for v in A[m])
+        assert Fraction(float(np.float16(np.float32(float(amax)) / np.float32(7)))) == Fraction(float(sA[m]))
+        s = Fraction(float(sA[m]))
+        for k in range(A.shape[1]):
+            x = Fraction(float(A[m, k])) / s
+            frac = x - (x.numerator // x.denominator)
+            if abs(frac - Fraction(1, 2)) < Fraction(1, 10 ** 5):
+                continue
+            assert int(A4[m, k]) == max(-7, min(7, _nearest_even(x))), (m, k)
+            n_checked += 1
+    assert n_checked > 1200
+    # the outlier channels reach the range ends (the scale is fixed by them)
+    assert (np.abs(A4).max(1) == 7).all()
+
+
+def test_act4_static_codes_exact_rational_with_saturation():
+    A = _rand_act(4, 256, 22)
+    A[1] *= 30  # an outlier token: many codes saturate under the tensor scale
+    s = np.float16(0.5)
+    A4, sA, rs = O.quantize_act4_static(A, s)
+    assert (sA.view(np.uint16) == np.uint16(s.view(np.uint16))).all()
+    assert (rs == A4.astype(np.int64).sum(1)).all()
+    S = Fraction(float(s))
+    n_checked = n_clamped = 0
+    for m in range(A.shape[0]):
+        for k in range(A.shape[1]):
+            x = Fraction(float(A[m, k])) / S
+            frac = x - (x.numerator // x.denominator)
+            if abs(frac - Fraction(1, 2)) < Fraction(1, 10 ** 5):
+                continue
+            want = max(-7, min(7, _nearest_even(x)))
+            n_clamped += abs(want) == 7 and abs(x) > Fraction(15, 2)
+            assert int(A4[m, k]) == want, (m, k)
+            n_checked += 1
+    assert n_checked > 900 and n_clamped > 50
+
+
+def test_act4_constant_zero_rows_and_symmetries():
+    c = np.float16(3.5)
+    A = np.full((2, 128), c, dtype=np.float16)
+    A[1] = 0
+    A4, sA, rs = O.quantize_act4(A)
+    assert (A4[0] == 7).all() and rs[0] == 7 * 128
+    assert sA[0] == np.float16(np.float32(c) / np.float32(7)) and not A4[1].any() and sA[1] == 0
+    B = _rand_act(6, 384, 23)
+    P4, Ps, _ = O.quantize_act4(B)
+    N4, Ns, _ = O.quantize_act4(-B)
+    assert (N4 == -P4).all() and (Ns == Ps).all()  # rint is odd, amax even
+    Q4, Qs, _ = O.quantize_act4((B.astype(np.float32) * 8).astype(np.float16))
+    assert (Q4 == P4).all() and (Qs.astype(np.float32) == Ps.astype(np.float32) * 8).all()
+
+
+def test_act4_static_reduces_to_dynamic_per_row():
+    A = _rand_act(5, 512, 24)
+    A4d, sAd, rsd = O.quantize_act4(A)
+    for m in range(A.shape[0]):
+        A4s, sAs, rss = O.quantize_act4_static(A[m:m + 1], sAd[m])
+        assert (A4s[0] == A4d[m]).all() and rss[0] == rsd[m]
+
+
+def test_act4_pack_hand_bytes_and_full_domain():
+    codes = np.array([[1, -1, 7, -7, 0, -8, 3, 4]], dtype=np.int8)
+    # byte j: code 2j in bits 0-3, code 2j+1 in bits 4-7 (two's complement)
+    assert O.pack_act4(codes).tolist() == [[0xF1, 0x97, 0x80, 0x43]]
+    lo, hi = np.meshgrid(np.arange(-8, 8), np.arange(-8, 8), indexing="ij")
+    pairs = np.stack([lo.ravel(), hi.ravel()], axis=1).reshape(1, -1).astype(np.int8)
+    P = O.pack_act4(pairs)
+    assert sorted(P[0].tolist()) == list(range(256))  # a bijection on bytes
+    assert (O.unpack_act4(P) == pairs).all()
+
+
+def test_w4a4_gemm_brute_force():
+    """Pure-Python loops on the 4-bit codes and the element-wise dequantized
+    weights, epilogue in fp64: the oracle is within 1 fp16 ulp."""
+    rng = np.random.default_rng(25)
+    M, N, K = 3, 4, 256
+    A4, sA, _ = O.quantize_act4(_rand_act(M, K, 26))
+    q = rng.integers(0, 16, (N, K)).astype(np.uint8)
+    z = rng.integers(0, 16, (N, K // 128)).astype(np.uint8)
+    s2 = rng.integers(1, 9, (N, K // 128)).astype(np.uint8)
+    s1 = rng.uniform(0.001, 0.01, N).astype(np.float16)
+    Y = O.w4a4_gemm(O.pack_act4(A4), sA, q, z, s2, s1)
+    for m in range(M):
+        for n in range(N):
+            acc = sum(int(A4[m, k]) * (int(q[n, k]) - int(z[n, k // 128])) * int(s2[n, k // 128]) for k in range(K))
+            ref = np.float16(float(sA[m]) * float(s1[n]) * acc)
+            assert max_ulp_fp16(Y[m:m + 1, n:n + 1], np.array([[ref]])) <= 1, (m, n)
+    # 4-bit codes are a subset of the 8-bit codes: the 8-bit GEMM fed with them agrees exactly
+    assert (Y.view(np.uint16) == O.w4a8_gemm(A4, sA, q, z, s2, s1).view(np.uint16)).all()
