@@ -62,10 +62,13 @@ def weight_bytes(N, K):
     return (N // 128) * (K // 128) * TILE_BYTES + 2 * N
 
 
-def algorithmic_bytes(M, N, K):
-    """Bytes a W4A8 GEMM must move at least: packed weights, int8
-    activations, the activation scales, the fp16 output."""
-    return weight_bytes(N, K) + M * K + 2 * M + 2 * M * N
+def algorithmic_bytes(M, N, K, act_bits=8):
+    """Bytes a W4A8 (W4A4: act_bits=4) GEMM must move at least: packed
+    weights, the activation codes, the activation scales, the fp16 output."""
+    return weight_bytes(N, K) + M * K * act_bits // 8 + 2 * M + 2 * M * N
+
+
+ACT_BITS = {"dynamic": 8, "static": 8, "dynamic4": 4, "static4": 4}
 
 
 def gemm_ops(M, N, K):
@@ -223,10 +226,11 @@ class ClockSampler:
 _ORACLE_WEIGHTS = {}
 
 
-def cpu_oracle_run(workload, budget_s, reps=1):
-    """Times the CPU oracle (quantize_act + GEMM with the fp32 epilogue) on
-    this host over a bounded sample of the workload's cases; returns
-    (weight GB/s, description of the sample, threads used)."""
+def cpu_oracle_run(workload, budget_s, reps=1, act_bits=8):
+    """Times the CPU oracle (activation quantization + GEMM with the fp32
+    epilogue; 4-bit activations with act_bits=4) on this host over a bounded
+    sample of the workload's cases; returns (weight GB/s, description of the
+    sample, threads used)."""
     from oracle import w4a8_oracle as O
     cases = cases_of(workload)
     prepared = _ORACLE_WEIGHTS
@@ -247,8 +251,12 @@ def cpu_oracle_run(workload, budget_s, reps=1):
         A = I.activations(M, K, I.activation_seed(workload, M, K))
         for _ in range(reps):
             t0 = time.perf_counter()
-            A8, sA, _ = O.quantize_act(A)
-            O.w4a8_gemm(A8, sA, q, z, s2, s1)
+            if act_bits == 4:
+                A4, sA, _ = O.quantize_act4(A)
+                O.w4a4_gemm(O.pack_act4(A4), sA, q, z, s2, s1)
+            else:
+                A8, sA, _ = O.quantize_act(A)
+                O.w4a8_gemm(A8, sA, q, z, s2, s1)
             done_time += time.perf_counter() - t0
             done_bytes += weight_bytes(N, K)
         done.append(f"M={M} {name} {N}x{K}")
@@ -294,19 +302,29 @@ def run_gpu(args, world, rank, local):
 
     # ---- activations and outputs, resident in HBM
     acts, outs = {}, {}
-    ws = torch.zeros(max(w4a8.workspace_bytes(M, N, K) for (M, _, N, K) in cases), dtype=torch.uint8, device=dev)
+    ws_size = w4a8.w4a4_workspace_bytes if ACT_BITS[args.act] == 4 else w4a8.workspace_bytes
+    ws = torch.zeros(max(ws_size(M, N, K) for (M, _, N, K) in cases), dtype=torch.uint8, device=dev)
     for (M, name, N, K) in cases:
         acts[(M, name)] = torch.from_numpy(I.activations(M, K, I.activation_seed(args.workload, M, K))).to(dev)
-        outs[(M, name)] = (torch.empty((M, K), dtype=torch.int8, device=dev),
+        codes = (torch.empty((M, K), dtype=torch.int8, device=dev) if ACT_BITS[args.act] == 8 else
+                 torch.empty((M, K // 2), dtype=torch.uint8, device=dev))
+        outs[(M, name)] = (codes,
                            torch.empty((M,), dtype=torch.float16, device=dev),
                            torch.empty((M,), dtype=torch.int32, device=dev),
                            torch.empty((M, N), dtype=torch.float16, device=dev))
     copy_of = {M: i for i, M in enumerate(wl.ms)}
     static_scales = None
-    if args.act == "static":
+    if args.act in ("static", "static4"):
         # offline calibration: one scale per activation tensor, from its range
-        static_scales = {key: (A.float().abs().max() / 127).to(torch.float16).reshape(1)
+        qmax = 127 if args.act == "static" else 7
+        static_scales = {key: (A.float().abs().max() / qmax).to(torch.float16).reshape(1)
                          for key, A in acts.items()}
+    if ACT_BITS[args.act] == 4:
+        quantize = (w4a8.w4a4_quantize_act_static if static_scales is not None else w4a8.w4a4_quantize_act)
+        gemm = w4a8.w4a4_gemm
+    else:
+        quantize = (w4a8.quantize_act_static if static_scales is not None else w4a8.quantize_act)
+        gemm = w4a8.gemm
 
     def step(events=None, h2d=None, d2h=None, gemm_only=False):
         for i, (M, name, N, K) in enumerate(cases):
@@ -316,12 +334,12 @@ def run_gpu(args, world, rank, local):
             A8, sA, rs, Y = outs[(M, name)]
             if not gemm_only:
                 if static_scales is not None:
-                    w4a8.quantize_act_static(A, static_scales[(M, name)], out=(A8, sA, rs))
+                    quantize(A, static_scales[(M, name)], out=(A8, sA, rs))
                 else:
-                    w4a8.quantize_act(A, out=(A8, sA, rs))
+                    quantize(A, out=(A8, sA, rs))
             if events is not None:
                 events[i][0].record()
-            w4a8.gemm(A8, sA, rs, blobs[(name, copy_of[M])], N, K, out=Y, workspace=ws)
+            gemm(A8, sA, rs, blobs[(name, copy_of[M])], N, K, out=Y, workspace=ws)
             if events is not None:
                 events[i][1].record()
             if d2h is not None:
@@ -439,9 +457,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cases", default=None,
                     help="subset of the workload's cases, e.g. 16:gate_up,1:o (profiling)")
-    ap.add_argument("--act", default="dynamic", choices=["dynamic", "static"],
-                    help="activation scales: per-token dynamic (w4a8_quantize_act), or one per-tensor static "
-                         "scale calibrated once before timing (w4a8_quantize_act_static)")
+    ap.add_argument("--act", default="dynamic", choices=["dynamic", "static", "dynamic4", "static4"],
+                    help="activation codes and scales: 8-bit per-token dynamic (w4a8_quantize_act) or per-tensor "
+                         "static calibrated once before timing (w4a8_quantize_act_static); 4-bit (W4A4: "
+                         "w4a4_quantize_act / w4a4_quantize_act_static + w4a4_gemm)")
     ap.add_argument("--profile", type=int, default=0,
                     help="run this many eager steps for an external profiler and exit (no timing)")
     args = ap.parse_args()
@@ -464,7 +483,7 @@ def main():
     cases = r["cases"]
     peaks = load_peaks()
     wbytes = sum(weight_bytes(N, K) for (M, _, N, K) in cases)
-    abytes = [algorithmic_bytes(M, N, K) for (M, _, N, K) in cases]
+    abytes = [algorithmic_bytes(M, N, K, ACT_BITS[args.act]) for (M, _, N, K) in cases]
     ops = [gemm_ops(M, N, K) for (M, _, N, K) in cases]
     ms_step = r["max_ms"] / args.steps
     value = world * wbytes / (ms_step * 1e-3) / 1e9
@@ -486,7 +505,7 @@ def main():
         achieved = sum(ops) / (gemm_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": int8_peak_tops,
                     "unit": "TOPS", "frac": round(achieved / int8_peak_tops, 4)}
-    traffic = recorded_traffic(args.workload)
+    traffic = recorded_traffic(args.workload) if ACT_BITS[args.act] == 8 else None
     roofline["traffic"] = traffic
     roofline["peak_source"] = (f"{peaks['source']} HBM copy" if hbm_bound else
                                f"{peaks['source']} sustained bf16 x {INT8_OVER_BF16:g} (nominal int8/bf16 ratio)")
@@ -522,7 +541,7 @@ def main():
         "gpu": r["gpu_name"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds)
+        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds, act_bits=ACT_BITS[args.act])
         line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
                                 "sample": f"{len(sample)} of {len(cases)} cases ({'; '.join(sample)}), "
                                           f"{t:.1f} s of oracle time"}
@@ -538,11 +557,12 @@ def main_reference(args, world, rank):
     if rank != 0:
         return
     cases = cases_of(args.workload)
-    cpu_oracle_run(args.workload, 0.0)  # untimed warm-up (one case)
+    cpu_oracle_run(args.workload, 0.0, act_bits=ACT_BITS[args.act])  # untimed warm-up (one case)
     t0 = time.perf_counter()
     tot_bytes, tot_t, samples = 0.0, 0.0, []
     for _ in range(args.steps):
-        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds / max(args.steps, 1))
+        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds / max(args.steps, 1),
+                                               act_bits=ACT_BITS[args.act])
         tot_t += t
         tot_bytes += v * t * 1e9
         samples = sample

@@ -215,6 +215,69 @@ W4A8_API w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const int3
                                     size_t workspace_bytes, const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
 
 /*
+ * W4A4: 4-bit weights against 4-bit activations, the W4A4KV4 models of
+ * "PrefixQuant: Static Quantization Beats Dynamic through Prefixed Outliers
+ * in LLMs" (Key Findings), which quantizes activations per tensor with a
+ * static scale once the outlier tokens are prefixed. The pages give no code
+ * range or storage for the 4-bit activations; this library uses the 8-bit
+ * scheme with the symmetric 4-bit range:
+ *   A4[m,k] = clamp(rint(A[m,k] / float(s)), -7, 7)   (IEEE fp32 divide, ties to even)
+ * stored two codes per byte: byte j of token m holds code 2j in bits 0-3 and
+ * code 2j+1 in bits 4-7 (4-bit two's complement), i.e. A4 is uint8 [M, K/2].
+ * The GEMM computes exactly what w4a8_gemm computes on those codes:
+ *   Y[m,n] = fp16_rn(float(sum_k A4[m,k] * W8[n,k]) * (float(sA[m]) * float(s1[n])))
+ * (the tensor cores have no 4-bit integer mode: the kernel expands each
+ * activation tile to int8 in shared memory).
+ */
+
+/*
+ * Per-token dynamic 4-bit activations: sA[m] = fp16_rn(amax_m / 7) (IEEE
+ * fp32 divide), s = sA[m] above; sA == 0 gives zero codes.
+ * A: fp16 [M, K]. A4: uint8 [M, K/2] (16-byte aligned). sA: fp16 [M] (2-byte
+ * aligned). rowsum: int32 [M] (4-byte aligned) or NULL, sum_k A4[m,k].
+ * Limits: K % 8 == 0, 0 < K <= 65536, M >= 0 (M == 0 is a no-op).
+ */
+W4A8_API w4a8_status_t w4a4_quantize_act(const void* A, int64_t M, int64_t K, uint8_t* A4, void* sA,
+                                         int32_t* rowsum, w4a8_stream_t stream);
+
+/*
+ * Per-tensor static 4-bit activations (PrefixQuant's scheme): one fp16 scale
+ * s (device pointer, read on the device) for the whole tensor; sA[m] = s so
+ * that the GEMM's per-token epilogue applies it. Other arguments and limits
+ * as for w4a4_quantize_act.
+ */
+W4A8_API w4a8_status_t w4a4_quantize_act_static(const void* A, int64_t M, int64_t K, const void* s, uint8_t* A4,
+                                                void* sA, int32_t* rowsum, w4a8_stream_t stream);
+
+/*
+ * W4A4 GEMM: A4 uint8 [M, K/2] from w4a4_quantize_act(_static) (16-byte
+ * aligned), rowsum its code sums (required, as for w4a8_gemm). Other
+ * arguments, the workspace and the limits as for w4a8_gemm.
+ */
+W4A8_API w4a8_status_t w4a4_gemm(const uint8_t* A4, const void* sA, const int32_t* rowsum, const void* packed,
+                                 int64_t M, int64_t N, int64_t K, void* Y, void* workspace, size_t workspace_bytes,
+                                 w4a8_stream_t stream);
+
+/*
+ * Workspace for w4a4_gemm / w4a4_gemm_ex: w4a8_gemm_workspace_bytes(M, N, K)
+ * rounded up to a multiple of 256, plus M * K. Its first
+ * w4a8_gemm_workspace_bytes(M, N, K) bytes follow the rules of the w4a8
+ * workspace (zero-filled once by the caller, left zero-filled by every call);
+ * each call expands the packed activation codes once (one small extra
+ * kernel) into the workspace's LAST M * K bytes (from a 256-byte boundary),
+ * which need no particular contents, instead of inside the GEMM once per
+ * output tile. A workspace of the returned size serves every M' <= M,
+ * N' <= N, K' <= K. With a workspace too small for that scratch the GEMM
+ * expands the codes itself in shared memory (same results, slower).
+ */
+W4A8_API size_t w4a4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K);
+
+/* w4a4_gemm with the output choice and overrides of w4a8_gemm_ex. */
+W4A8_API w4a8_status_t w4a4_gemm_ex(const uint8_t* A4, const void* sA, const int32_t* rowsum, const void* packed,
+                                    int64_t M, int64_t N, int64_t K, void* Y, int32_t* acc, void* workspace,
+                                    size_t workspace_bytes, const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
+
+/*
  * Allocation-free GEMM: the same computation and results as w4a8_gemm, for
  * callers that cannot hand the library a workspace. This entry point has no
  * counterpart in the papers; it exists for deployment. Typical callers: a

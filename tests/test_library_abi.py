@@ -24,7 +24,7 @@ def L():
 
 def declared_functions():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4a8_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4a[48]_\w+)\s*\(", src)))
 
 
 def test_header_declares_entry_points():
@@ -124,6 +124,25 @@ def test_gemm_validation(L):
     assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, both, None, 0, None, None) == 1  # Y and acc
     assert L.w4a8_gemm_debug_acc(FAKE, FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1  # no acc
     assert ex(None, None, None, None, 0, 128, 256, None, None, None, 0, None, None) == 0   # M == 0
+
+
+def test_w4a4_validation(L):
+    q = L.w4a4_quantize_act
+    assert q(FAKE, 4, 7, FAKE, FAKE, None, None) == 2                # K % 8
+    assert q(FAKE, 4, 128, None, FAKE, None, None) == 1              # no output
+    assert q(FAKE, 4, 128, FAKE_ODD, FAKE, None, None) == 3          # packed codes alignment
+    assert q(FAKE, 0, 128, None, None, None, None) == 0              # M == 0: no-op
+    qs = L.w4a4_quantize_act_static
+    assert qs(FAKE, 4, 128, None, FAKE, FAKE, None, None) == 1       # no scale
+    assert qs(FAKE, 4, 128, FAKE_ODD, FAKE, FAKE, None, None) == 3   # scale alignment
+    g = L.w4a4_gemm
+    assert g(FAKE, FAKE, FAKE, FAKE, 4, 100, 256, FAKE, None, 0, None) == 2   # N % 128
+    assert g(FAKE, FAKE, FAKE, FAKE, 4, 128, 200, FAKE, None, 0, None) == 2   # K % 128
+    assert g(FAKE, FAKE, None, FAKE, 4, 128, 256, FAKE, None, 0, None) == 1   # no rowsum
+    assert g(FAKE_ODD, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, None, 0, None) == 3
+    assert g(FAKE, FAKE, FAKE, FAKE, 0, 128, 256, FAKE, None, 0, None) == 0   # M == 0: no-op
+    ex = L.w4a4_gemm_ex
+    assert ex(FAKE, FAKE, FAKE, FAKE, 4, 128, 256, FAKE, FAKE, None, 0, None, None) == 1  # Y and acc
 
 
 def test_python_binding_refuses_cpu_tensors(L):

@@ -19,7 +19,8 @@ __all__ = [
     "W4A8Error", "lib", "library_path", "EXPORTED_SYMBOLS", "status_string", "quantize_act",
     "quantize_weights", "packed_bytes", "pack_weights", "workspace_bytes", "Workspace", "gemm",
     "gemm_debug_acc", "gemm_ex", "gemm_noalloc", "get_device_error", "clear_device_error",
-    "selftest_bounded_wait", "quantize_act_static",
+    "selftest_bounded_wait", "quantize_act_static", "w4a4_quantize_act", "w4a4_quantize_act_static",
+    "w4a4_gemm", "w4a4_gemm_ex", "w4a4_workspace_bytes",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -30,6 +31,7 @@ EXPORTED_SYMBOLS = (
     "w4a8_packed_bytes", "w4a8_pack_weights", "w4a8_gemm_workspace_bytes", "w4a8_gemm",
     "w4a8_gemm_debug_acc", "w4a8_gemm_ex", "w4a8_get_device_error", "w4a8_clear_device_error",
     "w4a8_gemm_noalloc", "w4a8_selftest_bounded_wait", "w4a8_quantize_act_static",
+    "w4a4_quantize_act", "w4a4_quantize_act_static", "w4a4_gemm", "w4a4_gemm_ex", "w4a4_gemm_workspace_bytes",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
@@ -74,6 +76,12 @@ def lib() -> ctypes.CDLL:
         "w4a8_gemm_noalloc": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp]),
         "w4a8_selftest_bounded_wait": (ctypes.c_int, [i64, vp]),
         "w4a8_quantize_act_static": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp, vp]),
+        "w4a4_quantize_act": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp]),
+        "w4a4_quantize_act_static": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp, vp]),
+        "w4a4_gemm": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "w4a4_gemm_workspace_bytes": (sz, [i64, i64, i64]),
+        "w4a4_gemm_ex": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, sz,
+                                        ctypes.POINTER(GemmOpts), vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -261,6 +269,101 @@ def gemm_ex(A8, sA, rowsum, blob, N: int, K: int, Y=None, acc=None, workspace=No
     """GEMM with explicit scheduling overrides (for tests and tuning)."""
     _gemm_common(A8, sA, rowsum, blob, N, K, Y, acc, workspace, (schedule, block_m, max_ctas, 0))
     return Y if Y is not None else acc
+
+
+# ------------------------------------------------------------------ W4A4
+def w4a4_workspace_bytes(M: int, N: int, K: int) -> int:
+    return int(lib().w4a4_gemm_workspace_bytes(M, N, K))
+
+
+def _w4a4_workspace_for(device, M, N, K):
+    """A cached W4A4 workspace shared by all shapes: its zero-filled prefix
+    covers the largest w4a8 part seen and its scratch end the largest M * K
+    seen, so no shape's scratch (at the buffer's end) reaches another shape's
+    zero-filled prefix."""
+    torch = _torch()
+    if w4a4_workspace_bytes(M, N, K) == 0:
+        return None
+    key = ("w4a4", str(device))
+    buf, base, codes = _default_ws.get(key, (None, 0, 0))
+    base2, codes2 = max(base, workspace_bytes(M, N, K)), max(codes, M * K)
+    if buf is None or base2 > base or codes2 > codes:
+        need = (base2 + 255) // 256 * 256 + codes2 + 256
+        buf = torch.zeros((need,), dtype=torch.uint8, device=device)
+        _default_ws[key] = (buf, base2, codes2)
+    return buf
+
+
+def _act4_outputs(A, out):
+    torch = _torch()
+    M, K = A.shape
+    if out is None:
+        return (torch.empty((M, K // 2), dtype=torch.uint8, device=A.device),
+                torch.empty((M,), dtype=torch.float16, device=A.device),
+                torch.empty((M,), dtype=torch.int32, device=A.device))
+    _require_cuda(*out)
+    return out
+
+
+def w4a4_quantize_act(A, out=None):
+    """fp16 [M, K] -> (A4 uint8 [M, K/2] packed 4-bit codes, sA fp16 [M], rowsum int32 [M])."""
+    torch = _torch()
+    _require_cuda(A)
+    if A.dtype != torch.float16 or A.dim() != 2:
+        raise W4A8Error("A must be a 2-D fp16 tensor")
+    A4, sA, rowsum = _act4_outputs(A, out)
+    M, K = A.shape
+    _check(lib().w4a4_quantize_act(_ptr(A), M, K, _ptr(A4), _ptr(sA), _ptr(rowsum), _stream(A.device)),
+           "w4a4_quantize_act")
+    return A4, sA, rowsum
+
+
+def w4a4_quantize_act_static(A, s, out=None):
+    """Per-tensor static 4-bit codes with the fp16 scale `s` (a 1-element CUDA
+    tensor): fp16 [M, K] -> (A4 uint8 [M, K/2], sA fp16 [M] = s, rowsum int32 [M])."""
+    torch = _torch()
+    _require_cuda(A, s)
+    if A.dtype != torch.float16 or A.dim() != 2 or s.dtype != torch.float16 or s.numel() != 1:
+        raise W4A8Error("A must be a 2-D fp16 tensor and s a 1-element fp16 tensor")
+    A4, sA, rowsum = _act4_outputs(A, out)
+    M, K = A.shape
+    _check(lib().w4a4_quantize_act_static(_ptr(A), M, K, _ptr(s), _ptr(A4), _ptr(sA), _ptr(rowsum),
+                                          _stream(A.device)), "w4a4_quantize_act_static")
+    return A4, sA, rowsum
+
+
+def w4a4_gemm_ex(A4, sA, rowsum, blob, N: int, K: int, Y=None, acc=None, workspace=None, schedule=0, block_m=0,
+                 max_ctas=0):
+    """W4A4 GEMM on packed 4-bit activation codes A4 uint8 [M, K/2]: fp16 Y
+    and/or (acc given) the raw int32 accumulators; scheduling overrides as gemm_ex."""
+    torch = _torch()
+    _require_cuda(A4, sA, rowsum, blob, Y, acc, workspace)
+    M = A4.shape[0]
+    if A4.dtype != torch.uint8 or A4.dim() != 2 or A4.shape[1] * 2 != K:
+        raise W4A8Error("A4 must be uint8 [M, K/2]")
+    if workspace is None:
+        workspace = _w4a4_workspace_for(A4.device, M, N, K)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    o = ctypes.byref(GemmOpts(schedule, block_m, max_ctas, 0))
+    _check(lib().w4a4_gemm_ex(_ptr(A4), _ptr(sA), _ptr(rowsum), _ptr(blob), M, N, K, _ptr(Y), _ptr(acc),
+                              _ptr(workspace), ws_bytes, o, _stream(A4.device)), "w4a4_gemm_ex")
+    return Y if Y is not None else acc
+
+
+def w4a4_gemm(A4, sA, rowsum, blob, N: int, K: int, out=None, workspace=None):
+    """Y fp16 [M, N] = fp16(sA * s1 * (A4 @ W8^T)) on packed 4-bit activation codes."""
+    torch = _torch()
+    _require_cuda(A4, sA, rowsum, blob, out, workspace)
+    M = A4.shape[0]
+    if A4.dtype != torch.uint8 or A4.dim() != 2 or A4.shape[1] * 2 != K:
+        raise W4A8Error("A4 must be uint8 [M, K/2]")
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A4.device)
+    if workspace is None:
+        workspace = _w4a4_workspace_for(A4.device, M, N, K)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().w4a4_gemm(_ptr(A4), _ptr(sA), _ptr(rowsum), _ptr(blob), M, N, K, _ptr(Y), _ptr(workspace),
+                           ws_bytes, _stream(A4.device)), "w4a4_gemm")
+    return Y
 
 
 NOALLOC_SCRATCH_BYTES = 8 << 20

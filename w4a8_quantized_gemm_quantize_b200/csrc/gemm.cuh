@@ -62,6 +62,7 @@ struct GemmArgs {
   int m_tiles, num_tiles;
   int sk_tiles;          // the first sk_tiles tiles are split stream-K over all CTAs
   int split;             // > 1: cluster split-K, `split` CTAs (one cluster) per tile
+  int a4;                // activation codes are 4-bit, two per byte (W4A4), unpacked in shared memory
 };
 
 struct Seg {
@@ -195,7 +196,8 @@ struct GemmCfg {
   static constexpr int kOffW = NS * kASlot;        // 16-aligned weight slots
   static constexpr int kOffRecv = kOffW + NS * kWSlot;
   static constexpr int kOffBar = (kOffRecv + kRecvSlots * kRecvSlotBytes + 15) / 16 * 16;
-  static constexpr int kNumBars = 4 * NS + 2 * NT + 2 * NACC + 1 + 4;  // + one receive barrier per lane quarter
+  // + one receive barrier per lane quarter + one packed-activation barrier per slot
+  static constexpr int kNumBars = 4 * NS + 2 * NT + 2 * NACC + 1 + 4 + NS;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   // epilogue per-token operands (128 int32 + 128 float), then the store
   // transpose (1 KB per epilogue warp, read as 16-byte vectors: 16-aligned)
@@ -500,6 +502,166 @@ __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg
   return true;
 }
 
+// Four 4-bit two's complement codes (one per byte, bits 0-3) -> four int8.
+__device__ __forceinline__ uint32_t sign_extend_nibbles(uint32_t x) {
+  return x | ((x & 0x08080808u) * 0x1Eu);  // bit 3 set: OR 0xF0 into that byte (no carry leaves a byte)
+}
+
+// 16 packed 4-bit codes (8 bytes, code 2j in the low nibble of byte j) ->
+// 16 int8 codes in k order.
+__device__ __forceinline__ uint4 expand_codes4(uint2 p) {
+  const uint32_t e0 = p.x & 0x0F0F0F0Fu, o0 = (p.x >> 4) & 0x0F0F0F0Fu;  // codes 0,2,4,6 / 1,3,5,7
+  const uint32_t e1 = p.y & 0x0F0F0F0Fu, o1 = (p.y >> 4) & 0x0F0F0F0Fu;  // codes 8,.. / 9,..
+  uint4 o;
+  o.x = sign_extend_nibbles(__byte_perm(e0, o0, 0x5140));  // codes 0..3
+  o.y = sign_extend_nibbles(__byte_perm(e0, o0, 0x7362));  // codes 4..7
+  o.z = sign_extend_nibbles(__byte_perm(e1, o1, 0x5140));  // codes 8..11
+  o.w = sign_extend_nibbles(__byte_perm(e1, o1, 0x7362));  // codes 12..15
+  return o;
+}
+
+// Expands packed 4-bit activation codes [M, K/2] into int8 codes [M, K]
+// (16 codes per thread and step, 8 bytes in, 16 out; HBM-bound). Used before
+// the int8 GEMM when the token tiles are large: each activation tile is then
+// expanded once instead of once per output tile.
+__global__ void expand_act4_kernel(const uint2* __restrict__ packed, int64_t units, uint4* __restrict__ out) {
+  grid_launch_dependents();  // the GEMM after this kernel may start its weight stream
+  grid_dependency_wait();    // the codes come from the preceding kernel
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < units; i += stride)
+    out[i] = expand_codes4(__ldcs(packed + i));
+}
+
+// Activation producer for 4-bit activations (W4A4, "PrefixQuant ...", Key
+// Findings): the codes arrive packed, two per byte (64 bytes per token per
+// k-block). Lane 0 loads each k-block's packed tile (BN rows x 64 bytes) by
+// TMA into the upper half of its activation slot; the warp then expands it in
+// place into the int8 layout the MMA reads (BN rows x 128 bytes, 128-byte
+// swizzle: 16-byte piece c of row r at r * 128 + ((c ^ (r & 7)) * 16)) and
+// releases the slot to the MMA issuers. Rows are expanded in ascending groups
+// of four, in batches of up to eight groups; the packed bytes of every row a
+// group overwrites have been read by then (group g writes bytes
+// [512 g, 512 g + 512), which hold packed rows 8 g - BN .. 8 g - BN + 7 <=
+// 4 g + 3), and all lanes read a batch before any lane writes it.
+// The warp polls two conditions (non-blocking tests, with a short sleep when
+// neither holds) and serves whichever is ready, expansion first: the oldest
+// loaded chunk has arrived (expand it, in load order), or
+// the slot of the next chunk is free (load it). A load never waits behind an
+// expansion nor an expansion behind a free slot, so the loads run up to NS
+// chunks ahead while every arrived chunk reaches the MMA at once. Neither
+// wait can be part of a cycle: a slot frees when the MMAs of the chunk
+// loaded NS chunks earlier finish, and that chunk was expanded before.
+template <class C>
+__device__ __forceinline__ void act4_producer(const GemmArgs& args, const CUtensorMap* tmap, uint8_t* sA8,
+                                              uint64_t* afull, uint64_t* aempty, uint64_t* astage, int lane,
+                                              volatile int* dep_done, volatile int* abort_flag, DevErr err) {
+  constexpr int BN = C::BN, KS = C::KS, NS = C::NS;
+  constexpr int kPackedRow = 64;  // bytes of one token's 128 codes
+  grid_dependency_wait();         // the codes come from the preceding kernel
+  if (lane == 0) *dep_done = 1;
+  int cnt_ring[NS] = {};
+  Sched sch;
+  sch.init(args);
+  Seg sg;
+  bool have_seg = sch.next(sg);
+  int kb = have_seg ? sg.kb0 : 0;
+  int issued = 0, expanded = 0;
+  bool ok = true;
+  uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    bool progressed = false;
+    if (expanded < issued) {
+      const int a = expanded % NS;
+      if (__all_sync(0xffffffffu, mbar_test_wait(smem_u32(&astage[a]), (expanded / NS) & 1))) {
+        const int cnt = cnt_ring[a];
+        for (int j = 0; j < cnt; ++j) {
+          uint8_t* base = sA8 + a * C::kASlot + j * C::kA8Bytes;
+          const uint8_t* packed = base + BN * kPackedRow;
+          // batches of up to 8 row groups: all of a batch's packed bytes are
+          // read (independent loads) before any of its rows is written
+          constexpr int kGroups = BN / 4, kBatch = kGroups < 8 ? kGroups : 8;
+          const int c = lane & 7;
+#pragma unroll 1
+          for (int g0 = 0; g0 < kGroups; g0 += kBatch) {
+            uint2 p[kBatch];
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b)
+              p[b] = *reinterpret_cast<const uint2*>(packed + (4 * (g0 + b) + (lane >> 3)) * kPackedRow + c * 8);
+            __syncwarp();
+#pragma unroll
+            for (int b = 0; b < kBatch; ++b) {
+              const int row = 4 * (g0 + b) + (lane >> 3);
+              *reinterpret_cast<uint4*>(base + row * 128 + ((c ^ (row & 7)) << 4)) = expand_codes4(p[b]);
+            }
+            __syncwarp();
+          }
+        }
+        fence_proxy_async_smem();  // the MMA (async proxy) reads what these generic stores wrote
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&afull[a]);
+        ++expanded;
+        progressed = true;
+      }
+    }
+    if (!progressed && have_seg) {
+      const int a = issued % NS;
+      if (__all_sync(0xffffffffu, mbar_test_wait(smem_u32(&aempty[a]), ((issued / NS) & 1) ^ 1))) {
+        const int cnt = min(KS, sg.kb1 - kb);
+        const int m0 = (sg.tile % args.m_tiles) * BN;
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&astage[a], cnt * BN * kPackedRow);
+          for (int j = 0; j < cnt; ++j)
+            tma_load_2d(sA8 + a * C::kASlot + j * C::kA8Bytes + BN * kPackedRow, tmap, &astage[a],
+                        (kb + j) * kPackedRow, m0);
+        }
+        cnt_ring[a] = cnt;
+        ++issued;
+        kb += KS;
+        if (kb >= sg.kb1) {
+          have_seg = sch.next(sg);
+          if (have_seg) kb = sg.kb0;
+        }
+        progressed = true;
+      }
+    }
+    if (!have_seg && expanded == issued) break;
+    if (progressed) {
+      t0 = global_timer_ns();
+      continue;
+    }
+    // nothing ready: sleep briefly instead of spinning, which would take issue
+    // slots from the dequantizer warps on this SM sub-partition
+    __nanosleep(128);
+    if ((it & 31u) == 0) {
+      // nothing ready: the same bounds as every other wait of the kernel,
+      // decided once for the whole warp
+      if (__any_sync(0xffffffffu, *abort_flag != 0)) {
+        ok = false;
+        break;
+      }
+      const uint64_t now = global_timer_ns();
+      bool expired = false;
+      if (now < t0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        expired = true;
+      }
+      if (__any_sync(0xffffffffu, expired)) {
+        if (lane == 0) {
+          *abort_flag = 1;
+          atomicCAS(err.word, 0, kErrProducer);
+        }
+        ok = false;
+        break;
+      }
+    }
+  }
+  (void)ok;
+  // copies still in flight must land before the CTA exits
+  for (int u = expanded; u < issued; ++u) mbar_wait(&astage[u % NS], (u / NS) & 1, nullptr, err, kErrDrain);
+  __syncwarp();
+}
+
 template <class C>
 __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                                                     const GemmArgs args) {
@@ -518,6 +680,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
   uint64_t* accempty = accfull + NACC;                               // epilogue has read the accumulator
   uint64_t* done = accempty + NACC;                                  // all MMAs finished
   uint64_t* recvbar = done + 1;                                      // cluster partials received, per quarter
+  uint64_t* astage = recvbar + 4;                                    // packed 4-bit activations loaded
   uint32_t* recv = reinterpret_cast<uint32_t*>(smem + C::kOffRecv);
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
@@ -561,6 +724,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     for (int i = 0; i < NS; ++i) {
       mbar_init(&afull[i], 1);
       mbar_init(&aempty[i], 1);
+      mbar_init(&astage[i], 1);
     }
     for (int i = 0; i < NT; ++i) {
       mbar_init(&tfull[i], 4);
@@ -637,6 +801,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       for (int i = first; i < c; ++i) mbar_wait(&wfull[i % NS], (i / NS) & 1, nullptr, err, kErrDrain);
     }
     __syncwarp();
+  } else if (warp == 3 && args.a4) {
+    // -------------------------------- activation producer, 4-bit activations
+    act4_producer<C>(args, &tmap_a, sA8, afull, aempty, astage, lane, dep_done, abort_flag, err);
   } else if (warp == 3) {
     // ------------------------------------------------- activation producer
     if (lane == 0) {

@@ -47,16 +47,45 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
   return red[0];
 }
 
-__device__ __forceinline__ int quant_one(float x, float sf) {
+// Code of one value: clamp(rint(x / sf), -QMAX, QMAX), IEEE fp32 divide,
+// ties to even. QMAX = 127 (8-bit codes) or 7 (4-bit codes).
+template <int QMAX>
+__device__ __forceinline__ int quant_code(float x, float sf) {
   int q = __float2int_rn(__fdiv_rn(x, sf));
-  return max(-127, min(127, q));
+  return max(-QMAX, min(QMAX, q));
 }
 
+// Codes per token: 8 = one int8 per code (row of K bytes); 4 = two codes per
+// byte, code 2j in bits 0-3 and code 2j+1 in bits 4-7 of byte j, 4-bit two's
+// complement (row of K / 2 bytes; the W4A4 activations of "PrefixQuant ...",
+// Key Findings).
+template <int BITS>
+struct CodeOut {
+  static constexpr int kQmax = BITS == 8 ? 127 : 7;
+  // stores the 8 codes of 16-byte input vector idx of a row
+  __device__ __forceinline__ static void store(void* row, int idx, const int (&q)[8]) {
+    if constexpr (BITS == 8) {
+      uint32_t w[2] = {0u, 0u};
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w[j >> 2] |= (static_cast<uint32_t>(q[j]) & 0xFFu) << ((j & 3) * 8);
+      reinterpret_cast<uint2*>(row)[idx] = make_uint2(w[0], w[1]);
+    } else {
+      uint32_t w = 0u;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) w |= (static_cast<uint32_t>(q[j]) & 0xFu) << (j * 4);
+      reinterpret_cast<uint32_t*>(row)[idx] = w;
+    }
+  }
+};
+
 // VPT: 16-byte vectors (8 halves) per thread; K <= THREADS * VPT * 8.
-template <int THREADS, int VPT>
+// BITS: 8 (int8 codes, sA = amax / 127) or 4 (packed 4-bit codes,
+// sA = amax / 7).
+template <int THREADS, int VPT, int BITS = 8>
 __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __restrict__ A, int64_t K,
-                                                                int8_t* __restrict__ A8, __half* __restrict__ sA,
+                                                                void* __restrict__ codes, __half* __restrict__ sA,
                                                                 int32_t* __restrict__ rowsum, int early_release) {
+  using Out = CodeOut<BITS>;
   __shared__ float fred[32];
   __shared__ int ird[32];
   // Launched as a programmatic dependent: this grid waits for the preceding
@@ -90,27 +119,26 @@ __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __r
     }
   }
   amax = block_max<THREADS>(amax, fred);
-  const __half s_h = __float2half_rn(__fdiv_rn(amax, 127.0f));
+  const __half s_h = __float2half_rn(__fdiv_rn(amax, static_cast<float>(Out::kQmax)));
   const float sf = __half2float(s_h);
   int local = 0;
-  uint2* out = reinterpret_cast<uint2*>(A8 + m * K);
+  void* out = static_cast<uint8_t*>(codes) + m * K * BITS / 8;
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
     const int idx = threadIdx.x + i * THREADS;
     if (idx < nvec) {
       const __half2* h = reinterpret_cast<const __half2*>(&v[i]);
-      uint32_t packed[2] = {0u, 0u};
+      int q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       if (sf != 0.0f) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = __half22float2(h[j]);
-          const int q0 = quant_one(f.x, sf), q1 = quant_one(f.y, sf);
-          local += q0 + q1;
-          packed[j >> 1] |= ((static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8))
-                            << ((j & 1) * 16);
+          q[2 * j] = quant_code<Out::kQmax>(f.x, sf);
+          q[2 * j + 1] = quant_code<Out::kQmax>(f.y, sf);
+          local += q[2 * j] + q[2 * j + 1];
         }
       }
-      out[idx] = make_uint2(packed[0], packed[1]);
+      Out::store(out, idx, q);
     }
   }
   if (rowsum != nullptr) {
@@ -127,13 +155,14 @@ __global__ void __launch_bounds__(THREADS) quantize_act_kernel(const __half* __r
 // A, A8 = clamp(rint(A / float(s)), -127, 127) (IEEE fp32 divide, ties to
 // even; s == 0 gives zero codes), rowsum, and sA[m] = s so that the GEMM's
 // per-token epilogue applies the tensor scale. One CTA per token.
-template <int THREADS, int VPT>
+template <int THREADS, int VPT, int BITS = 8>
 __global__ void __launch_bounds__(THREADS) quantize_act_static_kernel(const __half* __restrict__ A, int64_t K,
                                                                        const __half* __restrict__ s,
-                                                                       int8_t* __restrict__ A8,
+                                                                       void* __restrict__ codes,
                                                                        __half* __restrict__ sA,
                                                                        int32_t* __restrict__ rowsum,
                                                                        int early_release) {
+  using Out = CodeOut<BITS>;
   __shared__ int ird[32];
   if (early_release) grid_launch_dependents();  // as in quantize_act_kernel
   grid_dependency_wait();                       // A (and s) may come from the preceding kernel
@@ -142,7 +171,7 @@ __global__ void __launch_bounds__(THREADS) quantize_act_static_kernel(const __ha
   const __half s_h = *s;
   const float sf = __half2float(s_h);
   const uint4* row = reinterpret_cast<const uint4*>(A + m * K);
-  uint2* out = reinterpret_cast<uint2*>(A8 + m * K);
+  void* out = static_cast<uint8_t*>(codes) + m * K * BITS / 8;
   const int nvec = static_cast<int>(K >> 3);
   int local = 0;
 #pragma unroll
@@ -153,18 +182,17 @@ __global__ void __launch_bounds__(THREADS) quantize_act_static_kernel(const __ha
     const uint4 v = __ldcs(row + (idx < nvec ? idx : nvec - 1));
     if (idx < nvec) {
       const __half2* h = reinterpret_cast<const __half2*>(&v);
-      uint32_t packed[2] = {0u, 0u};
+      int q[8] = {0, 0, 0, 0, 0, 0, 0, 0};
       if (sf != 0.0f) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const float2 f = __half22float2(h[j]);
-          const int q0 = quant_one(f.x, sf), q1 = quant_one(f.y, sf);
-          local += q0 + q1;
-          packed[j >> 1] |= ((static_cast<uint32_t>(q0) & 0xFFu) | ((static_cast<uint32_t>(q1) & 0xFFu) << 8))
-                            << ((j & 1) * 16);
+          q[2 * j] = quant_code<Out::kQmax>(f.x, sf);
+          q[2 * j + 1] = quant_code<Out::kQmax>(f.y, sf);
+          local += q[2 * j] + q[2 * j + 1];
         }
       }
-      out[idx] = make_uint2(packed[0], packed[1]);
+      Out::store(out, idx, q);
     }
   }
   if (rowsum != nullptr) {

@@ -163,18 +163,23 @@ w4a8_status_t max_clusters(int dev, int split, int* out) {
   return W4A8_OK;
 }
 
+// The activation tensor map: int8 codes as [M, K] bytes, loaded as 128-byte
+// rows with the 128-byte swizzle the MMA descriptor expects; or (W4A4) the
+// packed 4-bit codes as [M, K / 2] bytes, loaded as plain 64-byte rows that
+// the kernel expands in shared memory.
 template <class C>
-w4a8_status_t launch_gemm_cfg(const int8_t* A8, int64_t M, int64_t K, GemmArgs args, int grid,
+w4a8_status_t launch_gemm_cfg(const void* act, int64_t M, int64_t K, GemmArgs args, int grid,
                               cudaStream_t stream) {
   if (args.split > C::kMaxSplit) return W4A8_ERR_INVALID_ARG;
   CUtensorMap map;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
-  const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(C::BN)};
+  const int64_t row_bytes = args.a4 ? K / 2 : K;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  const cuuint32_t box[2] = {args.a4 ? 64u : 128u, static_cast<cuuint32_t>(C::BN)};
   const cuuint32_t estr[2] = {1u, 1u};
-  if (g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(A8), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+  if (g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(act), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, args.a4 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return W4A8_ERR_CUDA;
   return launch_pdl(w4a8_gemm_kernel<C>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, args.split, map,
                     args);
@@ -193,11 +198,65 @@ size_t ws_counter_bytes(int64_t M, int64_t N) {
   return static_cast<size_t>((tiles * 4 + 255) / 256 * 256);
 }
 
+// Activation quantizers (one CTA per token), dispatched on the row length;
+// BITS = 8 writes int8 codes, 4 packed 4-bit codes.
+template <int BITS>
+w4a8_status_t launch_quantize_dynamic(const __half* a, int64_t M, int64_t K, void* codes, __half* s, int32_t* rowsum,
+                                      cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>(M));
+  const int64_t nvec = K / 8;
+  const int early = M <= kEarlyReleaseRows ? 1 : 0;
+  if (nvec <= 128)
+    return launch_pdl(quantize_act_kernel<128, 1, BITS>, grid, dim3(128), 0, st, 1, a, K, codes, s, rowsum, early);
+  if (nvec <= 256)
+    return launch_pdl(quantize_act_kernel<256, 1, BITS>, grid, dim3(256), 0, st, 1, a, K, codes, s, rowsum, early);
+  if (nvec <= 512)
+    return launch_pdl(quantize_act_kernel<256, 2, BITS>, grid, dim3(256), 0, st, 1, a, K, codes, s, rowsum, early);
+  if (nvec <= 1024)
+    return launch_pdl(quantize_act_kernel<256, 4, BITS>, grid, dim3(256), 0, st, 1, a, K, codes, s, rowsum, early);
+  if (nvec <= 2048)
+    return launch_pdl(quantize_act_kernel<256, 8, BITS>, grid, dim3(256), 0, st, 1, a, K, codes, s, rowsum, early);
+  if (nvec <= 4096)
+    return launch_pdl(quantize_act_kernel<512, 8, BITS>, grid, dim3(512), 0, st, 1, a, K, codes, s, rowsum, early);
+  return launch_pdl(quantize_act_kernel<1024, 8, BITS>, grid, dim3(1024), 0, st, 1, a, K, codes, s, rowsum, early);
+}
+
+template <int BITS>
+w4a8_status_t launch_quantize_static(const __half* a, int64_t M, int64_t K, const __half* sc, void* codes,
+                                     __half* so, int32_t* rowsum, cudaStream_t st) {
+  const dim3 grid(static_cast<unsigned>(M));
+  const int64_t nvec = K / 8;
+  const int early = M <= kEarlyReleaseRows ? 1 : 0;
+  if (nvec <= 128)
+    return launch_pdl(quantize_act_static_kernel<128, 1, BITS>, grid, dim3(128), 0, st, 1, a, K, sc, codes, so,
+                      rowsum, early);
+  if (nvec <= 512)
+    return launch_pdl(quantize_act_static_kernel<256, 2, BITS>, grid, dim3(256), 0, st, 1, a, K, sc, codes, so,
+                      rowsum, early);
+  if (nvec <= 2048)
+    return launch_pdl(quantize_act_static_kernel<256, 8, BITS>, grid, dim3(256), 0, st, 1, a, K, sc, codes, so,
+                      rowsum, early);
+  return launch_pdl(quantize_act_static_kernel<1024, 8, BITS>, grid, dim3(1024), 0, st, 1, a, K, sc, codes, so,
+                    rowsum, early);
+}
+
+w4a8_status_t check_quantize_args(const void* A, int64_t M, int64_t K, const void* codes, const void* sA,
+                                  const void* rowsum) {
+  if (M < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if (K == 0 || K % 8 != 0 || K > kMaxK || M > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (M == 0) return W4A8_OK;
+  if (A == nullptr || codes == nullptr || sA == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(codes, 16) || !aligned(sA, 2) || !aligned(rowsum, 4)) return W4A8_ERR_MISALIGNED;
+  return W4A8_OK;
+}
+
 }  // namespace
 
-w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+// A8: the int8 activation codes [M, K], or with a4 the packed 4-bit codes
+// [M, K / 2] (W4A4).
+w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
                         int64_t N, int64_t K, void* Y, int32_t* acc, void* ws, size_t ws_bytes,
-                        const w4a8_gemm_opts_t* opts, cudaStream_t stream) {
+                        const w4a8_gemm_opts_t* opts, cudaStream_t stream, int a4 = 0) {
   w4a8_gemm_opts_t o = {0, 0, 0, 0};
   if (opts != nullptr) o = *opts;
   if (o.reserved != 0 || o.schedule < 0 || o.schedule > 3 || o.max_ctas < 0) return W4A8_ERR_INVALID_ARG;
@@ -254,6 +313,28 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum,
   if (o.schedule == 3 && split == 1) return W4A8_ERR_UNSUPPORTED_SHAPE;
 
   const size_t need_ws = ws_counter_bytes(M, N) + static_cast<size_t>(M) * N * 4;
+  if (a4) {
+    // W4A4: expand the packed codes once into the workspace's scratch tail,
+    // then run the int8 GEMM on them (expanding inside the GEMM repeats the
+    // work for every output tile and, with one producer warp, limits the
+    // activation rate). Without room for the tail the GEMM expands them
+    // itself.
+    // The expanded codes occupy the LAST M * K bytes of the workspace (from a
+    // 256-byte boundary): a workspace sized for (M, N, K) then serves every
+    // smaller shape without its scratch ever touching a zero-filled prefix.
+    const size_t codes = static_cast<size_t>(M) * K;
+    const size_t tail = ws_bytes >= codes ? (ws_bytes - codes) / 256 * 256 : 0;
+    if (ws != nullptr && ws_bytes >= codes && tail >= need_ws) {
+      int8_t* A8x = static_cast<int8_t*>(ws) + tail;
+      const int64_t units = static_cast<int64_t>(codes / 16);
+      const int64_t blocks = (units + 255) / 256;
+      const int grid_x = static_cast<int>(blocks < 8L * dev->sms ? blocks : 8L * dev->sms);
+      st = launch_pdl(expand_act4_kernel, dim3(grid_x), dim3(256), 0, stream, 1, static_cast<const uint2*>(A8),
+                      units, reinterpret_cast<uint4*>(A8x));
+      if (st != W4A8_OK) return st;
+      return gemm_impl(A8x, sA, rowsum, packed, M, N, K, Y, acc, ws, tail, opts, stream, 0);
+    }
+  }
   const bool ws_ok = ws != nullptr && ws_bytes >= need_ws;
   // Tiles split stream-K (the rest go whole, round robin): everything when
   // the tiles do not fill one wave, else the tiles beyond the full waves, so
@@ -294,6 +375,7 @@ w4a8_status_t gemm_impl(const int8_t* A8, const void* sA, const int32_t* rowsum,
   a.num_tiles = num_tiles;
   a.sk_tiles = sk_tiles;
   a.split = split;
+  a.a4 = a4;
   switch (bn) {
     case 16: return launch_gemm_cfg<Cfg16>(A8, M, K, a, grid, stream);
     case 32: return launch_gemm_cfg<Cfg32>(A8, M, K, a, grid, stream);
@@ -325,48 +407,38 @@ int w4a8_version(void) { return 100; }
 
 w4a8_status_t w4a8_quantize_act(const void* A, int64_t M, int64_t K, int8_t* A8, void* sA, int32_t* rowsum,
                                 w4a8_stream_t stream) {
-  if (M < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
-  if (K == 0 || K % 8 != 0 || K > kMaxK || M > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
-  if (M == 0) return W4A8_OK;
-  if (A == nullptr || A8 == nullptr || sA == nullptr) return W4A8_ERR_INVALID_ARG;
-  if (!aligned(A, 16) || !aligned(A8, 16) || !aligned(sA, 2) || !aligned(rowsum, 4)) return W4A8_ERR_MISALIGNED;
-  const __half* a = static_cast<const __half*>(A);
-  __half* s = static_cast<__half*>(sA);
-  const dim3 grid(static_cast<unsigned>(M));
-  const int early = M <= kEarlyReleaseRows ? 1 : 0;
-  const int64_t nvec = K / 8;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (nvec <= 128) return launch_pdl(quantize_act_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, A8, s, rowsum, early);
-  if (nvec <= 256) return launch_pdl(quantize_act_kernel<256, 1>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
-  if (nvec <= 512) return launch_pdl(quantize_act_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
-  if (nvec <= 1024) return launch_pdl(quantize_act_kernel<256, 4>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
-  if (nvec <= 2048) return launch_pdl(quantize_act_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, A8, s, rowsum, early);
-  if (nvec <= 4096) return launch_pdl(quantize_act_kernel<512, 8>, grid, dim3(512), 0, st, 1, a, K, A8, s, rowsum, early);
-  return launch_pdl(quantize_act_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, A8, s, rowsum, early);
+  const w4a8_status_t st = check_quantize_args(A, M, K, A8, sA, rowsum);
+  if (st != W4A8_OK || M == 0) return st;
+  return launch_quantize_dynamic<8>(static_cast<const __half*>(A), M, K, A8, static_cast<__half*>(sA), rowsum,
+                                    reinterpret_cast<cudaStream_t>(stream));
 }
 
 w4a8_status_t w4a8_quantize_act_static(const void* A, int64_t M, int64_t K, const void* s, int8_t* A8, void* sA,
                                        int32_t* rowsum, w4a8_stream_t stream) {
-  if (M < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
-  if (K == 0 || K % 8 != 0 || K > kMaxK || M > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
-  if (M == 0) return W4A8_OK;
-  if (A == nullptr || s == nullptr || A8 == nullptr || sA == nullptr) return W4A8_ERR_INVALID_ARG;
-  if (!aligned(A, 16) || !aligned(A8, 16) || !aligned(s, 2) || !aligned(sA, 2) || !aligned(rowsum, 4))
-    return W4A8_ERR_MISALIGNED;
-  const __half* a = static_cast<const __half*>(A);
-  const __half* sc = static_cast<const __half*>(s);
-  __half* so = static_cast<__half*>(sA);
-  const dim3 grid(static_cast<unsigned>(M));
-  const int early = M <= kEarlyReleaseRows ? 1 : 0;
-  const int64_t nvec = K / 8;
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (nvec <= 128)
-    return launch_pdl(quantize_act_static_kernel<128, 1>, grid, dim3(128), 0, st, 1, a, K, sc, A8, so, rowsum, early);
-  if (nvec <= 512)
-    return launch_pdl(quantize_act_static_kernel<256, 2>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum, early);
-  if (nvec <= 2048)
-    return launch_pdl(quantize_act_static_kernel<256, 8>, grid, dim3(256), 0, st, 1, a, K, sc, A8, so, rowsum, early);
-  return launch_pdl(quantize_act_static_kernel<1024, 8>, grid, dim3(1024), 0, st, 1, a, K, sc, A8, so, rowsum, early);
+  const w4a8_status_t st = check_quantize_args(A, M, K, A8, sA, rowsum);
+  if (st != W4A8_OK || M == 0) return st;
+  if (s == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(s, 2)) return W4A8_ERR_MISALIGNED;
+  return launch_quantize_static<8>(static_cast<const __half*>(A), M, K, static_cast<const __half*>(s), A8,
+                                   static_cast<__half*>(sA), rowsum, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4a8_status_t w4a4_quantize_act(const void* A, int64_t M, int64_t K, uint8_t* A4, void* sA, int32_t* rowsum,
+                                w4a8_stream_t stream) {
+  const w4a8_status_t st = check_quantize_args(A, M, K, A4, sA, rowsum);
+  if (st != W4A8_OK || M == 0) return st;
+  return launch_quantize_dynamic<4>(static_cast<const __half*>(A), M, K, A4, static_cast<__half*>(sA), rowsum,
+                                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4a8_status_t w4a4_quantize_act_static(const void* A, int64_t M, int64_t K, const void* s, uint8_t* A4, void* sA,
+                                       int32_t* rowsum, w4a8_stream_t stream) {
+  const w4a8_status_t st = check_quantize_args(A, M, K, A4, sA, rowsum);
+  if (st != W4A8_OK || M == 0) return st;
+  if (s == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(s, 2)) return W4A8_ERR_MISALIGNED;
+  return launch_quantize_static<4>(static_cast<const __half*>(A), M, K, static_cast<const __half*>(s), A4,
+                                   static_cast<__half*>(sA), rowsum, reinterpret_cast<cudaStream_t>(stream));
 }
 
 w4a8_status_t w4a8_quantize_weights(const float* W, int64_t N, int64_t K, int32_t group, uint8_t* q, uint8_t* z,
@@ -416,6 +488,12 @@ size_t w4a8_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
   return ws_counter_bytes(M, N) + static_cast<size_t>(M) * N * 4;
 }
 
+size_t w4a4_gemm_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+  const size_t base = w4a8_gemm_workspace_bytes(M, N, K);
+  if (base == 0 || K <= 0) return base;
+  return (base + 255) / 256 * 256 + static_cast<size_t>(M) * K;
+}
+
 w4a8_status_t w4a8_gemm(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
                         int64_t N, int64_t K, void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
   return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
@@ -434,6 +512,19 @@ w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const int32_t* rows
                            const w4a8_gemm_opts_t* opts, w4a8_stream_t stream) {
   return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, acc, workspace, workspace_bytes, opts,
                    reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4a8_status_t w4a4_gemm(const uint8_t* A4, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+                        int64_t N, int64_t K, void* Y, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
+  return gemm_impl(A4, sA, rowsum, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream), 1);
+}
+
+w4a8_status_t w4a4_gemm_ex(const uint8_t* A4, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+                           int64_t N, int64_t K, void* Y, int32_t* acc, void* workspace, size_t workspace_bytes,
+                           const w4a8_gemm_opts_t* opts, w4a8_stream_t stream) {
+  return gemm_impl(A4, sA, rowsum, packed, M, N, K, Y, acc, workspace, workspace_bytes, opts,
+                   reinterpret_cast<cudaStream_t>(stream), 1);
 }
 
 w4a8_status_t w4a8_get_device_error(w4a8_stream_t stream, int32_t* code) {
