@@ -29,6 +29,9 @@ What the pages fix and what this file reads into them
 * 4-bit activations (W4A4): the W4A4KV4 models of "PrefixQuant ..." (Key
   Findings) with per-tensor static scales; readings of the 4-bit code range,
   rounding and nibble order are stated at `quantize_act4`.
+* Lookup-table weight-only GEMM ("Fast Matrix Multiplications for Lookup
+  Table-Quantized LLMs", FLUTE, abstract): readings at `lut_dequant` and
+  the section heading there.
 * Offline weight reordering ("QServe/QoQ" abstract: compute-aware weight
   reordering; "QUICK: Quantization-aware Interleaving and Conflict-free
   Kernel ...", abstract: offline interleaving; "Fast Matrix Multiplications
@@ -374,3 +377,154 @@ def w4a4_gemm(A4_packed, sA, q, z, s2, s1, group: int = GROUP) -> np.ndarray:
     4-bit activation codes A4 = unpack_act4(A4_packed); the same int32 sum and
     fp32 epilogue as the 8-bit GEMM."""
     return epilogue(gemm_acc(unpack_act4(A4_packed), dequant_weights(q, z, s2, group)), sA, s1)
+
+
+# ---------------------------------------------------------------------------
+# Lookup-table weight-only GEMM (FLUTE)
+# ---------------------------------------------------------------------------
+# "Fast Matrix Multiplications for Lookup Table-Quantized LLMs" (FLUTE,
+# abstract): weight-only quantization in which every weight is an index into
+# a non-uniform table (NormalFloat being the example), with a scale per group
+# of 128 inputs; the activations stay in 16-bit floating point, and the GEMM
+# fuses the table lookup with the matrix multiplication. The pages fix no
+# arithmetic; the readings here: 4-bit indices q into a 16-entry fp16 table
+# T, one fp16 scale s per (output channel, group of 128 inputs), the weight
+# W[n,k] = fp16_rn(float(T[q[n,k]]) * float(s[n, k // 128])) (the exact
+# product rounded once), fp16 activations A, and
+#   Y[m,n] = fp16_rn(sum_k A[m,k] * W[n,k]),
+# the sum exact here (fp64 of exact fp16 x fp16 products); the GPU sums in
+# fp32 in an unspecified order, within `lut_error_bound` of it.
+LUT_MAGIC = 0x544C3457  # b"W4LT" little-endian
+LUT_TILE_SCALE_BYTES = 2 * TILE_N  # 256
+LUT_TILE_BYTES = TILE_CODE_BYTES + LUT_TILE_SCALE_BYTES  # 8448
+
+
+def lut_dequant(q: np.ndarray, s: np.ndarray, T: np.ndarray, group: int = GROUP) -> np.ndarray:
+    """W[n,k] = fp16_rn(float(T[q[n,k]]) * float(s[n, k // group])): fp16 [N, K].
+    (The product of two fp16 values is exact in fp32, so this is one rounding.)"""
+    Tv = T.astype(np.float32)[q]
+    sk = np.repeat(s.astype(np.float32), group, axis=1)
+    return (Tv * sk).astype(np.float16)
+
+
+def lut_gemm_exact(A: np.ndarray, q, s, T, group: int = GROUP) -> np.ndarray:
+    """sum_k A[m,k] * W[n,k] in fp64 (exact products; fp64 sums, relative error
+    below K * 2**-53), [M, N] float64."""
+    W = lut_dequant(q, s, T, group)
+    return A.astype(np.float64) @ W.astype(np.float64).T
+
+
+def lut_gemm(A: np.ndarray, q, s, T, group: int = GROUP) -> np.ndarray:
+    """Y = fp16_rn(sum_k A[m,k] * W[n,k]) with the sum exact (fp64)."""
+    with np.errstate(over="ignore"):
+        return lut_gemm_exact(A, q, s, T, group).astype(np.float16)
+
+
+def lut_error_bound(A: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """Bound on |fp32-accumulated sum - exact sum| for sum_k A[m,k] W[n,k]:
+    gamma_K * sum_k |A W|, gamma_K = K u / (1 - K u), with u = 2**-23 (one
+    fp32 ulp per addition, which also covers additions that truncate rather
+    than round). The products themselves are exact in fp32."""
+    K = A.shape[1]
+    u = 2.0 ** -23
+    gamma = K * u / (1 - K * u)
+    return gamma * (np.abs(A.astype(np.float64)) @ np.abs(W.astype(np.float64)).T)
+
+
+def lut_quantize_weights(W: np.ndarray, T: np.ndarray, group: int = GROUP):
+    """Offline lookup-table quantization of fp32 W [N, K] with table T:
+    s[n,g] = fp16_rn(max |W_g| / max |T|) (fp32 divide; 0 -> 1), and q[n,k] the
+    index of the table entry nearest to W[n,k] / float(s) (fp32 divide; ties
+    to the lower index). Returns (q uint8 [N,K], s fp16 [N, K/group])."""
+    N, K = W.shape
+    G = K // group
+    Wg = W.reshape(N, G, group)
+    tmax = np.float32(np.max(np.abs(T.astype(np.float32))))
+    s = (np.max(np.abs(Wg), axis=2) / tmax).astype(np.float16)
+    s[s == 0] = np.float16(1.0)
+    t = Wg / s.astype(np.float32)[:, :, None]
+    dist = np.abs(t[..., None] - T.astype(np.float32)[None, None, None, :])
+    q = np.argmin(dist, axis=3).astype(np.uint8)  # argmin takes the first (lowest) index on ties
+    return q.reshape(N, K), s
+
+
+def lut_packed_bytes(N: int, K: int, group: int = GROUP) -> int:
+    """Header + (N/128)*(K/128) tiles of 8448 bytes + the table (16 fp16) padded to 64 bytes."""
+    return HEADER_BYTES + (N // TILE_N) * (K // TILE_K) * LUT_TILE_BYTES + 64
+
+
+def lut_code_byte_offset(r: int, kk: int):
+    """Byte offset inside a tile's code area of row r, in-tile k index kk, and
+    whether the index is the high nibble. Row r's indices for in-tile
+    k = 2j, 2j+1 share byte j of the row (k = 2j in bits 0-3); the row's 64
+    bytes are four 16-byte vectors, vector c at ((c * 128) + r) * 16, so 32
+    consecutive rows read 512 contiguous bytes."""
+    j, high = divmod(kk, 2)
+    c, b = divmod(j, 16)
+    return (c * TILE_N + r) * 16 + b, bool(high)
+
+
+def lut_pack_weights(q, s, T, group: int = GROUP) -> np.ndarray:
+    """Writes the lookup-table weight blob from its definition.
+
+    Header (64 bytes, little-endian): u32 magic 'W4LT', u32 version 1,
+    i64 N, i64 K, i32 group, u32 tile bytes (8448), u64 byte offset of the
+    table; the rest zero. Tile (nt, kt) starts at 64 + (nt*(K/128) + kt)*8448:
+    8192 index bytes (see `lut_code_byte_offset`), then the 128 rows' fp16
+    scales of group kt (256 bytes, row r at 8192 + 2r). After the tiles: the
+    16 fp16 table entries, zero padded to 64 bytes."""
+    assert group == GROUP
+    N, K = q.shape
+    KT = K // TILE_K
+    out = np.zeros(lut_packed_bytes(N, K, group), dtype=np.uint8)
+    t_off = HEADER_BYTES + (N // TILE_N) * KT * LUT_TILE_BYTES
+    hdr = bytearray(HEADER_BYTES)
+    hdr[0:4] = LUT_MAGIC.to_bytes(4, "little")
+    hdr[4:8] = (1).to_bytes(4, "little")
+    hdr[8:16] = int(N).to_bytes(8, "little", signed=True)
+    hdr[16:24] = int(K).to_bytes(8, "little", signed=True)
+    hdr[24:28] = int(group).to_bytes(4, "little", signed=True)
+    hdr[28:32] = LUT_TILE_BYTES.to_bytes(4, "little")
+    hdr[32:40] = int(t_off).to_bytes(8, "little")
+    out[:HEADER_BYTES] = np.frombuffer(bytes(hdr), dtype=np.uint8)
+    n = np.arange(N)[:, None, None]
+    kt = np.arange(KT)[None, :, None]
+    j = np.arange(64)[None, None, :]
+    r = n % TILE_N
+    k_lo = kt * TILE_K + 2 * j
+    byte = (q[n, k_lo].astype(np.uint16) | (q[n, k_lo + 1].astype(np.uint16) << 4)).astype(np.uint8)
+    c, b = j // 16, j % 16
+    dest = HEADER_BYTES + ((n // TILE_N) * KT + kt) * LUT_TILE_BYTES + (c * TILE_N + r) * 16 + b
+    out[dest.ravel()] = byte.ravel()
+    n = np.arange(N)[:, None]
+    g = np.arange(KT)[None, :]
+    sb = s.astype(np.float16).view(np.uint8).reshape(N, KT, 2)
+    sdest = HEADER_BYTES + (n // TILE_N * KT + g) * LUT_TILE_BYTES + TILE_CODE_BYTES + 2 * (n % TILE_N)
+    out[sdest.ravel()] = sb[:, :, 0].ravel()
+    out[sdest.ravel() + 1] = sb[:, :, 1].ravel()
+    out[t_off:t_off + 32] = np.frombuffer(T.astype(np.float16).tobytes(), dtype=np.uint8)
+    return out
+
+
+def lut_unpack_weights(blob: np.ndarray):
+    """Inverse of `lut_pack_weights`: returns (q, s, T, N, K)."""
+    hdr = bytes(blob[:HEADER_BYTES])
+    assert int.from_bytes(hdr[0:4], "little") == LUT_MAGIC
+    N = int.from_bytes(hdr[8:16], "little", signed=True)
+    K = int.from_bytes(hdr[16:24], "little", signed=True)
+    t_off = int.from_bytes(hdr[32:40], "little")
+    KT = K // TILE_K
+    n = np.arange(N)[:, None]
+    k = np.arange(K)[None, :]
+    nt, r = n // TILE_N, n % TILE_N
+    kt, kk = k // TILE_K, k % TILE_K
+    j, high = kk // 2, kk % 2
+    c, b = j // 16, j % 16
+    src = HEADER_BYTES + (nt * KT + kt) * LUT_TILE_BYTES + (c * TILE_N + r) * 16 + b
+    byte = blob[src]
+    q = np.where(high == 1, byte >> 4, byte & 0x0F).astype(np.uint8)
+    g = np.arange(KT)[None, :]
+    ssrc = HEADER_BYTES + (nt * KT + g) * LUT_TILE_BYTES + TILE_CODE_BYTES + 2 * r
+    s = (blob[ssrc].astype(np.uint16) | (blob[ssrc + 1].astype(np.uint16) << 8)).view(np.float16)
+    T = np.frombuffer(bytes(blob[t_off:t_off + 32]), dtype=np.float16).copy()
+    return q, s, T, N, K

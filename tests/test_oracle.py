@@ -554,3 +554,122 @@ def test_w4a4_gemm_brute_force():
             assert max_ulp_fp16(Y[m:m + 1, n:n + 1], np.array([[ref]])) <= 1, (m, n)
     # 4-bit codes are a subset of the 8-bit codes: the 8-bit GEMM fed with them agrees exactly
     assert (Y.view(np.uint16) == O.w4a8_gemm(A4, sA, q, z, s2, s1).view(np.uint16)).all()
+
+
+# ---------------------------------------------- lookup-table weights (FLUTE)
+def _fp16_is_nearest(c: np.float16, exact: Fraction) -> bool:
+    """c is an fp16 value nearest to `exact` (ties: even mantissa)."""
+    d = abs(Fraction(float(c)) - exact)
+    for nb in (np.nextafter(c, np.float16(np.inf)), np.nextafter(c, np.float16(-np.inf))):
+        dn = abs(Fraction(float(nb)) - exact)
+        if dn < d or (dn == d and int(np.float16(nb).view(np.uint16)) % 2 == 0 and int(c.view(np.uint16)) % 2 == 1):
+            return False
+    return True
+
+
+def test_lut_dequant_rounds_the_exact_product_once():
+    from w4a8_quantized_gemm_quantize_b200 import inputs as I
+    T = I.lut_table()
+    q, s = I.lut_codes(4, 256, 31)
+    W = O.lut_dequant(q, s, T)
+    for n in range(4):
+        for k in range(0, 256, 3):
+            exact = Fraction(float(T[q[n, k]])) * Fraction(float(s[n, k // 128]))
+            assert _fp16_is_nearest(W[n, k], exact), (n, k)
+    # a power-of-two scale is exact: W = T[q] * 2^-3
+    s8 = np.full((4, 2), np.float16(0.125))
+    assert (O.lut_dequant(q, s8, T).astype(np.float64) == T.astype(np.float64)[q] / 8).all()
+
+
+def test_lut_gemm_brute_force_and_one_hot():
+    from w4a8_quantized_gemm_quantize_b200 import inputs as I
+    T = I.lut_table()
+    M, N, K = 3, 5, 256
+    q, s = I.lut_codes(N, K, 32)
+    A = _rand_act(M, K, 33)
+    W = O.lut_dequant(q, s, T)
+    ex = O.lut_gemm_exact(A, q, s, T)
+    Y = O.lut_gemm(A, q, s, T)
+    for m in range(M):
+        for n in range(N):
+            exact = sum(Fraction(float(A[m, k])) * Fraction(float(W[n, k])) for k in range(K))
+            assert abs(Fraction(ex[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 40) + Fraction(1, 2 ** 60)
+            assert _fp16_is_nearest(Y[m, n], Fraction(ex[m, n]))
+    # one-hot rows select a weight column: exact, and exact again in fp16
+    A1 = np.zeros((4, K), dtype=np.float16)
+    cols = [0, 77, 128, 255]
+    for m, j in enumerate(cols):
+        A1[m, j] = 1.0
+    Y1 = O.lut_gemm(A1, q, s, T)
+    assert (Y1.view(np.uint16) == W[:, cols].T.view(np.uint16)).all()
+
+
+def test_lut_error_bound_covers_fp32_accumulation_orders():
+    from w4a8_quantized_gemm_quantize_b200 import inputs as I
+    T = I.lut_table()
+    M, N, K = 2, 3, 1024
+    q, s = I.lut_codes(N, K, 34)
+    A = _rand_act(M, K, 35)
+    W = O.lut_dequant(q, s, T)
+    ex = O.lut_gemm_exact(A, q, s, T)
+    bound = O.lut_error_bound(A, W)
+    rng = np.random.default_rng(36)
+    for m in range(M):
+        for n in range(N):
+            prods = A[m].astype(np.float32) * W[n].astype(np.float32)  # exact in fp32
+            for _ in range(4):
+                acc = np.float32(0)
+                for p in prods[rng.permutation(K)]:
+                    acc = np.float32(acc + p)
+                assert abs(float(acc) - ex[m, n]) <= bound[m, n]
+    assert (bound > 0).all()
+
+
+def test_lut_pack_hand_positions_and_roundtrip():
+    from w4a8_quantized_gemm_quantize_b200 import inputs as I
+    T = I.lut_table()
+    N, K = 128, 256
+    q = np.zeros((N, K), dtype=np.uint8)
+    q[3, 5] = 9    # row 3, k 5: byte j = 2 of vector 0 -> offset (0*128 + 3)*16 + 2 = 50, high nibble
+    q[3, 4] = 6    # same byte, low nibble
+    q[7, 128 + 37] = 12  # tile kt = 1, k 37: j = 18 -> vector 1, byte 2 -> (128 + 7)*16 + 2 = 2162, high
+    s = np.full((N, 2), np.float16(0.25))
+    s[3, 1] = np.float16(-1.5)
+    blob = O.lut_pack_weights(q, s, T)
+    assert O.lut_code_byte_offset(3, 5) == (50, True)
+    assert O.lut_code_byte_offset(7, 37) == (2162, True)
+    tile1 = 64 + 8448
+    assert blob[64 + 50] == (9 << 4) | 6
+    assert blob[tile1 + 2162] == 12 << 4
+    assert blob[tile1 + 8192 + 2 * 3:tile1 + 8192 + 2 * 3 + 2].view(np.float16)[0] == np.float16(-1.5)
+    assert int.from_bytes(bytes(blob[0:4]), "little") == 0x544C3457
+    t_off = int.from_bytes(bytes(blob[32:40]), "little")
+    assert t_off == 64 + 2 * 8448 and (blob[t_off:t_off + 32].view(np.float16) == T).all()
+    q2, s2, T2, N2, K2 = O.lut_unpack_weights(blob)
+    assert (q2 == q).all() and (s2 == s).all() and (N2, K2) == (N, K)
+    qr, sr = I.lut_codes(256, 384, 37)
+    q3, s3, _, _, _ = O.lut_unpack_weights(O.lut_pack_weights(qr, sr, T))
+    assert (q3 == qr).all() and (s3.view(np.uint16) == sr.view(np.uint16)).all()
+
+
+def test_lut_quantize_picks_the_nearest_entry():
+    from w4a8_quantized_gemm_quantize_b200 import inputs as I
+    T = I.lut_table()
+    W = np.random.default_rng(38).standard_normal((3, 256)).astype(np.float32) * np.float32(0.02)
+    W[1, :128] = 0  # an all-zero group: scale 1, index of the zero entry
+    q, s = O.lut_quantize_weights(W, T)
+    tmax = max(abs(Fraction(float(t))) for t in T)
+    for n in range(3):
+        for g in range(2):
+            grp = W[n, 128 * g:128 * (g + 1)]
+            am = max(abs(Fraction(float(v))) for v in grp)
+            if am == 0:
+                assert s[n, g] == np.float16(1)
+                assert (T[q[n, 128 * g:128 * (g + 1)]] == 0).all()
+                continue
+            want = np.float16(np.float32(float(am)) / np.float32(float(tmax)))
+            assert s[n, g].view(np.uint16) == want.view(np.uint16)
+            for k in range(128 * g, 128 * (g + 1), 5):
+                x = Fraction(float(np.float32(W[n, k]) / np.float32(s[n, g])))
+                d = [abs(x - Fraction(float(t))) for t in T]
+                assert d[q[n, k]] == min(d) and q[n, k] == d.index(min(d)), (n, k)

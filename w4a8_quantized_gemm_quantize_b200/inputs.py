@@ -113,3 +113,24 @@ def activation_seed(workload: str, M: int, K: int) -> int:
 
 def weight_seed(workload: str, N: int, K: int) -> int:
     return seed_of("weight", workload, N, K)
+
+
+# ------------------------------------------------ lookup-table weights (LUT)
+def lut_table(delta: float = 0.03) -> np.ndarray:
+    """A NormalFloat-style 16-entry table (input data for the lookup-table
+    GEMM): standard-normal quantiles at evenly spaced probabilities, 8 below
+    and 7 above an exact zero, each side scaled to reach -1 / +1; fp16."""
+    from scipy.special import ndtri
+    neg = ndtri(np.linspace(delta, 0.5, 9)[:-1])
+    pos = ndtri(np.linspace(0.5, 1.0 - delta, 8)[1:])
+    t = np.concatenate([neg / -neg.min(), [0.0], pos / pos.max()])
+    return t.astype(np.float16)
+
+
+def lut_codes(N: int, K: int, seed: int, group: int = GROUP):
+    """Lookup-table weights drawn directly: indices q ~ U[0,15] (uint8 [N,K])
+    and per-(row, group) scales s ~ U[0.005, 0.05] (fp16 [N, K/group])."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
+    s = rng.uniform(0.005, 0.05, size=(N, K // group)).astype(np.float16)
+    return q, s
