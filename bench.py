@@ -57,14 +57,23 @@ KERNEL_SOURCES = ("gemm.cuh", "ptx.cuh", "pack.cuh", "w4a8_api.cu")
 
 
 # ------------------------------------------------------------ workload facts
-def weight_bytes(N, K):
-    """Packed weight bytes a GEMM must stream: codes + meta + s1."""
+LUT_TILE_BYTES = 8448
+
+
+def weight_bytes(N, K, lut=False):
+    """Packed weight bytes a GEMM must stream: codes + meta + s1, or (lookup-
+    table weights) indices + row scales + the table."""
+    if lut:
+        return (N // 128) * (K // 128) * LUT_TILE_BYTES + 64
     return (N // 128) * (K // 128) * TILE_BYTES + 2 * N
 
 
-def algorithmic_bytes(M, N, K, act_bits=8):
+def algorithmic_bytes(M, N, K, act_bits=8, lut=False):
     """Bytes a W4A8 (W4A4: act_bits=4) GEMM must move at least: packed
-    weights, the activation codes, the activation scales, the fp16 output."""
+    weights, the activation codes, the activation scales, the fp16 output;
+    the lookup-table GEMM reads fp16 activations and no scales."""
+    if lut:
+        return weight_bytes(N, K, True) + 2 * M * K + 2 * M * N
     return weight_bytes(N, K) + M * K * act_bits // 8 + 2 * M + 2 * M * N
 
 
@@ -226,7 +235,7 @@ class ClockSampler:
 _ORACLE_WEIGHTS = {}
 
 
-def cpu_oracle_run(workload, budget_s, reps=1, act_bits=8):
+def cpu_oracle_run(workload, budget_s, reps=1, act_bits=8, lut=False):
     """Times the CPU oracle (activation quantization + GEMM with the fp32
     epilogue; 4-bit activations with act_bits=4) on this host over a bounded
     sample of the workload's cases; returns (weight GB/s, description of the
@@ -240,17 +249,25 @@ def cpu_oracle_run(workload, budget_s, reps=1, act_bits=8):
         if time.perf_counter() - t_start > budget_s and done:
             break
         wl = I.WORKLOADS[workload]
-        key = (workload, N, K)
-        if key not in prepared:
+        key = (workload, N, K, lut)
+        if key not in prepared and lut:
+            prepared[key] = I.lut_codes(N, K, I.weight_seed(workload + "-lut", N, K))
+        elif key not in prepared:
             if wl.weight_std == 0.0:
                 prepared[key] = I.uniform_codes(N, K, I.weight_seed(workload, N, K))
             else:
                 W = I.dense_weights(N, K, wl.weight_std, I.weight_seed(workload, N, K))
                 prepared[key] = O.quantize_weights(W)
-        q, z, s2, s1 = prepared[key]
         A = I.activations(M, K, I.activation_seed(workload, M, K))
         for _ in range(reps):
             t0 = time.perf_counter()
+            if lut:
+                q, s = prepared[key]
+                O.lut_gemm(A, q, s, I.lut_table())
+                done_time += time.perf_counter() - t0
+                done_bytes += weight_bytes(N, K, True)
+                continue
+            q, z, s2, s1 = prepared[key]
             if act_bits == 4:
                 A4, sA, _ = O.quantize_act4(A)
                 O.w4a4_gemm(O.pack_act4(A4), sA, q, z, s2, s1)
@@ -286,7 +303,16 @@ def run_gpu(args, world, rank, local):
 
     # ---- offline: quantize + pack the weights (untimed), one copy per M
     blobs = {}
+    lut = args.weights == "lut"
+    table = torch.from_numpy(I.lut_table()).to(dev) if lut else None
     for (name, N, K) in wl.linears:
+        if lut:
+            q, s = (torch.from_numpy(x).to(dev) for x in I.lut_codes(N, K, I.weight_seed(args.workload + "-lut", N, K)))
+            blobs[(name, 0)] = w4a8.lut_pack_weights(q, s, table)
+            del q, s
+            for c in range(1, n_copies):
+                blobs[(name, c)] = blobs[(name, 0)].clone()
+            continue
         if wl.weight_std == 0.0:
             q, z, s2, s1 = (torch.from_numpy(x).to(dev) for x in I.uniform_codes(N, K, I.weight_seed(args.workload, N, K)))
         else:
@@ -319,7 +345,12 @@ def run_gpu(args, world, rank, local):
         qmax = 127 if args.act == "static" else 7
         static_scales = {key: (A.float().abs().max() / qmax).to(torch.float16).reshape(1)
                          for key, A in acts.items()}
-    if ACT_BITS[args.act] == 4:
+    if lut:
+        quantize = None
+
+        def gemm(A8, sA, rs, blob, N, K, out, workspace):  # weight-only: the fp16 activations feed the GEMM
+            return w4a8.lut_gemm(A8, blob, N, K, out=out, workspace=workspace)
+    elif ACT_BITS[args.act] == 4:
         quantize = (w4a8.w4a4_quantize_act_static if static_scales is not None else w4a8.w4a4_quantize_act)
         gemm = w4a8.w4a4_gemm
     else:
@@ -332,7 +363,9 @@ def run_gpu(args, world, rank, local):
             if h2d is not None:
                 A.copy_(h2d[(M, name)], non_blocking=True)
             A8, sA, rs, Y = outs[(M, name)]
-            if not gemm_only:
+            if lut:
+                A8 = A
+            elif not gemm_only:
                 if static_scales is not None:
                     quantize(A, static_scales[(M, name)], out=(A8, sA, rs))
                 else:
@@ -461,6 +494,10 @@ def main():
                     help="activation codes and scales: 8-bit per-token dynamic (w4a8_quantize_act) or per-tensor "
                          "static calibrated once before timing (w4a8_quantize_act_static); 4-bit (W4A4: "
                          "w4a4_quantize_act / w4a4_quantize_act_static + w4a4_gemm)")
+    ap.add_argument("--weights", default="w4a8", choices=["w4a8", "lut"],
+                    help="w4a8: two-level 4-bit weights against quantized activations; lut: 4-bit indices into a "
+                         "16-entry fp16 table with group scales against fp16 activations (weight-only, "
+                         "w4lut_gemm)")
     ap.add_argument("--profile", type=int, default=0,
                     help="run this many eager steps for an external profiler and exit (no timing)")
     args = ap.parse_args()
@@ -482,8 +519,9 @@ def main():
         return 0
     cases = r["cases"]
     peaks = load_peaks()
-    wbytes = sum(weight_bytes(N, K) for (M, _, N, K) in cases)
-    abytes = [algorithmic_bytes(M, N, K, ACT_BITS[args.act]) for (M, _, N, K) in cases]
+    lut = args.weights == "lut"
+    wbytes = sum(weight_bytes(N, K, lut) for (M, _, N, K) in cases)
+    abytes = [algorithmic_bytes(M, N, K, ACT_BITS[args.act], lut) for (M, _, N, K) in cases]
     ops = [gemm_ops(M, N, K) for (M, _, N, K) in cases]
     ms_step = r["max_ms"] / args.steps
     value = world * wbytes / (ms_step * 1e-3) / 1e9
@@ -505,7 +543,8 @@ def main():
         achieved = sum(ops) / (gemm_ms * 1e-3) / 1e12
         roofline = {"bound": "tensor", "achieved": round(achieved, 1), "peak": int8_peak_tops,
                     "unit": "TOPS", "frac": round(achieved / int8_peak_tops, 4)}
-    traffic = recorded_traffic(args.workload) if ACT_BITS[args.act] == 8 else None
+    traffic = (recorded_traffic(args.workload + "-lut") if lut else
+               recorded_traffic(args.workload) if ACT_BITS[args.act] == 8 else None)
     roofline["traffic"] = traffic
     roofline["peak_source"] = (f"{peaks['source']} HBM copy" if hbm_bound else
                                f"{peaks['source']} sustained bf16 x {INT8_OVER_BF16:g} (nominal int8/bf16 ratio)")
@@ -517,14 +556,15 @@ def main():
     per_case = []
     for (M, name, N, K), t, b, o, rt in zip(cases, per, abytes, ops, roof_t):
         per_case.append({"M": M, "layer": name, "N": N, "K": K, "us_with_events": round(t * 1e3, 2),
-                         "weight_GBs": round(weight_bytes(N, K) / (t * 1e-3) / 1e9, 1),
+                         "weight_GBs": round(weight_bytes(N, K, lut) / (t * 1e-3) / 1e9, 1),
                          "tops": round(o / (t * 1e-3) / 1e12, 2), "roofline_frac": round(rt / t, 3)})
 
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": args.workload, "activation_scales": args.act, "cases": len(cases),
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16" if lut else "int8", "data": "synthetic",
+        "config": {"workload": args.workload, "weights": args.weights,
+                   "activation_scales": "none (fp16 activations)" if lut else args.act, "cases": len(cases),
                    "shapes": [f"M={M} {n} {N}x{K}" for (M, n, N, K) in cases][:: max(1, len(cases) // 16)],
                    "group": 128, "weights_per_step_MB": round(wbytes / 1e6, 1),
                    "l2": f"inputs larger than L2: {r['n_copies']} weight copies, {wbytes / 1e6:.0f} MB per step",
@@ -532,7 +572,10 @@ def main():
                    "timing": "value: one CUDA graph of K unrolled steps; roofline: a second such graph with "
                              "events around each GEMM"},
         "tops": round(tops, 2),
-        "gpu_launches": 2 * len(cases) * args.steps,  # timed region of `value`: quantize_act + gemm per case
+        # timed region of `value`, per case: the activation quantizer (none for
+        # the weight-only GEMM), the 4-bit expansion pre-pass (W4A4), the GEMM
+        "gpu_launches": (1 + (0 if lut else 1) + (1 if ACT_BITS[args.act] == 4 and not lut else 0))
+                        * len(cases) * args.steps,
         "roofline": roofline,
         "e2e": {"value": round(world * wbytes / (r["e2e_ms"] / args.steps * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"]},
@@ -541,7 +584,7 @@ def main():
         "gpu": r["gpu_name"],
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds, act_bits=ACT_BITS[args.act])
+        v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds, act_bits=ACT_BITS[args.act], lut=lut)
         line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
                                 "sample": f"{len(sample)} of {len(cases)} cases ({'; '.join(sample)}), "
                                           f"{t:.1f} s of oracle time"}
@@ -557,12 +600,13 @@ def main_reference(args, world, rank):
     if rank != 0:
         return
     cases = cases_of(args.workload)
-    cpu_oracle_run(args.workload, 0.0, act_bits=ACT_BITS[args.act])  # untimed warm-up (one case)
+    lut = args.weights == "lut"
+    cpu_oracle_run(args.workload, 0.0, act_bits=ACT_BITS[args.act], lut=lut)  # untimed warm-up (one case)
     t0 = time.perf_counter()
     tot_bytes, tot_t, samples = 0.0, 0.0, []
     for _ in range(args.steps):
         v, sample, threads, t = cpu_oracle_run(args.workload, args.cpu_seconds / max(args.steps, 1),
-                                               act_bits=ACT_BITS[args.act])
+                                               act_bits=ACT_BITS[args.act], lut=lut)
         tot_t += t
         tot_bytes += v * t * 1e9
         samples = sample
@@ -570,8 +614,8 @@ def main_reference(args, world, rank):
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-        "config": {"workload": args.workload, "cases": len(cases), "group": 128},
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16" if lut else "int8", "data": "synthetic",
+        "config": {"workload": args.workload, "weights": args.weights, "cases": len(cases), "group": 128},
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
                          "sample": f"per step: {len(samples)} of {len(cases)} cases ({'; '.join(samples)})"},

@@ -278,6 +278,57 @@ W4A8_API w4a8_status_t w4a4_gemm_ex(const uint8_t* A4, const void* sA, const int
                                     size_t workspace_bytes, const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
 
 /*
+ * Lookup-table weight-only GEMM (the LUT-quantized GEMM of "Fast Matrix
+ * Multiplications for Lookup Table-Quantized LLMs", FLUTE, abstract): every
+ * weight is a 4-bit index q into a 16-entry fp16 table T (NormalFloat-style
+ * tables, for instance), with one fp16 scale s per output channel and group
+ * of 128 inputs; the activations stay fp16. The pages fix no arithmetic;
+ * this library computes
+ *   W[n,k] = fp16_rn(float(T[q[n,k]]) * float(s[n, k/128]))   (exact product, one rounding)
+ *   Y[m,n] = fp16_rn(sum_k A[m,k] * W[n,k])
+ * with the products exact and the sum accumulated in fp32 in an unspecified
+ * order (so within K * 2^-23 * sum_k |A W| of the exact sum).
+ *
+ * Packed blob, little-endian: header (64 bytes: u32 magic "W4LT", u32 version
+ * 1, i64 N, i64 K, i32 group, u32 tile bytes 8448, u64 byte offset of the
+ * table, zeros); (N/128) x (K/128) tiles of 8448 bytes, tile (nt, kt) at
+ * 64 + (nt * K/128 + kt) * 8448: 8192 index bytes, byte j of row r's 64 bytes
+ * holding the indices of in-tile k = 2j (bits 0-3) and k = 2j+1 (bits 4-7),
+ * the row's 16-byte vector c at (c * 128 + r) * 16; then the 128 fp16 row
+ * scales of group kt (row r at 8192 + 2r); after the tiles the 16 fp16 table
+ * entries, zero padded to 64 bytes.
+ */
+
+/* Size in bytes of the lookup-table blob for an N x K weight (0 if unsupported). */
+W4A8_API size_t w4lut_packed_bytes(int64_t N, int64_t K, int32_t group);
+
+/*
+ * Packs q (uint8 [N, K], one index 0..15 per byte, 16-byte aligned), s (fp16
+ * [N, K/128], 2-byte aligned) and table (16 fp16 values, 2-byte aligned) into
+ * the blob above. Limits: group == 128, N % 128 == 0, K % 128 == 0,
+ * 0 < K <= 65536; packed_bytes >= w4lut_packed_bytes(N, K, group).
+ */
+W4A8_API w4a8_status_t w4lut_pack_weights(const uint8_t* q, const void* s, const void* table, int64_t N, int64_t K,
+                                          int32_t group, void* packed, size_t packed_bytes, w4a8_stream_t stream);
+
+/*
+ * Y fp16 [M, N] = the lookup-table GEMM of A (fp16 [M, K], 16-byte aligned)
+ * with the blob. workspace: as for w4a8_gemm, sized by
+ * w4a8_gemm_workspace_bytes(M, N, K) (its partial sums hold fp32 here).
+ * Limits as for w4a8_gemm.
+ */
+W4A8_API w4a8_status_t w4lut_gemm(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
+                                  void* workspace, size_t workspace_bytes, w4a8_stream_t stream);
+
+/*
+ * w4lut_gemm with overrides (block_m 0, 16 or 32 only): exactly one of Y and
+ * acc (fp32 [M, N], the sums before the rounding to fp16) must be non-NULL.
+ */
+W4A8_API w4a8_status_t w4lut_gemm_ex(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
+                                     float* acc, void* workspace, size_t workspace_bytes,
+                                     const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
+
+/*
  * Allocation-free GEMM: the same computation and results as w4a8_gemm, for
  * callers that cannot hand the library a workspace. This entry point has no
  * counterpart in the papers; it exists for deployment. Typical callers: a

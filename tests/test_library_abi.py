@@ -24,7 +24,7 @@ def L():
 
 def declared_functions():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4a[48]_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4(?:a[48]|lut)_\w+)\s*\(", src)))
 
 
 def test_header_declares_entry_points():
@@ -149,3 +149,22 @@ def test_python_binding_refuses_cpu_tensors(L):
     torch = pytest.importorskip("torch")
     with pytest.raises(w4a8.W4A8Error):
         w4a8.quantize_act(torch.zeros((2, 128), dtype=torch.float16))
+
+
+def test_lut_validation(L):
+    assert L.w4lut_packed_bytes(256, 512, 128) == 64 + 2 * 4 * 8448 + 64
+    assert L.w4lut_packed_bytes(200, 512, 128) == 0
+    p = L.w4lut_pack_weights
+    nb = L.w4lut_packed_bytes(256, 256, 128)
+    assert p(FAKE, FAKE, FAKE, 200, 256, 128, FAKE, nb, None) == 2
+    assert p(FAKE, FAKE, None, 256, 256, 128, FAKE, nb, None) == 1       # no table
+    assert p(FAKE, FAKE, FAKE, 256, 256, 128, FAKE, nb - 1, None) == 1
+    assert p(FAKE_ODD, FAKE, FAKE, 256, 256, 128, FAKE, nb, None) == 3
+    g = L.w4lut_gemm
+    assert g(FAKE, FAKE, 4, 100, 256, FAKE, None, 0, None) == 2           # N % 128
+    assert g(FAKE, FAKE, 4, 128, 200, FAKE, None, 0, None) == 2           # K % 128
+    assert g(FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1           # no Y
+    assert g(FAKE_ODD, FAKE, 4, 128, 256, FAKE, None, 0, None) == 3
+    assert g(FAKE, FAKE, 0, 128, 256, FAKE, None, 0, None) == 0           # M == 0: no-op
+    bad = w4a8.GemmOpts(0, 64, 0, 0)                                       # 64-token tiles: not for this GEMM
+    assert L.w4lut_gemm_ex(FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1

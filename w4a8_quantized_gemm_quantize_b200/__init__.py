@@ -20,7 +20,8 @@ __all__ = [
     "quantize_weights", "packed_bytes", "pack_weights", "workspace_bytes", "Workspace", "gemm",
     "gemm_debug_acc", "gemm_ex", "gemm_noalloc", "get_device_error", "clear_device_error",
     "selftest_bounded_wait", "quantize_act_static", "w4a4_quantize_act", "w4a4_quantize_act_static",
-    "w4a4_gemm", "w4a4_gemm_ex", "w4a4_workspace_bytes",
+    "w4a4_gemm", "w4a4_gemm_ex", "w4a4_workspace_bytes", "lut_packed_bytes", "lut_pack_weights", "lut_gemm",
+    "lut_gemm_ex",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -32,6 +33,7 @@ EXPORTED_SYMBOLS = (
     "w4a8_gemm_debug_acc", "w4a8_gemm_ex", "w4a8_get_device_error", "w4a8_clear_device_error",
     "w4a8_gemm_noalloc", "w4a8_selftest_bounded_wait", "w4a8_quantize_act_static",
     "w4a4_quantize_act", "w4a4_quantize_act_static", "w4a4_gemm", "w4a4_gemm_ex", "w4a4_gemm_workspace_bytes",
+    "w4lut_packed_bytes", "w4lut_pack_weights", "w4lut_gemm", "w4lut_gemm_ex",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
@@ -80,6 +82,10 @@ def lib() -> ctypes.CDLL:
         "w4a4_quantize_act_static": (ctypes.c_int, [vp, i64, i64, vp, vp, vp, vp, vp]),
         "w4a4_gemm": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, sz, vp]),
         "w4a4_gemm_workspace_bytes": (sz, [i64, i64, i64]),
+        "w4lut_packed_bytes": (sz, [i64, i64, i32]),
+        "w4lut_pack_weights": (ctypes.c_int, [vp, vp, vp, i64, i64, i32, vp, sz, vp]),
+        "w4lut_gemm": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "w4lut_gemm_ex": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, vp, sz, ctypes.POINTER(GemmOpts), vp]),
         "w4a4_gemm_ex": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, sz,
                                         ctypes.POINTER(GemmOpts), vp]),
     }
@@ -363,6 +369,58 @@ def w4a4_gemm(A4, sA, rowsum, blob, N: int, K: int, out=None, workspace=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().w4a4_gemm(_ptr(A4), _ptr(sA), _ptr(rowsum), _ptr(blob), M, N, K, _ptr(Y), _ptr(workspace),
                            ws_bytes, _stream(A4.device)), "w4a4_gemm")
+    return Y
+
+
+# ---------------------------------------------- lookup-table weight-only GEMM
+def lut_packed_bytes(N: int, K: int, group: int = 128) -> int:
+    return int(lib().w4lut_packed_bytes(N, K, group))
+
+
+def lut_pack_weights(q, s, table, group: int = 128):
+    """Indices q uint8 [N, K], scales s fp16 [N, K/128], table fp16 [16] -> blob."""
+    torch = _torch()
+    _require_cuda(q, s, table)
+    N, K = q.shape
+    nbytes = lut_packed_bytes(N, K, group)
+    if nbytes == 0:
+        raise W4A8Error(f"unsupported weight shape {N}x{K} (group {group})")
+    blob = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
+    _check(lib().w4lut_pack_weights(_ptr(q), _ptr(s), _ptr(table), N, K, group, _ptr(blob), nbytes,
+                                    _stream(q.device)), "w4lut_pack_weights")
+    return blob
+
+
+def lut_gemm_ex(A, blob, N: int, K: int, Y=None, acc=None, workspace=None, schedule=0, block_m=0, max_ctas=0):
+    """Lookup-table GEMM of fp16 A [M, K]: fp16 Y and/or (acc given) the fp32
+    sums before rounding; scheduling overrides as gemm_ex (block_m 0/16/32)."""
+    torch = _torch()
+    _require_cuda(A, blob, Y, acc, workspace)
+    if A.dtype != torch.float16 or A.dim() != 2 or A.shape[1] != K:
+        raise W4A8Error("A must be fp16 [M, K]")
+    M = A.shape[0]
+    if workspace is None:
+        workspace = _workspace_for(A.device, M, N, K)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    o = ctypes.byref(GemmOpts(schedule, block_m, max_ctas, 0))
+    _check(lib().w4lut_gemm_ex(_ptr(A), _ptr(blob), M, N, K, _ptr(Y), _ptr(acc), _ptr(workspace), ws_bytes, o,
+                               _stream(A.device)), "w4lut_gemm_ex")
+    return Y if Y is not None else acc
+
+
+def lut_gemm(A, blob, N: int, K: int, out=None, workspace=None):
+    """Y fp16 [M, N] = fp16(sum_k A[m,k] * fp16(T[q[n,k]] * s[n,k/128]))."""
+    torch = _torch()
+    _require_cuda(A, blob, out, workspace)
+    if A.dtype != torch.float16 or A.dim() != 2 or A.shape[1] != K:
+        raise W4A8Error("A must be fp16 [M, K]")
+    M = A.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A.device)
+    if workspace is None:
+        workspace = _workspace_for(A.device, M, N, K)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().w4lut_gemm(_ptr(A), _ptr(blob), M, N, K, _ptr(Y), _ptr(workspace), ws_bytes, _stream(A.device)),
+           "w4lut_gemm")
     return Y
 
 

@@ -63,6 +63,7 @@ struct GemmArgs {
   int sk_tiles;          // the first sk_tiles tiles are split stream-K over all CTAs
   int split;             // > 1: cluster split-K, `split` CTAs (one cluster) per tile
   int a4;                // activation codes are 4-bit, two per byte (W4A4), unpacked in shared memory
+  const __half* lut_table;  // lookup-table weights: the 16 fp16 table entries (inside the blob)
 };
 
 struct Seg {
@@ -127,9 +128,20 @@ struct Sched {
   }
 };
 
-template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_, int NMMA_>
+// Lookup-table weight tiles (weight-only GEMM, "Fast Matrix Multiplications
+// for Lookup Table-Quantized LLMs"): 8192 index bytes + 128 fp16 row scales.
+constexpr int kLutTileBytes = kTileCodeBytes + 2 * kTileN;  // 8448
+
+template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_, int NMMA_, bool LUT_ = false>
 struct GemmCfg {
   static constexpr int BN = BN_, KS = KS_, NS = NS_, NT = NT_, DQ = DQ_, NACC = NACC_, NMMA = NMMA_;
+  // LUT: lookup-table weights against fp16 activations (kind::f16 MMA, fp32
+  // accumulators); otherwise two-level 4-bit weights against int8 (kind::i8)
+  static constexpr bool kLut = LUT_;
+  static constexpr int kTileB = kLut ? kLutTileBytes : kTileBytes;  // packed bytes of one weight tile
+  static constexpr int kKbCols = kLut ? 64 : 32;                    // TMEM columns of one dequantized k-block
+  static constexpr int kMmaPerKb = kLut ? 8 : 4;                    // MMAs per k-block (K = 16 / 32)
+  static constexpr int kLutTableBytes = kLut ? 256 * 32 * 4 : 0;    // pair table, one copy per lane
   // One CTA per SM, persistent. Work moves in chunks of up to KS k-blocks of
   // one tile (one weight copy, one wait and one commit per chunk amortize the
   // fixed latencies of the synchronization operations).
@@ -151,9 +163,9 @@ struct GemmCfg {
   static constexpr int kDqWarp0 = 4;
   static constexpr int kEpWarp0 = 4 + 4 * DQ;
   static constexpr int kThreads = 32 * (4 + 4 * DQ + 4);
-  static constexpr int kA8Bytes = BN * 128;        // one k-block of activations
+  static constexpr int kA8Bytes = BN * (kLut ? 256 : 128);  // one k-block of activations
   static constexpr int kASlot = KS * kA8Bytes;
-  static constexpr int kWSlot = KS * kTileBytes;   // KS consecutive packed tiles
+  static constexpr int kWSlot = KS * kTileB;                // KS consecutive packed tiles
   static_assert(NMMA == 1 || NMMA == 2, "one or two MMA issuers (warps 1 and 2)");
   // Launch overlap for the small-token (decode) configurations, whose
   // launches are short enough for start-up and hand-over latency to matter:
@@ -169,20 +181,28 @@ struct GemmCfg {
   // full-ring start delayed the first weight bytes by ~1 us per launch).
   static constexpr int kStartChunks = kEarlyStart ? (NS < 2 ? NS : 2) : 0;
   static constexpr int kTmemA = NACC * BN;  // accumulators first, then the TMEM weight ring
-  static constexpr int kTSlotCols = KS * 32;
+  static constexpr int kTSlotCols = KS * kKbCols;
   // tensor memory columns allocated (a power of two >= 32)
   static constexpr int kTmemCols = kTmemA + NT * kTSlotCols <= 256 ? 256 : 512;
   static_assert(kTmemA + NT * kTSlotCols <= kTmemCols, "tensor memory budget");
-  static_assert(NT > DQ, "every dequantizer group needs a TMEM slot of its own");
   static_assert(NS >= 2 && NT >= 2, "two slots per ring at least");
-  // Several dequantizer groups wait on the weight ring out of order; bounding
-  // them by the TMEM ring keeps every parity wait within one phase.
+  // Chunk c goes to dequantizer group c % DQ and to MMA issuer c % NMMA, and
+  // every ring barrier is waited on by phase parity. A parity wait is exact
+  // only if the waiting thread itself waited on the slot's previous phase
+  // (the barrier is then at most one phase ahead): were a slot shared by two
+  // groups or two issuers, a thread could find it one phase behind, and the
+  // wait would pass on the stale parity (a TMEM slot or an activation slot
+  // read before it is written). So every slot of a ring belongs to one
+  // dequantizer group and one issuer: each ring depth is a multiple of both.
+  static_assert(NS % DQ == 0 && NT % DQ == 0, "ring depths a multiple of the dequantizer groups");
+  static_assert(NS % NMMA == 0 && NT % NMMA == 0, "ring depths a multiple of the MMA issuers");
   static_assert(NS >= NT, "weight ring at least as deep as the TMEM ring");
   // With enough TMEM slots a group keeps a chunk's TMEM stores in flight
   // while it loads its next chunk (it publishes chunk c only when it starts
   // chunk c + DQ, which must not need a slot that chunk c + 1 still holds);
   // otherwise it completes them within the chunk.
   static constexpr bool kPipelinedStores = NT >= 2 * DQ && NT >= DQ + 2;
+  static_assert(!(kLut && kPipelinedStores), "the lookup-table dequantizer completes its stores per chunk");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
   // Cluster split-K (small BN only): up to kMaxSplit CTAs per tile. The
   // owner of TMEM lane quarter q is cluster rank q % split; it receives the
@@ -195,7 +215,8 @@ struct GemmCfg {
   static constexpr int kOffA8 = 0;                 // 1024-aligned activation slots
   static constexpr int kOffW = NS * kASlot;        // 16-aligned weight slots
   static constexpr int kOffRecv = kOffW + NS * kWSlot;
-  static constexpr int kOffBar = (kOffRecv + kRecvSlots * kRecvSlotBytes + 15) / 16 * 16;
+  static constexpr int kOffLut = (kOffRecv + kRecvSlots * kRecvSlotBytes + 15) / 16 * 16;
+  static constexpr int kOffBar = kOffLut + kLutTableBytes;
   // + one receive barrier per lane quarter + one packed-activation barrier per slot
   static constexpr int kNumBars = 4 * NS + 2 * NT + 2 * NACC + 1 + 4 + NS;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
@@ -239,6 +260,47 @@ __device__ __forceinline__ void dequant_tile_regs(const uint8_t* wt, int r, uint
   }
 }
 
+// Dequantizes half h (in-tile k = 64h .. 64h+63) of row r of a lookup-table
+// weight tile into 32 registers, register c holding the fp16 pair for
+// k = 64h + 2c, 2c+1 (low half first, the column order of the TMEM A operand):
+// W = fp16_rn(T[index] * s) by one 32-bit lookup of the pair table (entry e
+// holds T[e & 15], T[e >> 4], the two indices of one byte) and one fp16x2
+// multiply by the row's group scale s. The pair table has one copy per lane
+// (entry e of copy l at word e * 32 + l, bank l), so a warp's lookups never
+// conflict ("Fast Matrix Multiplications for Lookup Table-Quantized LLMs",
+// abstract: vectorized and duplicated lookup table).
+__device__ __forceinline__ void lut_dequant_half(const uint8_t* wt, int r, int h, const uint32_t* lut, int lane,
+                                                 uint32_t (&out)[32]) {
+  const __half sc = *reinterpret_cast<const __half*>(wt + kTileCodeBytes + 2 * r);
+  const __half2 ss = __halves2half2(sc, sc);
+#pragma unroll
+  for (int cc = 0; cc < 2; ++cc) {
+    const uint4 v = *reinterpret_cast<const uint4*>(wt + ((2 * h + cc) * kTileN + r) * 16);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t e = (w[jj] >> (8 * b)) & 0xFFu;
+        const uint32_t pair = lut[e * 32 + lane];
+        const __half2 x = __hmul2(*reinterpret_cast<const __half2*>(&pair), ss);
+        out[cc * 16 + jj * 4 + b] = *reinterpret_cast<const uint32_t*>(&x);
+      }
+    }
+  }
+}
+
+// Accumulator words: int32 sums (biased, see store_output) or, for the
+// lookup-table GEMM, fp32 bit patterns.
+template <bool LUT>
+__device__ __forceinline__ uint32_t acc_add(uint32_t a, uint32_t b) {
+  if constexpr (LUT) {
+    return __float_as_uint(__uint_as_float(a) + __uint_as_float(b));
+  } else {
+    return a + b;
+  }
+}
+
 // Per-token operands of the epilogue, staged in shared memory per segment:
 // thread t of the epilogue group loads token m0 + t before the group waits
 // for the accumulator (one global load per thread, hidden behind the
@@ -254,6 +316,7 @@ struct RowStage {
   int32_t* rowsum;  // [128]
   float* sa;        // [128]
   __device__ __forceinline__ void load(const GemmArgs& a, int m0, int t, int rows) {
+    if (a.rowsum == nullptr) return;  // lookup-table GEMM: no per-token operands
     if (t < rows) {
       const int m = m0 + t;
       const int mc = m < a.M ? m : a.M - 1;
@@ -286,6 +349,39 @@ __device__ __forceinline__ __half output_half(uint32_t biased, int32_t rowsum, f
   return __float2half_rn(__fmul_rn(__int2float_rn(acc), __fmul_rn(sa, s1f)));
 }
 
+// The same two for either kind of accumulator: the lookup-table GEMM's fp32
+// sum is the output before rounding to fp16 (the scales were applied to the
+// weights); the raw accumulator output holds its bit pattern.
+template <bool LUT>
+__device__ __forceinline__ void store_out(const GemmArgs& a, int64_t o, uint32_t v, int32_t rowsum, float sa,
+                                          float s1f) {
+  if constexpr (LUT) {
+    if (a.acc_out != nullptr) {
+      a.acc_out[o] = static_cast<int32_t>(v);
+    } else {
+      a.Y[o] = __float2half_rn(__uint_as_float(v));
+    }
+  } else {
+    store_output(a, o, v, rowsum, sa, s1f);
+  }
+}
+template <bool LUT>
+__device__ __forceinline__ __half out_half(uint32_t v, int32_t rowsum, float sa, float s1f) {
+  if constexpr (LUT) {
+    return __float2half_rn(__uint_as_float(v));
+  } else {
+    return output_half(v, rowsum, sa, s1f);
+  }
+}
+template <bool LUT>
+__device__ __forceinline__ void red_add_acc(int32_t* p, uint32_t v) {
+  if constexpr (LUT) {
+    red_add_f32(reinterpret_cast<float*>(p), __uint_as_float(v));
+  } else {
+    red_add_s32(p, static_cast<int32_t>(v));
+  }
+}
+
 // Stores a warp's 16 rows x 32 channels of fp16 output (lane = channel
 // n_base + lane, h[j] = row m_start + j) with 16-byte stores: the block is
 // transposed through the warp's 1 KB shared-memory stage so that each
@@ -310,7 +406,7 @@ __device__ __forceinline__ void store_y_rows16(const GemmArgs& a, __half* stage,
 // first lane's accumulator; lane j's accumulator is `lane_stride * j`
 // columns further; bit j of `lanes_used` says whether lane j holds a partial
 // sum for this segment. Returns false if the group has to abort.
-template <int BN>
+template <int BN, bool LUT>
 __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg& sg, bool ok_in, uint64_t* accfull,
                                                  uint32_t bph, uint64_t* accempty, uint32_t tacc,
                                                  uint32_t lane_stride, uint32_t lanes_used, int quarter, int lane,
@@ -321,7 +417,7 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
   const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
   const int m0 = m_tile * BN;
   const bool whole = (sg.kb0 == 0 && sg.kb1 == args.KB);
-  const float s1f = __half2float(args.s1[n]);
+  const float s1f = LUT ? 1.0f : __half2float(args.s1[n]);
   named_bar_sync(1, 128);  // the previous segment's reads of the stage are done
   rows.load(args, m0, quarter * 32 + lane, BN);
   // the four warps take one decision, so every named barrier below is
@@ -343,7 +439,7 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
         uint32_t u[16];
         tmem_ld_16_wait(tacc + l * lane_stride + c, u);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] += u[j];
+        for (int j = 0; j < 16; ++j) v[j] = acc_add<LUT>(v[j], u[j]);
       }
     }
     tmem_zero_16(tacc + c);  // every MMA accumulates: the buffer starts the next segment at zero
@@ -358,18 +454,18 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int m = m0 + c + j;
-        if (m < args.M) red_add_s32(args.ws_acc + static_cast<int64_t>(m) * N + n, static_cast<int32_t>(v[j]));
+        if (m < args.M) red_add_acc<LUT>(args.ws_acc + static_cast<int64_t>(m) * N + n, v[j]);
       }
     } else if (args.acc_out != nullptr) {
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int m = m0 + c + j;
-        if (m < args.M) store_output(args, static_cast<int64_t>(m) * N + n, v[j], rsv[j], sav[j], s1f);
+        if (m < args.M) store_out<LUT>(args, static_cast<int64_t>(m) * N + n, v[j], rsv[j], sav[j], s1f);
       }
     } else {
       __half h[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) h[j] = output_half(v[j], rsv[j], sav[j], s1f);
+      for (int j = 0; j < 16; ++j) h[j] = out_half<LUT>(v[j], rsv[j], sav[j], s1f);
       store_y_rows16(args, ystage, h, m0 + c, n - lane, lane);
     }
   }
@@ -408,7 +504,7 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
           if (m < args.M) {
             const int64_t o = static_cast<int64_t>(m) * N + n;
             __stcg(args.ws_acc + o, 0);
-            store_output(args, o, v[j], rows.rowsum[c + j], rows.sa[c + j], s1f);
+            store_out<LUT>(args, o, v[j], rows.rowsum[c + j], rows.sa[c + j], s1f);
           }
         }
       }
@@ -436,7 +532,7 @@ __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg
   const int64_t N = args.N;
   const int64_t n = static_cast<int64_t>(n_tile) * kTileN + quarter * 32 + lane;
   const int m0 = m_tile * BN;
-  const float s1f = __half2float(args.s1[n]);
+  const float s1f = C::kLut ? 1.0f : __half2float(args.s1[n]);
   rows.load(args, m0, quarter * 32 + lane, BN);  // made visible by the barrier after the accumulator wait
   cluster_wait();                                // every receive barrier of the cluster is armed
   bool ok = mbar_wait(accfull, 0, abort_flag, err, kErrEpilogue);
@@ -456,7 +552,7 @@ __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg
         uint32_t u[16];
         tmem_ld_16_wait(tacc + l * BN + c, u);
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[c + j] += u[j];
+        for (int j = 0; j < 16; ++j) v[c + j] = acc_add<C::kLut>(v[c + j], u[j]);
       }
     }
   }
@@ -482,13 +578,13 @@ __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg
   for (int sidx = 0; sidx < S - 1; ++sidx) {
     const uint32_t* src = recv + (slot0 + sidx) * (C::kRecvSlotBytes / 4) + lane;
 #pragma unroll
-    for (int j = 0; j < BN; ++j) v[j] += src[j * 32];
+    for (int j = 0; j < BN; ++j) v[j] = acc_add<C::kLut>(v[j], src[j * 32]);
   }
   if (args.acc_out != nullptr) {
 #pragma unroll
     for (int j = 0; j < BN; ++j) {
       const int m = m0 + j;
-      if (m < args.M) store_output(args, static_cast<int64_t>(m) * N + n, v[j], rows.rowsum[j], rows.sa[j], s1f);
+      if (m < args.M) store_out<C::kLut>(args, static_cast<int64_t>(m) * N + n, v[j], rows.rowsum[j], rows.sa[j], s1f);
     }
     return true;
   }
@@ -496,7 +592,7 @@ __device__ __forceinline__ bool epilogue_cluster(const GemmArgs& args, const Seg
   for (int c = 0; c < BN; c += 16) {
     __half h[16];
 #pragma unroll
-    for (int j = 0; j < 16; ++j) h[j] = output_half(v[c + j], rows.rowsum[c + j], rows.sa[c + j], s1f);
+    for (int j = 0; j < 16; ++j) h[j] = out_half<C::kLut>(v[c + j], rows.rowsum[c + j], rows.sa[c + j], s1f);
     store_y_rows16(args, ystage, h, m0 + c, n - lane, lane);
   }
   return true;
@@ -709,11 +805,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       Seg g0;
       int c = 0;
       while (c < C::kStartChunks && s0.next(g0)) {
-        const uint8_t* wsrc = args.tiles + static_cast<int64_t>(g0.tile / args.m_tiles) * args.KB * kTileBytes;
+        const uint8_t* wsrc = args.tiles + static_cast<int64_t>(g0.tile / args.m_tiles) * args.KB * C::kTileB;
         for (int kb = g0.kb0; kb < g0.kb1 && c < C::kStartChunks; kb += KS, ++c) {
           const int cnt = min(KS, g0.kb1 - kb);
-          mbar_arrive_expect_tx(&wfull[c], cnt * kTileBytes);
-          bulk_load(sW + c * C::kWSlot, wsrc + static_cast<int64_t>(kb) * kTileBytes, cnt * kTileBytes, &wfull[c],
+          mbar_arrive_expect_tx(&wfull[c], cnt * C::kTileB);
+          bulk_load(sW + c * C::kWSlot, wsrc + static_cast<int64_t>(kb) * C::kTileB, cnt * C::kTileB, &wfull[c],
                     pol_w);
         }
       }
@@ -748,6 +844,15 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     fence_barrier_init();
     fence_proxy_async_smem();
   }
+  if constexpr (C::kLut) {
+    // pair table: entry e = (T[e & 15], T[e >> 4]) as fp16x2, one copy per lane
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::kOffLut);
+    const uint16_t* T = reinterpret_cast<const uint16_t*>(args.lut_table);
+    for (int i = threadIdx.x; i < 256 * 32; i += C::kThreads) {
+      const int e = i >> 5;
+      lut[i] = static_cast<uint32_t>(__ldg(T + (e & 15))) | (static_cast<uint32_t>(__ldg(T + (e >> 4))) << 16);
+    }
+  }
   if (warp == 0) {
     tmem_alloc(&misc[0], C::kTmemCols);
     tmem_relinquish();
@@ -777,7 +882,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
       int c = 0;
       bool ok = true;
       while (ok && sch.next(sg)) {
-        const uint8_t* wsrc = args.tiles + static_cast<int64_t>(sg.tile / args.m_tiles) * args.KB * kTileBytes;
+        const uint8_t* wsrc = args.tiles + static_cast<int64_t>(sg.tile / args.m_tiles) * args.KB * C::kTileB;
         for (int kb = sg.kb0; kb < sg.kb1; kb += KS, ++c) {
           if (c < C::kStartChunks) continue;
           const int cnt = min(KS, sg.kb1 - kb);
@@ -786,8 +891,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&wfull[w], cnt * kTileBytes);
-          bulk_load(sW + w * C::kWSlot, wsrc + static_cast<int64_t>(kb) * kTileBytes, cnt * kTileBytes, &wfull[w],
+          mbar_arrive_expect_tx(&wfull[w], cnt * C::kTileB);
+          bulk_load(sW + w * C::kWSlot, wsrc + static_cast<int64_t>(kb) * C::kTileB, cnt * C::kTileB, &wfull[w],
                     pol_w);
         }
       }
@@ -803,7 +908,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     __syncwarp();
   } else if (warp == 3 && args.a4) {
     // -------------------------------- activation producer, 4-bit activations
-    act4_producer<C>(args, &tmap_a, sA8, afull, aempty, astage, lane, dep_done, abort_flag, err);
+    if constexpr (!C::kLut) act4_producer<C>(args, &tmap_a, sA8, afull, aempty, astage, lane, dep_done, abort_flag, err);
   } else if (warp == 3) {
     // ------------------------------------------------- activation producer
     if (lane == 0) {
@@ -821,8 +926,16 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
             break;
           }
           mbar_arrive_expect_tx(&afull[a], cnt * C::kA8Bytes);
-          for (int j = 0; j < cnt; ++j)
-            tma_load_2d(sA8 + a * C::kASlot + j * C::kA8Bytes, &tmap_a, &afull[a], (kb + j) * 128, m0);
+          for (int j = 0; j < cnt; ++j) {
+            if constexpr (C::kLut) {
+              // fp16 activations: a k-block is two 128-byte swizzle spans of 64 values
+              tma_load_2d(sA8 + a * C::kASlot + j * C::kA8Bytes, &tmap_a, &afull[a], (kb + j) * 128, m0);
+              tma_load_2d(sA8 + a * C::kASlot + j * C::kA8Bytes + BN * 128, &tmap_a, &afull[a], (kb + j) * 128 + 64,
+                          m0);
+            } else {
+              tma_load_2d(sA8 + a * C::kASlot + j * C::kA8Bytes, &tmap_a, &afull[a], (kb + j) * 128, m0);
+            }
+          }
         }
       }
       const int first = c - NS > 0 ? c - NS : 0;
@@ -831,7 +944,8 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     __syncwarp();
   } else if (warp >= 1 && warp < 1 + NMMA) {
     // ----------------------------------------------------------- MMA issuers
-    // Issuer mi takes chunks c = mi (mod NMMA). Both issuers accumulate into
+    // Issuer mi takes chunks c = mi (mod NMMA) and with them whole ring slots
+    // (depths are multiples of NMMA). Both issuers accumulate into
     // the segment's one accumulator buffer b: every MMA accumulates (the
     // epilogue hands the buffer back zeroed), so the order in which the tensor
     // pipe runs the two threads' MMAs does not change the exact int32 sums.
@@ -839,7 +953,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     // MMAs of its own in that segment.
     if (lane == 0) {
       const int mi = warp - 1;
-      constexpr uint32_t idesc = idesc_i8(128, BN);
+      constexpr uint32_t idesc = C::kLut ? idesc_f16(128, BN) : idesc_i8(128, BN);
       int c = 0, seg_i = 0;
       bool ok = true;
       while (ok && sch.next(sg)) {
@@ -861,10 +975,16 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
           const uint32_t b_addr = smem_u32(sA8 + a * C::kASlot);
           for (int j = 0; j < cnt; ++j) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              mma_i8_ts(d_tmem, a_tmem + j * 32 + kk * 8,
-                        smem_desc_k128_sw128(b_addr + j * C::kA8Bytes + kk * 32), idesc,
-                        1u);
+            for (int kk = 0; kk < C::kMmaPerKb; ++kk) {
+              // each MMA consumes 32 bytes of every row of both operands (8
+              // TMEM columns of A); fp16 activations span two swizzle atoms
+              const uint32_t b_off = C::kLut ? (kk >> 2) * (BN * 128) + (kk & 3) * 32 : kk * 32;
+              const uint64_t bdesc = smem_desc_k128_sw128(b_addr + j * C::kA8Bytes + b_off);
+              if constexpr (C::kLut) {
+                mma_f16_ts(d_tmem, a_tmem + j * C::kKbCols + kk * 8, bdesc, idesc, 1u);
+              } else {
+                mma_i8_ts(d_tmem, a_tmem + j * C::kKbCols + kk * 8, bdesc, idesc, 1u);
+              }
             }
           }
           mma_commit(&aempty[a]);
@@ -897,10 +1017,9 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
         if (c % DQ != g) continue;
         const int cnt = min(KS, sg.kb1 - kb);
         const int w = c % NS, t = c % NT;
-        // TMEM slot first: once the MMAs of chunk c - NT are done, every
-        // chunk up to c - NT has been loaded, so (NS >= NT) the weight slot's
-        // barrier is at most one phase behind and its parity wait cannot
-        // alias an older phase, however far the other groups lag.
+        // TMEM slot first, then the weight slot: both slots serve this group
+        // alone (ring depths are multiples of DQ), so each parity wait is for
+        // the phase after the one this group last waited on.
         if (!__all_sync(0xffffffffu, mbar_wait(&tempty[t], ((c / NT) & 1) ^ 1, abort_flag, err, kErrDequant) &&
                                          mbar_wait(&wfull[w], (c / NS) & 1, abort_flag, err, kErrDequant))) {
           ok = false;
@@ -909,15 +1028,24 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
         tc_fence_after();
         for (int j = 0; j < cnt; ++j) {
           uint32_t out[32];
-          dequant_tile_regs(sW + w * C::kWSlot + j * kTileBytes, r, out);
-          if (C::kPipelinedStores && j == 0 && prev_t >= 0) {
-            // the previous chunk's stores are done once these ones may start
-            tmem_wait_st();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&tfull[prev_t]);
+          if constexpr (C::kLut) {
+            const uint32_t* lut = reinterpret_cast<const uint32_t*>(smem + C::kOffLut);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              lut_dequant_half(sW + w * C::kWSlot + j * C::kTileB, r, h, lut, lane, out);
+              tmem_st_32(tmem + C::kTmemA + t * C::kTSlotCols + j * C::kKbCols + h * 32 + lane_base, out);
+            }
+          } else {
+            dequant_tile_regs(sW + w * C::kWSlot + j * C::kTileB, r, out);
+            if (C::kPipelinedStores && j == 0 && prev_t >= 0) {
+              // the previous chunk's stores are done once these ones may start
+              tmem_wait_st();
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&tfull[prev_t]);
+            }
+            tmem_st_32(tmem + C::kTmemA + t * C::kTSlotCols + j * C::kKbCols + lane_base, out);
           }
-          tmem_st_32(tmem + C::kTmemA + t * C::kTSlotCols + j * 32 + lane_base, out);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&wempty[w]);
@@ -966,7 +1094,7 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
           break;
         }
       }
-      if (!epilogue_segment<BN>(args, sg, true, &accfull[b], (seg_i / NACC) & 1, &accempty[b],
+      if (!epilogue_segment<BN, C::kLut>(args, sg, true, &accfull[b], (seg_i / NACC) & 1, &accempty[b],
                                 tmem + b * BN + lane_base, BN, used, quarter, lane, rows, ystage,
                                 abort_flag, epi_fail, last_flag, err))
         break;

@@ -90,4 +90,80 @@ __global__ void pack_meta_kernel(const uint8_t* __restrict__ z, const uint8_t* _
   }
 }
 
+// Lookup-table weight blob (weight-only GEMM, "Fast Matrix Multiplications
+// for Lookup Table-Quantized LLMs", abstract: offline restructuring of the
+// quantized weights). 64-byte header (u32 magic 'W4LT', u32 version 1,
+// i64 N, i64 K, i32 group, u32 tile bytes 8448, u64 byte offset of the
+// table), then (N/128) x (K/128) tiles of 8448 bytes, then the 16 fp16 table
+// entries padded to 64 bytes. Tile (nt, kt) = 8192 index bytes + 128 fp16
+// row scales of group kt: byte j of row r's 64 bytes holds the indices of
+// in-tile k = 2j (bits 0-3) and k = 2j+1 (bits 4-7), so one pair-table
+// lookup per byte yields two consecutive k; 16-byte vector c of the row is
+// at (c * 128 + r) * 16 (a warp reads 512 contiguous bytes).
+constexpr uint32_t kLutMagic = 0x544C3457u;  // "W4LT"
+constexpr int kLutTileBytesPack = kTileCodeBytes + 2 * kTileN;  // 8448
+
+// One thread per (row n, 32-k chunk): 32 indices in, one 16-byte vector out.
+__global__ void lut_pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K,
+                                      uint8_t* __restrict__ tiles) {
+  const int64_t KC = K >> 5;
+  const int64_t total = N * KC;
+  const int64_t KT = K >> 7;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / KC;
+    const int64_t kc = i - n * KC;
+    const uint4* src = reinterpret_cast<const uint4*>(q + n * K + kc * 32);
+    const uint4 a = src[0], b = src[1];
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};  // 4 indices per word, k ascending
+    uint32_t out[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      // 8 indices (k = 8jj .. 8jj+7 of the chunk) -> 4 bytes, pairs (2b, 2b+1)
+      const uint32_t lo = in[2 * jj], hi = in[2 * jj + 1];
+      const uint32_t e = __byte_perm(lo, hi, 0x6420) & 0x0F0F0F0Fu;  // indices k = 0, 2, 4, 6
+      const uint32_t o = __byte_perm(lo, hi, 0x7531) & 0x0F0F0F0Fu;  // indices k = 1, 3, 5, 7
+      out[jj] = e | (o << 4);
+    }
+    const int64_t nt = n >> 7, r = n & 127;
+    const int64_t kt = kc >> 2, c = kc & 3;
+    uint8_t* tile = tiles + (nt * KT + kt) * kLutTileBytesPack;
+    *reinterpret_cast<uint4*>(tile + (c * kTileN + r) * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+}
+
+// Row scales into their tiles, the table after the tiles, and the header.
+__global__ void lut_pack_meta_kernel(const __half* __restrict__ s, const __half* __restrict__ table, int64_t N,
+                                     int64_t K, uint8_t* __restrict__ blob, int64_t table_offset) {
+  const int64_t G = K >> 7;
+  const int64_t total = N * G;
+  uint8_t* tiles = blob + kHeaderBytes;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / G, g = i - n * G;
+    *reinterpret_cast<__half*>(tiles + ((n >> 7) * G + g) * kLutTileBytesPack + kTileCodeBytes + 2 * (n & 127)) = s[i];
+  }
+  if (blockIdx.x == 0 && threadIdx.x < 32) {
+    __half* t = reinterpret_cast<__half*>(blob + table_offset);
+    t[threadIdx.x] = threadIdx.x < 16 ? table[threadIdx.x] : __ushort_as_half(0);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < kHeaderBytes / 4) {
+    uint32_t w = 0;
+    switch (threadIdx.x) {
+      case 0: w = kLutMagic; break;
+      case 1: w = kLayoutVersion; break;
+      case 2: w = static_cast<uint32_t>(N); break;
+      case 3: w = static_cast<uint32_t>(static_cast<uint64_t>(N) >> 32); break;
+      case 4: w = static_cast<uint32_t>(K); break;
+      case 5: w = static_cast<uint32_t>(static_cast<uint64_t>(K) >> 32); break;
+      case 6: w = 128u; break;
+      case 7: w = static_cast<uint32_t>(kLutTileBytesPack); break;
+      case 8: w = static_cast<uint32_t>(table_offset); break;
+      case 9: w = static_cast<uint32_t>(static_cast<uint64_t>(table_offset) >> 32); break;
+      default: w = 0; break;
+    }
+    reinterpret_cast<uint32_t*>(blob)[threadIdx.x] = w;
+  }
+}
+
 }  // namespace w4a8

@@ -170,6 +170,16 @@ __device__ __forceinline__ void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 x fp16 -> fp32, one CTA.
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive (once) on an mbarrier when all previously issued tcgen05 ops of this
 // thread have completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -230,6 +240,16 @@ __device__ __forceinline__ uint64_t smem_desc_k128_sw128(uint32_t saddr) {
   return d;
 }
 
+// Instruction descriptor: kind::f16, D = f32, A = B = f16, both K-major,
+// shape M x N.
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n) {
+  return (1u << 4)                                     // D format: f32
+         | (0u << 7)                                   // A: f16
+         | (0u << 10)                                  // B: f16
+         | (static_cast<uint32_t>(n >> 3) << 17)       // N / 8
+         | (static_cast<uint32_t>(m >> 4) << 24);      // M / 16
+}
+
 // Instruction descriptor: kind::i8, D = s32, A = u8 (the biased weights),
 // B = s8 (the activations), both K-major, shape M x N (M = 128 here).
 __host__ __device__ constexpr uint32_t idesc_i8(int m, int n) {
@@ -246,6 +266,9 @@ __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
 
 __device__ __forceinline__ void red_add_s32(int32_t* p, int32_t v) {
   asm volatile("red.relaxed.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.relaxed.gpu.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
 }
 __device__ __forceinline__ void fence_acq_rel_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 __device__ __forceinline__ int atom_add_relaxed_gpu(int* p, int v) {

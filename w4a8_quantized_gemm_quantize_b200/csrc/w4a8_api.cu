@@ -105,6 +105,9 @@ w4a8_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 int64_t packed_s1_offset(int64_t N, int64_t K) { return kHeaderBytes + (N / kTileN) * (K / kTileK) * kTileBytes; }
+int64_t lut_table_offset(int64_t N, int64_t K) {
+  return kHeaderBytes + (N / kTileN) * (K / kTileK) * kLutTileBytesPack;
+}
 
 // ------------------------------------------------------------------ GEMM
 // Resident CTAs per SM of a configuration (shared memory, threads and tensor
@@ -172,6 +175,19 @@ w4a8_status_t launch_gemm_cfg(const void* act, int64_t M, int64_t K, GemmArgs ar
                               cudaStream_t stream) {
   if (args.split > C::kMaxSplit) return W4A8_ERR_INVALID_ARG;
   CUtensorMap map;
+  if constexpr (C::kLut) {
+    // fp16 activations [M, K]: 64-value (128-byte) spans, 128-byte swizzle
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(2 * K)};
+    const cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(C::BN)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void*>(act), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return W4A8_ERR_CUDA;
+    return launch_pdl(w4a8_gemm_kernel<C>, dim3(grid), dim3(C::kThreads), C::kSmemBytes, stream, args.split, map,
+                      args);
+  }
   const int64_t row_bytes = args.a4 ? K / 2 : K;
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(M)};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
@@ -188,9 +204,13 @@ w4a8_status_t launch_gemm_cfg(const void* act, int64_t M, int64_t K, GemmArgs ar
 // Tile configurations: tokens per tile, k-blocks per chunk, weight and
 // activation ring slots, TMEM ring slots, dequantizer groups, accumulator
 // buffers, MMA issuers.
-using Cfg16 = GemmCfg<16, 4, 5, 3, 2, 2, 2>;
-using Cfg32 = GemmCfg<32, 4, 4, 3, 2, 2, 2>;
+using Cfg16 = GemmCfg<16, 3, 4, 4, 2, 2, 2>;
+using Cfg32 = GemmCfg<32, 3, 4, 4, 2, 2, 2>;
 using Cfg64 = GemmCfg<64, 2, 6, 6, 2, 2, 2>;
+// lookup-table weights against fp16 activations (decode tile sizes; larger M
+// uses several 32-token tiles)
+using CfgL16 = GemmCfg<16, 2, 6, 2, 2, 2, 2, true>;
+using CfgL32 = GemmCfg<32, 2, 4, 2, 2, 2, 2, true>;
 using Cfg128 = GemmCfg<128, 4, 2, 2, 1, 2, 2>;
 
 size_t ws_counter_bytes(int64_t M, int64_t N) {
@@ -256,18 +276,19 @@ w4a8_status_t check_quantize_args(const void* A, int64_t M, int64_t K, const voi
 // [M, K / 2] (W4A4).
 w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
                         int64_t N, int64_t K, void* Y, int32_t* acc, void* ws, size_t ws_bytes,
-                        const w4a8_gemm_opts_t* opts, cudaStream_t stream, int a4 = 0) {
+                        const w4a8_gemm_opts_t* opts, cudaStream_t stream, int a4 = 0, int lut = 0) {
   w4a8_gemm_opts_t o = {0, 0, 0, 0};
   if (opts != nullptr) o = *opts;
   if (o.reserved != 0 || o.schedule < 0 || o.schedule > 3 || o.max_ctas < 0) return W4A8_ERR_INVALID_ARG;
   if (!(o.block_m == 0 || o.block_m == 16 || o.block_m == 32 || o.block_m == 64 || o.block_m == 128))
     return W4A8_ERR_INVALID_ARG;
+  if (lut && o.block_m > 32) return W4A8_ERR_INVALID_ARG;
   if (M < 0 || N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
   if (K == 0 || K % kTileK != 0 || K > kMaxK || N % kTileN != 0) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M > INT32_MAX || N > INT32_MAX || (N > 0 && M > (int64_t(1) << 62) / N)) return W4A8_ERR_UNSUPPORTED_SHAPE;
   if (M == 0 || N == 0) return W4A8_OK;
   if ((Y == nullptr) == (acc == nullptr)) return W4A8_ERR_INVALID_ARG;
-  if (A8 == nullptr || packed == nullptr || rowsum == nullptr || (acc == nullptr && sA == nullptr))
+  if (A8 == nullptr || packed == nullptr || (!lut && (rowsum == nullptr || (acc == nullptr && sA == nullptr))))
     return W4A8_ERR_INVALID_ARG;
   if (!aligned(A8, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(acc, 16) || !aligned(sA, 2) ||
       !aligned(rowsum, 4) || !aligned(ws, 256))
@@ -277,7 +298,7 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   if (st != W4A8_OK) return st;
 
   int bn = o.block_m;
-  if (bn == 0) bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+  if (bn == 0) bn = M <= 16 ? 16 : M <= 32 || lut ? 32 : M <= 64 ? 64 : 128;
   const int n_tiles = static_cast<int>(N / kTileN);
   const int m_tiles = static_cast<int>((M + bn - 1) / bn);
   const int64_t num_tiles64 = static_cast<int64_t>(n_tiles) * m_tiles;
@@ -287,11 +308,15 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   int dev_id = 0;
   cudaGetDevice(&dev_id);
   int per_sm = 1;
-  switch (bn) {
-    case 16: st = ctas_per_sm<Cfg16>(dev_id, &per_sm); break;
-    case 32: st = ctas_per_sm<Cfg32>(dev_id, &per_sm); break;
-    case 64: st = ctas_per_sm<Cfg64>(dev_id, &per_sm); break;
-    default: st = ctas_per_sm<Cfg128>(dev_id, &per_sm); break;
+  if (lut) {
+    st = bn == 16 ? ctas_per_sm<CfgL16>(dev_id, &per_sm) : ctas_per_sm<CfgL32>(dev_id, &per_sm);
+  } else {
+    switch (bn) {
+      case 16: st = ctas_per_sm<Cfg16>(dev_id, &per_sm); break;
+      case 32: st = ctas_per_sm<Cfg32>(dev_id, &per_sm); break;
+      case 64: st = ctas_per_sm<Cfg64>(dev_id, &per_sm); break;
+      default: st = ctas_per_sm<Cfg128>(dev_id, &per_sm); break;
+    }
   }
   if (st != W4A8_OK) return st;
   int max_ctas = dev->sms * per_sm;
@@ -305,7 +330,11 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
     for (int S = 4; S >= 2 && split == 1; --S) {
       if (S > KB) continue;
       int nclu = 0;
-      st = bn == 16 ? max_clusters<Cfg16>(dev_id, S, &nclu) : max_clusters<Cfg32>(dev_id, S, &nclu);
+      if (lut) {
+        st = bn == 16 ? max_clusters<CfgL16>(dev_id, S, &nclu) : max_clusters<CfgL32>(dev_id, S, &nclu);
+      } else {
+        st = bn == 16 ? max_clusters<Cfg16>(dev_id, S, &nclu) : max_clusters<Cfg32>(dev_id, S, &nclu);
+      }
       if (st != W4A8_OK) return st;
       if (num_tiles <= nclu && num_tiles * S <= max_ctas) split = S;
     }
@@ -360,7 +389,9 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
 
   GemmArgs a;
   a.tiles = static_cast<const uint8_t*>(packed) + kHeaderBytes;
-  a.s1 = reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + packed_s1_offset(N, K));
+  a.s1 = lut ? nullptr : reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + packed_s1_offset(N, K));
+  a.lut_table = lut ? reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + lut_table_offset(N, K))
+                    : nullptr;
   a.sA = static_cast<const __half*>(sA);
   a.rowsum = rowsum;
   a.Y = static_cast<__half*>(Y);
@@ -376,6 +407,12 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   a.sk_tiles = sk_tiles;
   a.split = split;
   a.a4 = a4;
+  if (lut) {
+    a.sA = nullptr;
+    a.rowsum = nullptr;
+    return bn == 16 ? launch_gemm_cfg<CfgL16>(A8, M, K, a, grid, stream)
+                    : launch_gemm_cfg<CfgL32>(A8, M, K, a, grid, stream);
+  }
   switch (bn) {
     case 16: return launch_gemm_cfg<Cfg16>(A8, M, K, a, grid, stream);
     case 32: return launch_gemm_cfg<Cfg32>(A8, M, K, a, grid, stream);
@@ -525,6 +562,46 @@ w4a8_status_t w4a4_gemm_ex(const uint8_t* A4, const void* sA, const int32_t* row
                            const w4a8_gemm_opts_t* opts, w4a8_stream_t stream) {
   return gemm_impl(A4, sA, rowsum, packed, M, N, K, Y, acc, workspace, workspace_bytes, opts,
                    reinterpret_cast<cudaStream_t>(stream), 1);
+}
+
+size_t w4lut_packed_bytes(int64_t N, int64_t K, int32_t group) {
+  if (group != 128 || N <= 0 || K <= 0 || N % 128 != 0 || K % 128 != 0 || K > kMaxK) return 0;
+  return static_cast<size_t>(lut_table_offset(N, K) + 64);
+}
+
+w4a8_status_t w4lut_pack_weights(const uint8_t* q, const void* s, const void* table, int64_t N, int64_t K,
+                                 int32_t group, void* packed, size_t packed_bytes, w4a8_stream_t stream) {
+  if (N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if (group != 128 || N == 0 || K == 0 || N % 128 != 0 || K % 128 != 0 || K > kMaxK)
+    return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (q == nullptr || s == nullptr || table == nullptr || packed == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(s, 2) || !aligned(table, 2) || !aligned(packed, 16)) return W4A8_ERR_MISALIGNED;
+  if (packed_bytes < w4lut_packed_bytes(N, K, group)) return W4A8_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* blob = static_cast<uint8_t*>(packed);
+  const int64_t chunks = N * (K / 32);
+  const int64_t blocks1 = (chunks + 255) / 256;
+  lut_pack_codes_kernel<<<static_cast<int>(blocks1 < 65535 * 16 ? blocks1 : 65535 * 16), 256, 0, st>>>(
+      q, N, K, blob + kHeaderBytes);
+  if (cudaPeekAtLastError() != cudaSuccess) return launch_status();
+  const int64_t metas = N * (K / 128);
+  const int64_t blocks2 = (metas + 255) / 256;
+  lut_pack_meta_kernel<<<static_cast<int>(blocks2 < 65535 ? blocks2 : 65535), 256, 0, st>>>(
+      static_cast<const __half*>(s), static_cast<const __half*>(table), N, K, blob, lut_table_offset(N, K));
+  return launch_status();
+}
+
+w4a8_status_t w4lut_gemm(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
+                         void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
+  return gemm_impl(A, nullptr, nullptr, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream), 0, 1);
+}
+
+w4a8_status_t w4lut_gemm_ex(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y, float* acc,
+                            void* workspace, size_t workspace_bytes, const w4a8_gemm_opts_t* opts,
+                            w4a8_stream_t stream) {
+  return gemm_impl(A, nullptr, nullptr, packed, M, N, K, Y, reinterpret_cast<int32_t*>(acc), workspace,
+                   workspace_bytes, opts, reinterpret_cast<cudaStream_t>(stream), 0, 1);
 }
 
 w4a8_status_t w4a8_get_device_error(w4a8_stream_t stream, int32_t* code) {
