@@ -202,7 +202,6 @@ struct GemmCfg {
   // chunk c + DQ, which must not need a slot that chunk c + 1 still holds);
   // otherwise it completes them within the chunk.
   static constexpr bool kPipelinedStores = NT >= 2 * DQ && NT >= DQ + 2;
-  static_assert(!(kLut && kPipelinedStores), "the lookup-table dequantizer completes its stores per chunk");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "MMA N for M = 128");
   // Cluster split-K (small BN only): up to kMaxSplit CTAs per tile. The
   // owner of TMEM lane quarter q is cluster rank q % split; it receives the
@@ -1033,6 +1032,12 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               lut_dequant_half(sW + w * C::kWSlot + j * C::kTileB, r, h, lut, lane, out);
+              if (C::kPipelinedStores && j == 0 && h == 0 && prev_t >= 0) {
+                tmem_wait_st();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tfull[prev_t]);
+              }
               tmem_st_32(tmem + C::kTmemA + t * C::kTSlotCols + j * C::kKbCols + h * 32 + lane_base, out);
             }
           } else {

@@ -208,9 +208,10 @@ using Cfg16 = GemmCfg<16, 3, 4, 4, 2, 2, 2>;
 using Cfg32 = GemmCfg<32, 3, 4, 4, 2, 2, 2>;
 using Cfg64 = GemmCfg<64, 2, 6, 6, 2, 2, 2>;
 // lookup-table weights against fp16 activations (decode tile sizes; larger M
-// uses several 32-token tiles)
-using CfgL16 = GemmCfg<16, 2, 6, 2, 2, 2, 2, true>;
-using CfgL32 = GemmCfg<32, 2, 4, 2, 2, 2, 2, true>;
+// uses several 32-token tiles): one k-block per chunk and a third
+// dequantizer group (the table lookups, not the weight bytes, limit it)
+using CfgL16 = GemmCfg<16, 1, 12, 6, 3, 2, 2, true>;
+using CfgL32 = GemmCfg<32, 1, 6, 6, 3, 2, 2, true>;
 using Cfg128 = GemmCfg<128, 4, 2, 2, 1, 2, 2>;
 
 size_t ws_counter_bytes(int64_t M, int64_t N) {
