@@ -134,3 +134,57 @@ def lut_codes(N: int, K: int, seed: int, group: int = GROUP):
     q = rng.integers(0, 16, size=(N, K), dtype=np.uint8)
     s = rng.uniform(0.005, 0.05, size=(N, K // group)).astype(np.float16)
     return q, s
+
+
+# ------------------------------------------------ 4-bit KV-cache attention
+# Attention geometry of the workloads' models: (query heads, kv heads, head dim).
+LLAMA3_8B_ATTN = (32, 8, 128)
+QWEN15_72B_ATTN = (64, 64, 128)
+
+
+@dataclass(frozen=True)
+class KvWorkload:
+    name: str
+    batch: int
+    max_len: int      # cache capacity per sequence (tokens)
+    heads: tuple      # (Hq, Hkv, D)
+    ragged: bool      # lengths drawn in [max_len / 2, max_len], else all max_len
+
+
+KV_WORKLOADS = {
+    "kv-tiny": KvWorkload("kv-tiny", 3, 300, (4, 2, 128), True),
+    "kv-decode": KvWorkload("kv-decode", 16, 4096, LLAMA3_8B_ATTN, True),
+    "kv-long": KvWorkload("kv-long", 4, 32768, LLAMA3_8B_ATTN, False),
+    "kv-qwen72b": KvWorkload("kv-qwen72b", 8, 4096, QWEN15_72B_ATTN, True),
+}
+
+
+def kv_vectors(B: int, H: int, L: int, D: int, seed: int, outlier_scale: float = 10.0) -> np.ndarray:
+    """fp16 [B, H, L, D]: N(0, 1), with round(0.04 D) channels per head
+    scaled by `outlier_scale` (the same channels for every token of a head,
+    as keys have; pass 1.0 for values)."""
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((B, H, L, D), dtype=np.float32)
+    n_out = int(np.floor(0.04 * D + 0.5))
+    if outlier_scale != 1.0 and n_out > 0:
+        for h in range(H):
+            ch = rng.choice(D, size=n_out, replace=False)
+            x[:, h, :, ch] *= outlier_scale
+    return x.astype(np.float16)
+
+
+def kv_queries(B: int, Hq: int, D: int, seed: int) -> np.ndarray:
+    """fp16 [B, Hq, D] decode queries, N(0, 1)."""
+    rng = np.random.default_rng(seed)
+    return rng.standard_normal((B, Hq, D), dtype=np.float32).astype(np.float16)
+
+
+def kv_seq_lens(wl: KvWorkload, seed: int) -> np.ndarray:
+    """int32 [B] cache lengths of a workload (ragged: uniform on
+    [max_len / 2, max_len], the first sequence always full)."""
+    if not wl.ragged:
+        return np.full(wl.batch, wl.max_len, dtype=np.int32)
+    rng = np.random.default_rng(seed)
+    lens = rng.integers(wl.max_len // 2, wl.max_len + 1, size=wl.batch).astype(np.int32)
+    lens[0] = wl.max_len
+    return lens
