@@ -131,7 +131,8 @@ def attention_error_bound(q, kc, kp, vc, vp, seq_lens, scale) -> np.ndarray:
 
     * score s_j: the D products q[d] K^[j,d] and their sum carry at most
       gamma_{D+1} sum_d |q K^| (gamma_n = n u / (1 - n u)), times `scale`,
-      plus u |s_j| for the scale multiply: delta_j; delta = max_j delta_j.
+      plus 2 u |s_j| for two rounded multiplies (the vector's scale applied
+      to the sum of q (code - z), and `scale`): delta_j; delta = max_j delta_j.
     * weight p_j = exp(s_j - max): the computed max is within delta of the
       exact one; the argument carries 2 delta + 2 u delta + 3 u |s_j - m|
       (subtraction, a change of exponent base, a rescale of a partial result
@@ -163,7 +164,7 @@ def attention_error_bound(q, kc, kp, vc, vp, seq_lens, scale) -> np.ndarray:
             qd = q[b, h].astype(np.float64)
             s = sc * (K @ qd)
             m = s.max()
-            delta = np.max(abs(sc) * gD * (np.abs(K) @ np.abs(qd)) + u * np.abs(s))
+            delta = np.max(abs(sc) * gD * (np.abs(K) @ np.abs(qd)) + 2 * u * np.abs(s))
             p = np.exp(s - m)
             o = (p @ V) / p.sum()
             R = 2 * delta * (1 + u) + 6 * u * np.abs(s - m) + 10 * u
