@@ -73,6 +73,7 @@ typedef enum {
 #define W4A8_DEVERR_EPILOGUE_WAIT 4
 #define W4A8_DEVERR_DRAIN_WAIT 5
 #define W4A8_DEVERR_SELFTEST_WAIT 6
+#define W4A8_DEVERR_KV_RANGE 7 /* a KV-cache length or position outside [0, Lmax] (clamped or skipped) */
 
 /* Human-readable name of a status code (static string, never NULL). */
 W4A8_API const char* w4a8_status_string(int status);
@@ -327,6 +328,68 @@ W4A8_API w4a8_status_t w4lut_gemm(const void* A, const void* packed, int64_t M, 
 W4A8_API w4a8_status_t w4lut_gemm_ex(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
                                      float* acc, void* workspace, size_t workspace_bytes,
                                      const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
+
+/*
+ * 4-bit KV cache and decode attention over it (the KV4 of W4A8KV4,
+ * "QServe/QoQ" abstract on the lmdeploy issue "[Feature] Support W4A8KV4
+ * Quantization(QServe/QoQ)", Motivation: 4-bit KV cache, memory-bound fused
+ * attention; "PrefixQuant ...", Key Findings: W4A4KV4). The pages fix no
+ * format or arithmetic; this library's:
+ *
+ * Cached vector (one token of one kv head, D = 128 values): on the range
+ * widened to include zero, lo = min(min x, 0), hi = max(max x, 0),
+ *   s = fp16_rn((hi - lo) / 15),  z = clamp(rint(-lo / s), 0, 15),
+ *   code = clamp(rint(x / s) + z, 0, 15)
+ * (fp32, IEEE divides, ties to even; s == 0 gives z = 0 and zero codes);
+ * dequantized value (code - z) * s. Stored as 64 code bytes (element 2i in
+ * bits 0-3 of byte i, 2i+1 in bits 4-7) and one 32-bit parameter word: fp16 s
+ * in bits 0-15, fp16 z in bits 16-31. A static per-tensor scheme is the same
+ * format with one (s, z) for every vector.
+ *
+ * Cache layout: codes uint8 [B, Hkv, Lmax, 64], parameter words uint32
+ * [B, Hkv, Lmax]; sequence b holds its tokens at positions 0 .. L_b - 1.
+ *
+ * Decode attention, one query token per sequence: query head h reads kv head
+ * h / (Hq / Hkv);
+ *   s_j = scale * (s_j^K * sum_d q[d] (code^K_jd - z^K_j)),  j < L_b
+ *   Y[b, h] = fp16_rn(sum_j softmax(s)_j (code^V_j - z^V_j) s^V_j)
+ * in fp32 (so within the fp32 evaluation bound of the exact result plus half
+ * an fp16 ulp); L_b == 0 gives Y = 0.
+ */
+
+/* Quantizes n contiguous fp16 vectors X [n, 128] (16-byte aligned) into codes
+ * [n, 64] (16-byte aligned) and parameter words [n] (4-byte aligned). D must
+ * be 128. */
+W4A8_API w4a8_status_t w4kv_quantize(const void* X, int64_t n, int32_t D, uint8_t* codes, uint32_t* params,
+                                     w4a8_stream_t stream);
+
+/* Appends one token per (sequence, kv head): K_new and V_new fp16 [B, Hkv,
+ * 128] are quantized into the caches at position positions[b] (int32 [B],
+ * device memory). A position outside [0, Lmax) is skipped and recorded as
+ * W4A8_DEVERR_KV_RANGE in the device error word. */
+W4A8_API w4a8_status_t w4kv_append(const void* K_new, const void* V_new, const int32_t* positions, int64_t B,
+                                   int64_t Hkv, int64_t Lmax, int32_t D, uint8_t* k_codes, uint32_t* k_params,
+                                   uint8_t* v_codes, uint32_t* v_params, w4a8_stream_t stream);
+
+/* Workspace bytes of w4kv_attention_decode (0 if the shape is unsupported). */
+W4A8_API size_t w4kv_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lmax, int32_t D);
+
+/*
+ * Y fp16 [B, Hq, 128] (16-byte aligned) = decode attention of q fp16 [B, Hq,
+ * 128] (16-byte aligned) over the caches (codes 16-byte, parameter words
+ * 4-byte aligned) with lengths seq_lens (int32 [B], device memory; a length
+ * outside [0, Lmax] is clamped and recorded as W4A8_DEVERR_KV_RANGE).
+ * Limits: D == 128, Hkv >= 1, Hq % Hkv == 0, Hq <= 65536, 1 <= Lmax <= 2^24,
+ * B <= 65535. workspace: 256-byte aligned, at least
+ * w4kv_attention_workspace_bytes(...) bytes, zero-filled before its first
+ * use; the call leaves its first part (the per-head-group tickets) zero again.
+ * Calls that share a workspace must not overlap on the GPU.
+ */
+W4A8_API w4a8_status_t w4kv_attention_decode(const void* q, const uint8_t* k_codes, const uint32_t* k_params,
+                                             const uint8_t* v_codes, const uint32_t* v_params,
+                                             const int32_t* seq_lens, int64_t B, int64_t Hq, int64_t Hkv,
+                                             int64_t Lmax, int32_t D, float scale, void* out, void* workspace,
+                                             size_t workspace_bytes, w4a8_stream_t stream);
 
 /*
  * Allocation-free GEMM: the same computation and results as w4a8_gemm, for

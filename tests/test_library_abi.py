@@ -24,7 +24,7 @@ def L():
 
 def declared_functions():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4(?:a[48]|lut)_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4(?:a[48]|lut|kv)_\w+)\s*\(", src)))
 
 
 def test_header_declares_entry_points():
@@ -168,3 +168,28 @@ def test_lut_validation(L):
     assert g(FAKE, FAKE, 0, 128, 256, FAKE, None, 0, None) == 0           # M == 0: no-op
     bad = w4a8.GemmOpts(0, 64, 0, 0)                                       # 64-token tiles: not for this GEMM
     assert L.w4lut_gemm_ex(FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
+
+
+def test_kv4_validation(L):
+    q = L.w4kv_quantize
+    assert q(FAKE, 4, 64, FAKE, FAKE, None) == 2                           # D != 128
+    assert q(FAKE, -1, 128, FAKE, FAKE, None) == 1
+    assert q(None, 4, 128, FAKE, FAKE, None) == 1
+    assert q(FAKE_ODD, 4, 128, FAKE, FAKE, None) == 3
+    assert q(None, 0, 128, None, None, None) == 0                         # n == 0: no-op
+    ws = L.w4kv_attention_workspace_bytes
+    assert ws(2, 32, 8, 4096, 128) == 256 + 2 * 32 * 16 * 130 * 4         # tickets, then partials
+    assert ws(2, 6, 4, 4096, 128) == 0                                    # Hq % Hkv
+    assert ws(2, 32, 8, 4096, 64) == 0                                    # D
+    a = L.w4kv_attention_decode
+    args = [FAKE, FAKE, FAKE, FAKE, FAKE, FAKE]
+    assert a(*args, 2, 32, 8, 0, 128, 1.0, FAKE, FAKE, 1 << 30, None) == 2   # Lmax == 0
+    assert a(*args, 2, 32, 8, 1024, 128, 1.0, FAKE, FAKE, 16, None) == 4     # workspace too small
+    assert a(*args, 2, 32, 8, 1024, 128, 1.0, FAKE, None, 1 << 30, None) == 4
+    assert a(*args, 2, 32, 8, 1024, 128, 1.0, None, FAKE, 1 << 30, None) == 1
+    assert a(FAKE_ODD, *args[1:], 2, 32, 8, 1024, 128, 1.0, FAKE, FAKE, 1 << 30, None) == 3
+    assert a(*args, 0, 32, 8, 1024, 128, 1.0, None, None, 0, None) == 0     # B == 0: no-op
+    ap = L.w4kv_append
+    assert ap(FAKE, FAKE, FAKE, 2, 8, 1024, 64, FAKE, FAKE, FAKE, FAKE, None) == 2
+    assert ap(FAKE, FAKE, None, 2, 8, 1024, 128, FAKE, FAKE, FAKE, FAKE, None) == 1
+    assert ap(FAKE, FAKE, FAKE, 0, 8, 1024, 128, FAKE, FAKE, FAKE, FAKE, None) == 0

@@ -21,7 +21,7 @@ __all__ = [
     "gemm_debug_acc", "gemm_ex", "gemm_noalloc", "get_device_error", "clear_device_error",
     "selftest_bounded_wait", "quantize_act_static", "w4a4_quantize_act", "w4a4_quantize_act_static",
     "w4a4_gemm", "w4a4_gemm_ex", "w4a4_workspace_bytes", "lut_packed_bytes", "lut_pack_weights", "lut_gemm",
-    "lut_gemm_ex",
+    "lut_gemm_ex", "kv4_quantize", "kv4_append", "kv4_workspace_bytes", "kv4_attention_decode",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -34,6 +34,7 @@ EXPORTED_SYMBOLS = (
     "w4a8_gemm_noalloc", "w4a8_selftest_bounded_wait", "w4a8_quantize_act_static",
     "w4a4_quantize_act", "w4a4_quantize_act_static", "w4a4_gemm", "w4a4_gemm_ex", "w4a4_gemm_workspace_bytes",
     "w4lut_packed_bytes", "w4lut_pack_weights", "w4lut_gemm", "w4lut_gemm_ex",
+    "w4kv_quantize", "w4kv_append", "w4kv_attention_workspace_bytes", "w4kv_attention_decode",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
@@ -88,6 +89,11 @@ def lib() -> ctypes.CDLL:
         "w4lut_gemm_ex": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, vp, sz, ctypes.POINTER(GemmOpts), vp]),
         "w4a4_gemm_ex": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, sz,
                                         ctypes.POINTER(GemmOpts), vp]),
+        "w4kv_quantize": (ctypes.c_int, [vp, i64, i32, vp, vp, vp]),
+        "w4kv_append": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp]),
+        "w4kv_attention_workspace_bytes": (sz, [i64, i64, i64, i64, i32]),
+        "w4kv_attention_decode": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, ctypes.c_float,
+                                                 vp, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -458,3 +464,59 @@ def selftest_bounded_wait(limit_ns: int, device=None):
     """Launches the failure-path self-test (a bounded wait that must give up
     after `limit_ns`); its code shows in get_device_error()."""
     _check(lib().w4a8_selftest_bounded_wait(int(limit_ns), _stream(device)), "w4a8_selftest_bounded_wait")
+
+
+# ------------------------------------------------------- 4-bit KV cache
+KV_HEAD_DIM = 128
+
+
+def kv4_quantize(X, codes=None, params=None):
+    """fp16 vectors X [..., 128] -> (codes uint8 [..., 64], parameter words
+    int32 [...] holding the fp16 pair (s, z), s in the low half)."""
+    torch = _torch()
+    _require_cuda(X, codes, params)
+    if X.dtype != torch.float16 or X.shape[-1] != KV_HEAD_DIM or not X.is_contiguous():
+        raise W4A8Error("X must be contiguous fp16 [..., 128]")
+    lead = tuple(X.shape[:-1])
+    n = X.numel() // KV_HEAD_DIM
+    codes = codes if codes is not None else torch.empty(lead + (KV_HEAD_DIM // 2,), dtype=torch.uint8,
+                                                        device=X.device)
+    params = params if params is not None else torch.empty(lead, dtype=torch.int32, device=X.device)
+    _check(lib().w4kv_quantize(_ptr(X), n, KV_HEAD_DIM, _ptr(codes), _ptr(params), _stream(X.device)),
+           "w4kv_quantize")
+    return codes, params
+
+
+def kv4_append(K_new, V_new, positions, k_codes, k_params, v_codes, v_params):
+    """Quantizes one token per (sequence, kv head), K_new and V_new fp16
+    [B, Hkv, 128], into the caches (codes [B, Hkv, Lmax, 64], parameter
+    words [B, Hkv, Lmax]) at positions int32 [B]."""
+    _require_cuda(K_new, V_new, positions, k_codes, k_params, v_codes, v_params)
+    B, Hkv, D = K_new.shape
+    Lmax = k_codes.shape[2]
+    _check(lib().w4kv_append(_ptr(K_new), _ptr(V_new), _ptr(positions), B, Hkv, Lmax, D, _ptr(k_codes),
+                             _ptr(k_params), _ptr(v_codes), _ptr(v_params), _stream(K_new.device)), "w4kv_append")
+
+
+def kv4_workspace_bytes(B: int, Hq: int, Hkv: int, Lmax: int) -> int:
+    return int(lib().w4kv_attention_workspace_bytes(B, Hq, Hkv, Lmax, KV_HEAD_DIM))
+
+
+def kv4_attention_decode(q, k_codes, k_params, v_codes, v_params, seq_lens, scale, out=None, workspace=None):
+    """Y fp16 [B, Hq, 128] = decode attention of q fp16 [B, Hq, 128] over the
+    4-bit caches with lengths seq_lens int32 [B]; workspace zero-filled
+    uint8 (allocated here if not given)."""
+    torch = _torch()
+    _require_cuda(q, k_codes, k_params, v_codes, v_params, seq_lens, out, workspace)
+    if q.dtype != torch.float16 or q.dim() != 3 or q.shape[2] != KV_HEAD_DIM:
+        raise W4A8Error("q must be fp16 [B, Hq, 128]")
+    B, Hq, D = q.shape
+    Hkv, Lmax = k_codes.shape[1], k_codes.shape[2]
+    Y = out if out is not None else torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    if workspace is None:
+        workspace = torch.zeros(max(kv4_workspace_bytes(B, Hq, Hkv, Lmax), 1), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _check(lib().w4kv_attention_decode(_ptr(q), _ptr(k_codes), _ptr(k_params), _ptr(v_codes), _ptr(v_params),
+                                       _ptr(seq_lens), B, Hq, Hkv, Lmax, D, float(scale), _ptr(Y), _ptr(workspace),
+                                       ws_bytes, _stream(q.device)), "w4kv_attention_decode")
+    return Y

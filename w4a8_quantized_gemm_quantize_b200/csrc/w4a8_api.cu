@@ -8,6 +8,7 @@
 #include <utility>
 
 #include "gemm.cuh"
+#include "kv4_attention.cuh"
 #include "pack.cuh"
 #include "quantize_act.cuh"
 #include "quantize_weights.cuh"
@@ -422,6 +423,48 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   }
 }
 
+
+// ------------------------------------------------------------ 4-bit KV cache
+constexpr int64_t kKvMaxLen = int64_t(1) << 24;
+
+int64_t kv_splits(int64_t Lmax) { return (Lmax + kKvChunk - 1) / kKvChunk; }
+int kv_heads_per_cta(int64_t G) { return G % 4 == 0 ? 4 : G % 2 == 0 ? 2 : 1; }
+int64_t round256(int64_t x) { return (x + 255) / 256 * 256; }
+
+// Shape check of the attention call; 0 = fine.
+w4a8_status_t check_kv_shape(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lmax, int32_t D) {
+  if (B < 0 || Hq < 0 || Hkv < 0 || Lmax < 0) return W4A8_ERR_INVALID_ARG;
+  if (D != kKvD || Hkv == 0 || Lmax == 0 || Hq % Hkv != 0 || Lmax > kKvMaxLen || B > 65535 || Hq > 65536)
+    return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (Hq > 0 && Hkv * ((Hq / Hkv) / kv_heads_per_cta(Hq / Hkv)) > 65535) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  return W4A8_OK;
+}
+
+int64_t kv_ticket_bytes(int64_t B, int64_t Hq, int64_t Hkv) {
+  const int64_t G = Hq / Hkv;
+  return round256(B * Hkv * (G / kv_heads_per_cta(G)) * 4);
+}
+
+w4a8_status_t kv_quantize_launch(const void* X, int64_t n, const int32_t* pos, int64_t H, int64_t Lmax,
+                                 uint8_t* codes, uint32_t* params, cudaStream_t stream) {
+  DeviceInfo* dev = nullptr;
+  w4a8_status_t st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+  KvQuantArgs a;
+  a.x = static_cast<const __half*>(X);
+  a.n = n;
+  a.codes = codes;
+  a.params = params;
+  a.pos = pos;
+  a.H = H;
+  a.Lmax = Lmax;
+  a.err = dev->err;
+  const int64_t blocks = (n + kKvWarps - 1) / kKvWarps;
+  const int64_t cap = static_cast<int64_t>(dev->sms) * 8;
+  return launch_pdl(kv4_quantize_kernel, dim3(static_cast<unsigned>(blocks < cap ? blocks : cap)), dim3(kKvThreads),
+                    0, stream, 1, a);
+}
+
 }  // namespace w4a8
 
 using namespace w4a8;
@@ -665,6 +708,86 @@ w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const int32_t*
   // the split-k tickets and partial sums must start at zero
   if (cudaMemsetAsync(scratch, 0, need, st) != cudaSuccess) return launch_status();
   return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, nullptr, scratch, need, nullptr, st);
+}
+
+
+w4a8_status_t w4kv_quantize(const void* X, int64_t n, int32_t D, uint8_t* codes, uint32_t* params,
+                            w4a8_stream_t stream) {
+  if (n < 0) return W4A8_ERR_INVALID_ARG;
+  if (D != kKvD) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (n == 0) return W4A8_OK;
+  if (X == nullptr || codes == nullptr || params == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(params, 4)) return W4A8_ERR_MISALIGNED;
+  return kv_quantize_launch(X, n, nullptr, 1, 1, codes, params, reinterpret_cast<cudaStream_t>(stream));
+}
+
+w4a8_status_t w4kv_append(const void* K_new, const void* V_new, const int32_t* positions, int64_t B, int64_t Hkv,
+                          int64_t Lmax, int32_t D, uint8_t* k_codes, uint32_t* k_params, uint8_t* v_codes,
+                          uint32_t* v_params, w4a8_stream_t stream) {
+  if (B < 0 || Hkv < 0 || Lmax < 0) return W4A8_ERR_INVALID_ARG;
+  if (D != kKvD || Lmax > kKvMaxLen) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (B == 0 || Hkv == 0) return W4A8_OK;
+  if (Lmax == 0) return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (K_new == nullptr || V_new == nullptr || positions == nullptr || k_codes == nullptr || k_params == nullptr ||
+      v_codes == nullptr || v_params == nullptr)
+    return W4A8_ERR_INVALID_ARG;
+  if (!aligned(K_new, 16) || !aligned(V_new, 16) || !aligned(positions, 4) || !aligned(k_codes, 16) ||
+      !aligned(v_codes, 16) || !aligned(k_params, 4) || !aligned(v_params, 4))
+    return W4A8_ERR_MISALIGNED;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const w4a8_status_t s1 = kv_quantize_launch(K_new, B * Hkv, positions, Hkv, Lmax, k_codes, k_params, st);
+  if (s1 != W4A8_OK) return s1;
+  return kv_quantize_launch(V_new, B * Hkv, positions, Hkv, Lmax, v_codes, v_params, st);
+}
+
+size_t w4kv_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lmax, int32_t D) {
+  if (check_kv_shape(B, Hq, Hkv, Lmax, D) != W4A8_OK) return 0;
+  return static_cast<size_t>(kv_ticket_bytes(B, Hq, Hkv) + B * Hq * kv_splits(Lmax) * (2 + kKvD) * 4);
+}
+
+w4a8_status_t w4kv_attention_decode(const void* q, const uint8_t* k_codes, const uint32_t* k_params,
+                                    const uint8_t* v_codes, const uint32_t* v_params, const int32_t* seq_lens,
+                                    int64_t B, int64_t Hq, int64_t Hkv, int64_t Lmax, int32_t D, float scale,
+                                    void* out, void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
+  const w4a8_status_t shape = check_kv_shape(B, Hq, Hkv, Lmax, D);
+  if (shape != W4A8_OK) return shape;
+  if (B == 0 || Hq == 0) return W4A8_OK;
+  if (q == nullptr || k_codes == nullptr || k_params == nullptr || v_codes == nullptr || v_params == nullptr ||
+      seq_lens == nullptr || out == nullptr)
+    return W4A8_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k_codes, 16) || !aligned(v_codes, 16) || !aligned(k_params, 4) ||
+      !aligned(v_params, 4) || !aligned(seq_lens, 4) || !aligned(out, 16) || !aligned(workspace, 256))
+    return W4A8_ERR_MISALIGNED;
+  if (workspace == nullptr || workspace_bytes < w4kv_attention_workspace_bytes(B, Hq, Hkv, Lmax, D))
+    return W4A8_ERR_WORKSPACE;
+  DeviceInfo* dev = nullptr;
+  w4a8_status_t st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+  const int64_t G = Hq / Hkv;
+  const int gc = kv_heads_per_cta(G);
+  KvAttnArgs a;
+  a.q = static_cast<const __half*>(q);
+  a.kc = k_codes;
+  a.kp = k_params;
+  a.vc = v_codes;
+  a.vp = v_params;
+  a.seq_lens = seq_lens;
+  a.out = static_cast<__half*>(out);
+  a.tickets = static_cast<int32_t*>(workspace);
+  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kv_ticket_bytes(B, Hq, Hkv));
+  a.Hq = static_cast<int>(Hq);
+  a.Hkv = static_cast<int>(Hkv);
+  a.nsplit = static_cast<int>(kv_splits(Lmax));
+  a.Lmax = Lmax;
+  a.scale = scale;
+  a.err = dev->err;
+  const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(Hkv * (G / gc)), static_cast<unsigned>(B));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  switch (gc) {
+    case 4: return launch_pdl(kv4_decode_kernel<4>, grid, dim3(kKvThreads), 0, s, 1, a);
+    case 2: return launch_pdl(kv4_decode_kernel<2>, grid, dim3(kKvThreads), 0, s, 1, a);
+    default: return launch_pdl(kv4_decode_kernel<1>, grid, dim3(kKvThreads), 0, s, 1, a);
+  }
 }
 
 }  // extern "C"
