@@ -57,7 +57,9 @@ def quantize_kv(X: np.ndarray):
     sf = s.astype(np.float32)
     pos = sf > 0
     safe = np.where(pos, sf, np.float32(1))
-    z = np.where(pos, np.clip(np.rint(-lo / safe), 0, KV_CODE_MAX), 0).astype(np.float32)
+    # z is an integer 0..15; stored as that integer's fp16 value (a range with
+    # lo = 0 gives rint(-0 / s) = -0, whose integer is 0, encoded +0)
+    z = np.where(pos, np.clip(np.rint(-lo / safe), 0, KV_CODE_MAX), 0).astype(np.int32).astype(np.float32)
     codes = np.clip(np.rint(x / safe[..., None]) + z[..., None], 0, KV_CODE_MAX)
     codes = np.where(pos[..., None], codes, 0)
     return codes.astype(np.uint8), s, z.astype(np.float16)

@@ -69,6 +69,15 @@ def test_zero_and_constant_vectors():
     assert abs(KV.dequant_kv(codes, s, z)[0, 0] + 3.0) <= 3.0 * 2.0 ** -11
 
 
+def test_zero_point_is_stored_as_its_integer():
+    """z is an integer 0..15 stored in fp16: a vector without negative
+    values (lo = 0) stores z = 0 as +0, not -0."""
+    x = np.abs(I.kv_vectors(1, 1, 8, 128, 17)[0, 0])
+    _, s, z = KV.quantize_kv(x)
+    assert (s > 0).all() and (z.view(np.uint16) == 0).all()
+    assert (KV.kv_params(s, z).view(np.uint32)[..., 0] >> 16 == 0).all()
+
+
 def test_static_parameters_reduce_to_codes():
     """A per-tensor (static) scheme stores one (s, z) for every vector; the
     dequantization only reads the pair, so vectors quantized with a shared

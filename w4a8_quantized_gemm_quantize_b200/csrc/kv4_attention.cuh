@@ -79,16 +79,19 @@ __global__ void __launch_bounds__(kKvThreads) kv4_quantize_kernel(KvQuantArgs a)
     hi = fmaxf(hi, 0.0f);
     const __half s = __float2half_rn(__fdiv_rn(__fsub_rn(hi, lo), 15.0f));
     const float sf = __half2float(s);
-    float z = 0.0f;
+    // z and the codes as integers (rint half to even, then clamp): z is
+    // stored as its integer's fp16 value, never a negative zero
+    int zi = 0;
     uint32_t packed = 0;
     if (sf > 0.0f) {
-      z = fminf(fmaxf(rintf(__fdiv_rn(-lo, sf)), 0.0f), 15.0f);
+      zi = min(max(__float2int_rn(__fdiv_rn(-lo, sf)), 0), 15);
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float c = fminf(fmaxf(rintf(__fdiv_rn(v[e], sf)) + z, 0.0f), 15.0f);
+        const int c = min(max(__float2int_rn(__fdiv_rn(v[e], sf)) + zi, 0), 15);
         packed |= static_cast<uint32_t>(c) << (4 * e);
       }
     }
+    const float z = static_cast<float>(zi);
     reinterpret_cast<uint16_t*>(a.codes + row * kKvRowBytes)[lane] = static_cast<uint16_t>(packed);
     if (lane == 0) {
       const __half zh = __float2half_rn(z);
