@@ -25,6 +25,13 @@ over the whole step (quantization included), summed over ranks.
 `--impl reference` times the CPU oracle on the host cores instead (bounded
 sample of the same workload), printing the same kind of line.
 
+`--workload kv-decode` (and the other kv-* workloads) measures the 4-bit
+KV-cache decode attention instead: one step = for each of LAYERS layer
+caches, `w4kv_append` of the new token's K and V (written at position
+L_b - 1) and `w4kv_attention_decode` over the L_b cached tokens of every
+sequence; `value` is cache bytes read per second (codes + parameter words
+of K and V).
+
 Multi-GPU: the path does not shard across GPUs here (replicas only): every
 rank runs the whole workload on its own GPU; the time is the max over ranks.
 """
@@ -478,12 +485,232 @@ def run_gpu(args, world, rank, local):
                 gpu_name=torch.cuda.get_device_name(dev))
 
 
+# ------------------------------------------------------ 4-bit KV attention
+KV_METRIC = "KV4 decode attention: 4-bit KV-cache bytes read per second on 1 B200, as % of HBM roofline"
+KV_LAYERS = 4  # distinct layer caches per step: the step's cache bytes exceed L2
+
+
+def kv_cache_bytes(lens, Hkv):
+    """Bytes of the cached K and V a decode step must read: per token and kv
+    head 64 code bytes + one 4-byte parameter word, for K and for V."""
+    return int(np.sum(lens)) * Hkv * 2 * (64 + 4)
+
+
+def kv_algorithmic_bytes(lens, Hq, Hkv):
+    """The attention launch's bytes: the cache it reads, the queries, the output."""
+    B = len(lens)
+    return kv_cache_bytes(lens, Hkv) + 2 * B * Hq * 128 * 2
+
+
+def kv_case(wl, seed_tag):
+    Hq, Hkv, D = wl.heads
+    K = I.kv_vectors(wl.batch, Hkv, wl.max_len, D, I.seed_of(seed_tag, "k", wl.name))
+    V = I.kv_vectors(wl.batch, Hkv, wl.max_len, D, I.seed_of(seed_tag, "v", wl.name), outlier_scale=1.0)
+    q = I.kv_queries(wl.batch, Hq, D, I.seed_of(seed_tag, "q", wl.name))
+    lens = I.kv_seq_lens(wl, I.seed_of(seed_tag, "lens", wl.name))
+    return K, V, q, lens
+
+
+def cpu_oracle_run_kv(workload, budget_s):
+    """Times the CPU oracle's decode attention on sequences of the workload
+    until the budget is spent; returns (cache GB/s, sample, threads, seconds)."""
+    from oracle import kv4_oracle as KV
+    wl = I.KV_WORKLOADS[workload]
+    Hq, Hkv, D = wl.heads
+    key = ("kv", workload)
+    if key not in _ORACLE_WEIGHTS:  # the cache, quantized once (untimed), as on the GPU
+        K, V, q, lens = kv_case(wl, "bench")
+        kc, ks, kz = KV.quantize_kv(K)
+        vc, vs, vz = KV.quantize_kv(V)
+        _ORACLE_WEIGHTS[key] = (K, V, q, lens, KV.pack_kv(kc), KV.kv_params(ks, kz), KV.pack_kv(vc),
+                                KV.kv_params(vs, vz))
+    K, V, q, lens, kc, kp, vc, vp = _ORACLE_WEIGHTS[key]
+    done_t, done_b, seqs = 0.0, 0, []
+    for b in range(wl.batch):
+        if done_t > budget_s and seqs:
+            break
+        L = int(lens[b])
+        sl = slice(b, b + 1)
+        t0 = time.perf_counter()
+        # the step of one sequence: quantize the new token's K and V, attend
+        KV.quantize_kv(K[b, :, L - 1])
+        KV.quantize_kv(V[b, :, L - 1])
+        KV.attention_decode(q[sl], kc[sl], kp[sl], vc[sl], vp[sl], lens[sl], 1.0 / np.sqrt(D))
+        done_t += time.perf_counter() - t0
+        done_b += kv_cache_bytes(lens[sl], Hkv)
+        seqs.append(f"seq {b} ({L} tokens)")
+    return done_b / done_t / 1e9, seqs, cpu_threads(), done_t
+
+
+def run_gpu_kv(args, world, rank, local):
+    import torch
+    import w4a8_quantized_gemm_quantize_b200 as w4a8
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = I.KV_WORKLOADS[args.workload]
+    Hq, Hkv, D = wl.heads
+    K, V, q, lens = kv_case(wl, "bench")
+    scale = float(np.float32(1.0 / np.sqrt(D)))
+    # ---- offline: the caches of KV_LAYERS layers (untimed)
+    caches = []
+    for _ in range(KV_LAYERS):
+        kc, kp = w4a8.kv4_quantize(torch.from_numpy(K).to(dev))
+        vc, vp = w4a8.kv4_quantize(torch.from_numpy(V).to(dev))
+        caches.append((kc, kp, vc, vp))
+    qd = torch.from_numpy(q).to(dev)
+    lens_d = torch.from_numpy(lens).to(dev)
+    pos_d = torch.from_numpy(np.maximum(lens - 1, 0).astype(np.int32)).to(dev)
+    k_new = torch.from_numpy(np.ascontiguousarray(K[np.arange(wl.batch), :, np.maximum(lens - 1, 0)])).to(dev)
+    v_new = torch.from_numpy(np.ascontiguousarray(V[np.arange(wl.batch), :, np.maximum(lens - 1, 0)])).to(dev)
+    outs = [torch.empty((wl.batch, Hq, D), dtype=torch.float16, device=dev) for _ in range(KV_LAYERS)]
+    ws = torch.zeros(w4a8.kv4_workspace_bytes(wl.batch, Hq, Hkv, wl.max_len), dtype=torch.uint8, device=dev)
+    torch.cuda.synchronize()
+
+    def step(attn_only=False, h2d=None, d2h=None):
+        for i, (kc, kp, vc, vp) in enumerate(caches):
+            if h2d is not None:
+                qd.copy_(h2d[0], non_blocking=True)
+                k_new.copy_(h2d[1], non_blocking=True)
+                v_new.copy_(h2d[2], non_blocking=True)
+            if not attn_only:
+                w4a8.kv4_append(k_new, v_new, pos_d, kc, kp, vc, vp)
+            w4a8.kv4_attention_decode(qd, kc, kp, vc, vp, lens_d, scale, out=outs[i], workspace=ws)
+            if d2h is not None:
+                d2h[i].copy_(outs[i], non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert w4a8.get_device_error(dev) == 0
+
+    def capture(attn_only):
+        g = torch.cuda.CUDAGraph()
+        cs = torch.cuda.Stream(dev)
+        cs.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(cs):
+            with torch.cuda.graph(g, stream=cs):
+                for _ in range(args.steps):
+                    step(attn_only)
+        torch.cuda.current_stream(dev).wait_stream(cs)
+        return g
+
+    g_plain, g_attn = capture(False), capture(True)
+    for g in (g_plain, g_attn):
+        g.replay()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    t0, t1, t2, t3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        t0.record(stream)
+        g_plain.replay()
+        t1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        t2.record(stream)
+        g_attn.replay()
+        t3.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    max_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    attn_ms = max_over_ranks(t2.elapsed_time(t3), world)
+    assert w4a8.get_device_error(dev) == 0
+    del g_plain, g_attn
+
+    # ---- end to end through the public API: pinned q and new K/V in, Y out
+    h2d = tuple(t.cpu().pin_memory() for t in (qd, k_new, v_new))
+    d2h = [torch.empty((wl.batch, Hq, D), dtype=torch.float16).pin_memory() for _ in range(KV_LAYERS)]
+    step(h2d=h2d, d2h=d2h)
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step(h2d=h2d, d2h=d2h)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    for i in range(KV_LAYERS):
+        assert torch.equal(d2h[i], outs[i].cpu())
+    return dict(max_ms=max_ms, attn_ms=attn_ms, e2e_ms=e2e_ms, clocks=clk.summary(), lens=lens,
+                h2d_bytes=KV_LAYERS * sum(t.numel() * t.element_size() for t in h2d),
+                d2h_bytes=KV_LAYERS * wl.batch * Hq * D * 2, gpu_name=torch.cuda.get_device_name(dev))
+
+
+def main_kv(args, world, rank, local):
+    wl = I.KV_WORKLOADS[args.workload]
+    Hq, Hkv, D = wl.heads
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cpu_oracle_run_kv(args.workload, 0.0)  # untimed warm-up (one sequence)
+        tot_b, tot_t, sample, threads = 0.0, 0.0, [], 1
+        for _ in range(args.steps):
+            v, sample, threads, t = cpu_oracle_run_kv(args.workload, args.cpu_seconds / max(args.steps, 1))
+            tot_b += v * t * 1e9
+            tot_t += t
+        value = tot_b / tot_t / 1e9
+        print(json.dumps({
+            "metric": KV_METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "heads": list(wl.heads), "batch": wl.batch,
+                       "max_len": wl.max_len},
+            "impl": "reference",
+            "cpu_baseline": {"value": round(value, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                             "sample": f"per step: {len(sample)} sequences ({'; '.join(sample)})"},
+            "e2e": {"value": round(value, 3), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+            flush=True)
+        return
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
+    r = run_gpu_kv(args, world, rank, local)
+    peaks = load_peaks()
+    lens = r["lens"]
+    cache_b = KV_LAYERS * kv_cache_bytes(lens, Hkv)
+    ms_step = r["max_ms"] / args.steps
+    attn_launch_ms = r["attn_ms"] / (args.steps * KV_LAYERS)
+    achieved = kv_algorithmic_bytes(lens, Hq, Hkv) / (attn_launch_ms * 1e-3) / 1e9
+    line = {
+        "metric": KV_METRIC, "value": round(world * cache_b / (ms_step * 1e-3) / 1e9, 1), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": args.workload, "heads": list(wl.heads), "batch": wl.batch, "max_len": wl.max_len,
+                   "tokens": int(np.sum(lens)), "layers_per_step": KV_LAYERS,
+                   "l2": f"inputs larger than L2: {KV_LAYERS} layer caches, {cache_b / 1e6:.0f} MB per step",
+                   "parallelism": f"replicas x{world}"},
+        "gpu_launches": 3 * KV_LAYERS * args.steps,
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
+                     "peak_source": f"{peaks['source']} HBM copy", "kernel": "kv4_decode_kernel",
+                     "avg_launch_us": round(attn_launch_ms * 1e3, 3)},
+        "e2e": {"value": round(world * cache_b / (r["e2e_ms"] / args.steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"]},
+        "clocks": r["clocks"], "gpu": r["gpu_name"],
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, sample, threads, t = cpu_oracle_run_kv(args.workload, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": round(v, 3), "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{len(sample)} of {wl.batch} sequences, {t:.1f} s of oracle time"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--workload", default="decode", choices=sorted(I.WORKLOADS) + sorted(I.KV_WORKLOADS))
     ap.add_argument("--impl", default="w4a8", choices=["w4a8", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the CPU-oracle baseline sample")
@@ -504,6 +731,8 @@ def main():
     args.warmup = max(args.warmup, 3)
 
     world, rank, local = dist_env()
+    if args.workload in I.KV_WORKLOADS:
+        return main_kv(args, world, rank, local)
     if args.impl == "reference":
         return main_reference(args, world, rank)
 
