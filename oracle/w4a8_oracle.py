@@ -528,3 +528,91 @@ def lut_unpack_weights(blob: np.ndarray):
     s = (blob[ssrc].astype(np.uint16) | (blob[ssrc + 1].astype(np.uint16) << 8)).view(np.float16)
     T = np.frombuffer(bytes(blob[t_off:t_off + 32]), dtype=np.float16).copy()
     return q, s, T, N, K
+
+
+# ---------------------------------------------------------------------------
+# 3-bit lookup-table weights ("Fast Matrix Multiplications for Lookup
+# Table-Quantized LLMs", abstract: bit widths that do not divide a byte).
+# Same arithmetic as above with an 8-entry table (`lut_dequant`,
+# `lut_gemm_exact`, `lut_error_bound` and `lut_quantize_weights` apply as they
+# stand). The storage is this file's reading: a tile row's 128 indices are
+# three 16-byte bit planes, plane c holding bit c of every index (bit kk of
+# the plane, i.e. bit kk % 8 of byte kk // 8, is bit c of the index at in-tile
+# k = kk), plane c of row r at (c * 128 + r) * 16, so no index straddles two
+# 16-byte vectors; then the tile's 128 fp16 row scales.
+LUT3_MAGIC = 0x544C3357  # b"W3LT" little-endian
+LUT3_TILE_CODE_BYTES = 3 * 16 * TILE_N  # 6144
+LUT3_TILE_BYTES = LUT3_TILE_CODE_BYTES + LUT_TILE_SCALE_BYTES  # 6400
+
+
+def lut3_packed_bytes(N: int, K: int, group: int = GROUP) -> int:
+    """Header + (N/128)*(K/128) tiles of 6400 bytes + the table (8 fp16) padded to 64 bytes."""
+    return HEADER_BYTES + (N // TILE_N) * (K // TILE_K) * LUT3_TILE_BYTES + 64
+
+
+def lut3_bit_position(r: int, kk: int, c: int):
+    """(byte offset inside a tile's index area, bit) of bit c of the index of
+    row r at in-tile k = kk."""
+    return (c * TILE_N + r) * 16 + kk // 8, kk % 8
+
+
+def lut3_pack_weights(q, s, T, group: int = GROUP) -> np.ndarray:
+    """Writes the 3-bit lookup-table blob from its definition. Header as the
+    4-bit blob's with magic 'W3LT' and tile bytes 6400; tile (nt, kt) at
+    64 + (nt*(K/128) + kt)*6400: the three bit planes of each row, then the
+    128 rows' fp16 scales of group kt (row r at 6144 + 2r); after the tiles
+    the 8 fp16 table entries, zero padded to 64 bytes."""
+    assert group == GROUP
+    q = np.asarray(q, dtype=np.uint8)
+    assert q.max(initial=0) < 8 and len(T) == 8
+    N, K = q.shape
+    KT = K // TILE_K
+    out = np.zeros(lut3_packed_bytes(N, K, group), dtype=np.uint8)
+    t_off = HEADER_BYTES + (N // TILE_N) * KT * LUT3_TILE_BYTES
+    hdr = bytearray(HEADER_BYTES)
+    hdr[0:4] = LUT3_MAGIC.to_bytes(4, "little")
+    hdr[4:8] = (1).to_bytes(4, "little")
+    hdr[8:16] = int(N).to_bytes(8, "little", signed=True)
+    hdr[16:24] = int(K).to_bytes(8, "little", signed=True)
+    hdr[24:28] = int(group).to_bytes(4, "little", signed=True)
+    hdr[28:32] = LUT3_TILE_BYTES.to_bytes(4, "little")
+    hdr[32:40] = int(t_off).to_bytes(8, "little")
+    out[:HEADER_BYTES] = np.frombuffer(bytes(hdr), dtype=np.uint8)
+    for n in range(N):
+        nt, r = divmod(n, TILE_N)
+        for kt in range(KT):
+            base = HEADER_BYTES + (nt * KT + kt) * LUT3_TILE_BYTES
+            row = q[n, kt * TILE_K:(kt + 1) * TILE_K]
+            for c in range(3):
+                bits = (row >> c) & 1
+                plane = np.packbits(bits, bitorder="little")  # bit kk -> byte kk // 8, bit kk % 8
+                off = base + (c * TILE_N + r) * 16
+                out[off:off + 16] = plane
+            sb = np.frombuffer(np.float16(s[n, kt]).tobytes(), dtype=np.uint8)
+            out[base + LUT3_TILE_CODE_BYTES + 2 * r:base + LUT3_TILE_CODE_BYTES + 2 * r + 2] = sb
+    out[t_off:t_off + 16] = np.frombuffer(np.asarray(T, dtype=np.float16).tobytes(), dtype=np.uint8)
+    return out
+
+
+def lut3_unpack_weights(blob: np.ndarray):
+    """Inverse of `lut3_pack_weights`: returns (q, s, T, N, K)."""
+    hdr = bytes(blob[:HEADER_BYTES])
+    assert int.from_bytes(hdr[0:4], "little") == LUT3_MAGIC
+    N = int.from_bytes(hdr[8:16], "little", signed=True)
+    K = int.from_bytes(hdr[16:24], "little", signed=True)
+    t_off = int.from_bytes(hdr[32:40], "little")
+    KT = K // TILE_K
+    q = np.zeros((N, K), dtype=np.uint8)
+    s = np.zeros((N, KT), dtype=np.float16)
+    for n in range(N):
+        nt, r = divmod(n, TILE_N)
+        for kt in range(KT):
+            base = HEADER_BYTES + (nt * KT + kt) * LUT3_TILE_BYTES
+            for c in range(3):
+                off = base + (c * TILE_N + r) * 16
+                bits = np.unpackbits(blob[off:off + 16], bitorder="little")
+                q[n, kt * TILE_K:(kt + 1) * TILE_K] |= (bits << c).astype(np.uint8)
+            so = base + LUT3_TILE_CODE_BYTES + 2 * r
+            s[n, kt] = np.frombuffer(bytes(blob[so:so + 2]), dtype=np.float16)[0]
+    T = np.frombuffer(bytes(blob[t_off:t_off + 16]), dtype=np.float16).copy()
+    return q, s, T, N, K

@@ -673,3 +673,64 @@ def test_lut_quantize_picks_the_nearest_entry():
                 x = Fraction(float(np.float32(W[n, k]) / np.float32(s[n, g])))
                 d = [abs(x - Fraction(float(t))) for t in T]
                 assert d[q[n, k]] == min(d) and q[n, k] == d.index(min(d)), (n, k)
+
+
+# ------------------------------------------------ 3-bit lookup-table storage
+from w4a8_quantized_gemm_quantize_b200 import inputs as I  # noqa: E402  (seeded generators only)
+
+def test_lut3_planes_hand_computed():
+    """Indices q[kk] = kk % 8 on every row: bit c of kk % 8 repeats with
+    period 8, so every byte of plane 0 is 0b10101010, of plane 1 0b11001100,
+    of plane 2 0b11110000; the scales follow the planes."""
+    N, K = 128, 256
+    q = np.tile((np.arange(K) % 8).astype(np.uint8), (N, 1))
+    s = np.full((N, K // 128), np.float16(0.5))
+    T = I.lut3_table()
+    blob = O.lut3_pack_weights(q, s, T)
+    assert blob.size == O.lut3_packed_bytes(N, K) == 64 + 2 * 6400 + 64
+    for kt in range(2):
+        base = 64 + kt * 6400
+        for c, want in enumerate((0xAA, 0xCC, 0xF0)):
+            assert (blob[base + c * 2048:base + (c + 1) * 2048] == want).all()
+        assert (blob[base + 6144:base + 6400].view(np.float16) == np.float16(0.5)).all()
+    assert int.from_bytes(bytes(blob[0:4]), "little") == O.LUT3_MAGIC
+    assert bytes(blob[0:4]) == b"W3LT"
+    t_off = int.from_bytes(bytes(blob[32:40]), "little")
+    assert t_off == 64 + 2 * 6400
+    assert (blob[t_off:t_off + 16].view(np.float16) == T).all() and not blob[t_off + 16:].any()
+
+
+def test_lut3_single_index_sets_its_bits():
+    """One nonzero index (7 = all three bits) at (n, k) sets exactly bit
+    k % 128 % 8 of byte k % 128 // 8 in each plane of row n % 128 of tile
+    (n // 128, k // 128), and nothing else in the index area."""
+    N, K = 256, 384
+    for n, k in [(0, 0), (5, 127), (130, 200), (255, 383)]:
+        q = np.zeros((N, K), np.uint8)
+        q[n, k] = 7
+        blob = O.lut3_pack_weights(q, np.zeros((N, K // 128), np.float16), I.lut3_table())
+        tile = 64 + ((n // 128) * (K // 128) + k // 128) * 6400
+        expect = set()
+        for c in range(3):
+            off, bit = O.lut3_bit_position(n % 128, k % 128, c)
+            assert off == (c * 128 + n % 128) * 16 + (k % 128) // 8 and bit == k % 8
+            expect.add((tile + off, bit))
+        t_off = int.from_bytes(bytes(blob[32:40]), "little")
+        nz = np.flatnonzero(blob[64:t_off]) + 64
+        got = {(int(i), b) for i in nz for b in range(8) if (blob[i] >> b) & 1}
+        assert got == expect
+
+
+def test_lut3_round_trip_and_dequant():
+    N, K = 256, 640
+    q, s = I.lut3_codes(N, K, 3)
+    T = I.lut3_table()
+    q2, s2, T2, N2, K2 = O.lut3_unpack_weights(O.lut3_pack_weights(q, s, T))
+    assert (N2, K2) == (N, K) and np.array_equal(q2, q)
+    assert np.array_equal(s2.view(np.uint16), s.view(np.uint16)) and np.array_equal(T2.view(np.uint16), T.view(np.uint16))
+    # the 3-bit weights dequantize exactly as the 4-bit path does with an 8-entry table
+    W = O.lut_dequant(q, s, T)
+    assert np.array_equal(W.astype(np.float64), (T.astype(np.float32)[q] * np.repeat(s.astype(np.float32), 128, axis=1)).astype(np.float16).astype(np.float64))
+    # and the nearest-entry quantizer returns 3-bit indices for an 8-entry table
+    qq, ss = O.lut_quantize_weights(O.lut_dequant(q, s, T).astype(np.float32), T)
+    assert qq.max() < 8

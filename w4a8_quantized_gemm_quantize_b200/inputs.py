@@ -188,3 +188,23 @@ def kv_seq_lens(wl: KvWorkload, seed: int) -> np.ndarray:
     lens = rng.integers(wl.max_len // 2, wl.max_len + 1, size=wl.batch).astype(np.int32)
     lens[0] = wl.max_len
     return lens
+
+
+def lut3_table(delta: float = 0.06) -> np.ndarray:
+    """An 8-entry NormalFloat-style table for 3-bit indices (input data):
+    standard-normal quantiles at evenly spaced probabilities, 4 below and 3
+    above an exact zero, each side scaled to reach -1 / +1; fp16."""
+    from scipy.special import ndtri
+    neg = ndtri(np.linspace(delta, 0.5, 5)[:-1])
+    pos = ndtri(np.linspace(0.5, 1.0 - delta, 4)[1:])
+    t = np.concatenate([neg / -neg.min(), [0.0], pos / pos.max()])
+    return t.astype(np.float16)
+
+
+def lut3_codes(N: int, K: int, seed: int, group: int = GROUP):
+    """3-bit lookup-table weights drawn directly: indices q ~ U[0,7] (uint8
+    [N,K]) and per-(row, group) scales s ~ U[0.005, 0.05] (fp16 [N, K/group])."""
+    rng = np.random.default_rng(seed)
+    q = rng.integers(0, 8, size=(N, K), dtype=np.uint8)
+    s = rng.uniform(0.005, 0.05, size=(N, K // group)).astype(np.float16)
+    return q, s
