@@ -54,3 +54,23 @@ def test_two_gloo_ranks_max_and_barrier():
     assert [(r, w) for r, w, _, _ in res] == [(0, 2), (1, 2)]
     assert all(got == 4.5 for _, _, got, _ in res)  # max over ranks of 1.5, 4.5
     assert res[0][3] == "skipped" and res[1][3] is None  # rank 1 leaves the reference arm at once
+
+
+def test_kv_reference_arm_prints_one_line():
+    """`bench.py --workload kv-tiny --impl reference` (the CPU oracle as the
+    reference arm of the KV-cache attention workload) prints one JSON line
+    with the contract's keys; the GEMM lines are not involved."""
+    import json
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "kv-tiny", "--impl",
+                        "reference", "--steps", "2", "--warmup", "3", "--cpu-seconds", "0.2"],
+                       capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "impl", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["value"] > 0 and d["config"]["workload"] == "kv-tiny"
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
