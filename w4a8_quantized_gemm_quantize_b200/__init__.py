@@ -502,10 +502,25 @@ def kv4_workspace_bytes(B: int, Hq: int, Hkv: int, Lmax: int) -> int:
     return int(lib().w4kv_attention_workspace_bytes(B, Hq, Hkv, Lmax, KV_HEAD_DIM))
 
 
+_kv_ws = {}
+
+
+def _kv_workspace_for(device, nbytes: int):
+    """A zero-filled workspace per device, grown on demand and reused: the
+    attention call leaves the part it must find zero (its tickets) zero."""
+    torch = _torch()
+    key = str(device)
+    ws = _kv_ws.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = _kv_ws[key] = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+    return ws
+
+
 def kv4_attention_decode(q, k_codes, k_params, v_codes, v_params, seq_lens, scale, out=None, workspace=None):
     """Y fp16 [B, Hq, 128] = decode attention of q fp16 [B, Hq, 128] over the
-    4-bit caches with lengths seq_lens int32 [B]; workspace zero-filled
-    uint8 (allocated here if not given)."""
+    4-bit caches with lengths seq_lens int32 [B]; workspace: zero-filled
+    uint8 (a per-device one is kept here if none is given; calls on one
+    device that share it must not overlap on the GPU)."""
     torch = _torch()
     _require_cuda(q, k_codes, k_params, v_codes, v_params, seq_lens, out, workspace)
     if q.dtype != torch.float16 or q.dim() != 3 or q.shape[2] != KV_HEAD_DIM:
@@ -514,7 +529,7 @@ def kv4_attention_decode(q, k_codes, k_params, v_codes, v_params, seq_lens, scal
     Hkv, Lmax = k_codes.shape[1], k_codes.shape[2]
     Y = out if out is not None else torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
     if workspace is None:
-        workspace = torch.zeros(max(kv4_workspace_bytes(B, Hq, Hkv, Lmax), 1), dtype=torch.uint8, device=q.device)
+        workspace = _kv_workspace_for(q.device, kv4_workspace_bytes(B, Hq, Hkv, Lmax))
     ws_bytes = workspace.numel() * workspace.element_size()
     _check(lib().w4kv_attention_decode(_ptr(q), _ptr(k_codes), _ptr(k_params), _ptr(v_codes), _ptr(v_params),
                                        _ptr(seq_lens), B, Hq, Hkv, Lmax, D, float(scale), _ptr(Y), _ptr(workspace),
