@@ -579,6 +579,15 @@ def run_gpu_kv(args, world, rank, local):
             if d2h is not None:
                 d2h[i].copy_(outs[i], non_blocking=True)
 
+    if args.profile:
+        # for an external profiler: eager steps only, no timing, no JSON line
+        for _ in range(args.profile):
+            step()
+        torch.cuda.synchronize()
+        assert w4a8.get_device_error(dev) == 0
+        print(f"profile: {args.profile} eager steps of {KV_LAYERS} layer caches done")
+        return None
+
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -671,6 +680,8 @@ def main_kv(args, world, rank, local):
         torch.cuda.set_device(local)
         dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=torch.device("cuda", local))
     r = run_gpu_kv(args, world, rank, local)
+    if r is None:  # --profile
+        return 0
     peaks = load_peaks()
     lens = r["lens"]
     cache_b = KV_LAYERS * kv_cache_bytes(lens, Hkv)

@@ -18,6 +18,16 @@ Qwen1.5-72B linears, "QServe/QoQ" abstract on the lmdeploy issue
 Activations are fp16 N(0, 1) with round(0.01*K) outlier channels scaled by
 20; the outlier channels depend on K only, so every token of a layer shares
 them. Dense weights are fp32 N(0, std) with std 0.02 (Llama) or 0.015 (Qwen).
+
+Lookup-table weights (`lut_table`, `lut_codes`, 3-bit `lut3_table`,
+`lut3_codes`): NormalFloat-style tables, uniform indices, group scales on
+[0.005, 0.05].
+
+KV-cache attention (`KV_WORKLOADS`): ``kv-tiny`` (3 sequences, 4 query / 2 kv
+heads, <= 300 tokens), ``kv-decode`` (Llama-3-8B attention, 32 / 8 heads of
+128, 16 sequences of 2048..4096 tokens), ``kv-long`` (4 x 32768),
+``kv-qwen72b`` (64 / 64 heads, 8 x 2048..4096). Keys N(0, 1) with
+round(0.04*D) outlier channels x10 per head, values and queries N(0, 1).
 """
 from __future__ import annotations
 
