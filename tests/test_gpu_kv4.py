@@ -173,3 +173,37 @@ def test_kv4_length_out_of_range_is_clamped_and_reported():
     assert w4a8.get_device_error(DEV) == 7
     w4a8.clear_device_error(DEV)
     assert np.array_equal(Y.view(np.uint16), Y_ok.view(np.uint16))
+
+
+def test_kv4_decode_flow_quantize_append_attend():
+    """The decode flow through the public calls: the cache of L tokens
+    quantized on the GPU, the new token appended at position L, attention
+    over L + 1 tokens; the oracle quantizes the same fp16 vectors itself."""
+    B, Hq, Hkv, Lmax = 3, 8, 2, 400
+    K = I.kv_vectors(B, Hkv, Lmax, 128, 301)
+    V = I.kv_vectors(B, Hkv, Lmax, 128, 302, outlier_scale=1.0)
+    q = I.kv_queries(B, Hq, 128, 303)
+    L = np.array([399, 256, 1], np.int32)       # tokens already cached
+    kc, kp = w4a8.kv4_quantize(dev(K))
+    vc, vp = w4a8.kv4_quantize(dev(V))
+    newK = np.ascontiguousarray(K[np.arange(B), :, L])   # the token at position L of each sequence
+    newV = np.ascontiguousarray(V[np.arange(B), :, L])
+    # positions >= L hold stale vectors until appended: overwrite position L with garbage first
+    bi = torch.arange(B, device=DEV)
+    li = torch.from_numpy(L).to(DEV).long()
+    kc[bi, :, li] = 0xFF
+    vp[bi, :, li] = -1
+    w4a8.kv4_append(dev(newK), dev(newV), dev(L), kc, kp, vc, vp)
+    lens = L + 1
+    ws = torch.zeros(w4a8.kv4_workspace_bytes(B, Hq, Hkv, Lmax), dtype=torch.uint8, device=DEV)
+    Y = w4a8.kv4_attention_decode(dev(q), kc, kp, vc, vp, dev(lens), SCALE, workspace=ws)
+    torch.cuda.synchronize()
+    okc, oks, okz = KV.quantize_kv(K)
+    ovc, ovs, ovz = KV.quantize_kv(V)
+    okc, okp, ovc, ovp = KV.pack_kv(okc), KV.kv_params(oks, okz), KV.pack_kv(ovc), KV.kv_params(ovs, ovz)
+    for b in range(B):  # the cached prefix and the appended token, byte for byte
+        n = lens[b]
+        assert (host(kc)[b, :, :n] == okc[b, :, :n]).all() and (host(vc)[b, :, :n] == ovc[b, :, :n]).all()
+        assert (host(kp).view(np.uint32)[b, :, :n] == okp.view(np.uint32)[b, :, :n, 0]).all()
+        assert (host(vp).view(np.uint32)[b, :, :n] == ovp.view(np.uint32)[b, :, :n, 0]).all()
+    check(host(Y), q, okc, okp, ovc, ovp, lens)
