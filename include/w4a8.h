@@ -330,6 +330,28 @@ W4A8_API w4a8_status_t w4lut_gemm_ex(const void* A, const void* packed, int64_t 
                                      const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
 
 /*
+ * 3-bit lookup-table weights ("Fast Matrix Multiplications for Lookup
+ * Table-Quantized LLMs", abstract: bit widths that do not divide a byte):
+ * the same GEMM with an 8-entry fp16 table and indices 0..7. Blob,
+ * little-endian: header as above with magic "W3LT" and tile bytes 6400;
+ * (N/128) x (K/128) tiles of 6400 bytes, tile (nt, kt) at 64 + (nt * K/128 +
+ * kt) * 6400: per row three 16-byte bit planes, plane c (bit c of the row's
+ * 128 indices; bit kk of the plane = bit kk % 8 of byte kk / 8 is bit c of
+ * the index at in-tile k = kk) at (c * 128 + r) * 16; then the 128 fp16 row
+ * scales (row r at 6144 + 2r); after the tiles the 8 fp16 table entries,
+ * zero padded to 64 bytes. Entry points as for the 4-bit table (q holds one
+ * index 0..7 per byte; table holds 8 fp16 values).
+ */
+W4A8_API size_t w4lut3_packed_bytes(int64_t N, int64_t K, int32_t group);
+W4A8_API w4a8_status_t w4lut3_pack_weights(const uint8_t* q, const void* s, const void* table, int64_t N, int64_t K,
+                                           int32_t group, void* packed, size_t packed_bytes, w4a8_stream_t stream);
+W4A8_API w4a8_status_t w4lut3_gemm(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
+                                   void* workspace, size_t workspace_bytes, w4a8_stream_t stream);
+W4A8_API w4a8_status_t w4lut3_gemm_ex(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
+                                      float* acc, void* workspace, size_t workspace_bytes,
+                                      const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
+
+/*
  * 4-bit KV cache and decode attention over it (the KV4 of W4A8KV4,
  * "QServe/QoQ" abstract on the lmdeploy issue "[Feature] Support W4A8KV4
  * Quantization(QServe/QoQ)", Motivation: 4-bit KV cache, memory-bound fused

@@ -24,7 +24,7 @@ def L():
 
 def declared_functions():
     src = open(HEADER).read()
-    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4(?:a[48]|lut|kv)_\w+)\s*\(", src)))
+    return sorted(set(re.findall(r"W4A8_API\s+[\w\s\*]+?\b(w4(?:a[48]|lut3?|kv)_\w+)\s*\(", src)))
 
 
 def test_header_declares_entry_points():
@@ -193,3 +193,20 @@ def test_kv4_validation(L):
     assert ap(FAKE, FAKE, FAKE, 2, 8, 1024, 64, FAKE, FAKE, FAKE, FAKE, None) == 2
     assert ap(FAKE, FAKE, None, 2, 8, 1024, 128, FAKE, FAKE, FAKE, FAKE, None) == 1
     assert ap(FAKE, FAKE, FAKE, 0, 8, 1024, 128, FAKE, FAKE, FAKE, FAKE, None) == 0
+
+
+def test_lut3_validation(L):
+    assert L.w4lut3_packed_bytes(256, 512, 128) == 64 + 2 * 4 * 6400 + 64
+    assert L.w4lut3_packed_bytes(200, 512, 128) == 0
+    p = L.w4lut3_pack_weights
+    nb = L.w4lut3_packed_bytes(256, 256, 128)
+    assert p(FAKE, FAKE, FAKE, 200, 256, 128, FAKE, nb, None) == 2
+    assert p(FAKE, FAKE, None, 256, 256, 128, FAKE, nb, None) == 1        # no table
+    assert p(FAKE, FAKE, FAKE, 256, 256, 128, FAKE, nb - 1, None) == 1
+    assert p(FAKE, FAKE, FAKE, 256, 256, 128, FAKE_ODD, nb, None) == 3    # blob alignment
+    g = L.w4lut3_gemm
+    assert g(FAKE, FAKE, 4, 100, 256, FAKE, None, 0, None) == 2
+    assert g(FAKE, FAKE, 4, 128, 256, None, None, 0, None) == 1
+    assert g(FAKE, FAKE, 0, 128, 256, FAKE, None, 0, None) == 0
+    bad = w4a8.GemmOpts(0, 64, 0, 0)
+    assert L.w4lut3_gemm_ex(FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1

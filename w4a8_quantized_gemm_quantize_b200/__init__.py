@@ -21,7 +21,7 @@ __all__ = [
     "gemm_debug_acc", "gemm_ex", "gemm_noalloc", "get_device_error", "clear_device_error",
     "selftest_bounded_wait", "quantize_act_static", "w4a4_quantize_act", "w4a4_quantize_act_static",
     "w4a4_gemm", "w4a4_gemm_ex", "w4a4_workspace_bytes", "lut_packed_bytes", "lut_pack_weights", "lut_gemm",
-    "lut_gemm_ex", "kv4_quantize", "kv4_append", "kv4_workspace_bytes", "kv4_attention_decode",
+    "lut_gemm_ex", "lut3_packed_bytes", "lut3_pack_weights", "lut3_gemm", "lut3_gemm_ex", "kv4_quantize", "kv4_append", "kv4_workspace_bytes", "kv4_attention_decode",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +35,7 @@ EXPORTED_SYMBOLS = (
     "w4a4_quantize_act", "w4a4_quantize_act_static", "w4a4_gemm", "w4a4_gemm_ex", "w4a4_gemm_workspace_bytes",
     "w4lut_packed_bytes", "w4lut_pack_weights", "w4lut_gemm", "w4lut_gemm_ex",
     "w4kv_quantize", "w4kv_append", "w4kv_attention_workspace_bytes", "w4kv_attention_decode",
+    "w4lut3_packed_bytes", "w4lut3_pack_weights", "w4lut3_gemm", "w4lut3_gemm_ex",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
@@ -89,6 +90,10 @@ def lib() -> ctypes.CDLL:
         "w4lut_gemm_ex": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, vp, sz, ctypes.POINTER(GemmOpts), vp]),
         "w4a4_gemm_ex": (ctypes.c_int, [vp, vp, vp, vp, i64, i64, i64, vp, vp, vp, sz,
                                         ctypes.POINTER(GemmOpts), vp]),
+        "w4lut3_packed_bytes": (sz, [i64, i64, i32]),
+        "w4lut3_pack_weights": (ctypes.c_int, [vp, vp, vp, i64, i64, i32, vp, sz, vp]),
+        "w4lut3_gemm": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, sz, vp]),
+        "w4lut3_gemm_ex": (ctypes.c_int, [vp, vp, i64, i64, i64, vp, vp, vp, sz, ctypes.POINTER(GemmOpts), vp]),
         "w4kv_quantize": (ctypes.c_int, [vp, i64, i32, vp, vp, vp]),
         "w4kv_append": (ctypes.c_int, [vp, vp, vp, i64, i64, i64, i32, vp, vp, vp, vp, vp]),
         "w4kv_attention_workspace_bytes": (sz, [i64, i64, i64, i64, i32]),
@@ -427,6 +432,56 @@ def lut_gemm(A, blob, N: int, K: int, out=None, workspace=None):
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().w4lut_gemm(_ptr(A), _ptr(blob), M, N, K, _ptr(Y), _ptr(workspace), ws_bytes, _stream(A.device)),
            "w4lut_gemm")
+    return Y
+
+
+def lut3_packed_bytes(N: int, K: int, group: int = 128) -> int:
+    return int(lib().w4lut3_packed_bytes(N, K, group))
+
+
+def lut3_pack_weights(q, s, table, group: int = 128):
+    """3-bit indices q uint8 [N, K] (0..7), scales s fp16 [N, K/128], table fp16 [8] -> blob."""
+    torch = _torch()
+    _require_cuda(q, s, table)
+    N, K = q.shape
+    nbytes = lut3_packed_bytes(N, K, group)
+    if nbytes == 0:
+        raise W4A8Error(f"unsupported weight shape {N}x{K} (group {group})")
+    blob = torch.empty((nbytes,), dtype=torch.uint8, device=q.device)
+    _check(lib().w4lut3_pack_weights(_ptr(q), _ptr(s), _ptr(table), N, K, group, _ptr(blob), nbytes,
+                                     _stream(q.device)), "w4lut3_pack_weights")
+    return blob
+
+
+def lut3_gemm_ex(A, blob, N: int, K: int, Y=None, acc=None, workspace=None, schedule=0, block_m=0, max_ctas=0):
+    """3-bit lookup-table GEMM (as lut_gemm_ex)."""
+    torch = _torch()
+    _require_cuda(A, blob, Y, acc, workspace)
+    if A.dtype != torch.float16 or A.dim() != 2 or A.shape[1] != K:
+        raise W4A8Error("A must be fp16 [M, K]")
+    M = A.shape[0]
+    if workspace is None:
+        workspace = _workspace_for(A.device, M, N, K)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    o = ctypes.byref(GemmOpts(schedule, block_m, max_ctas, 0))
+    _check(lib().w4lut3_gemm_ex(_ptr(A), _ptr(blob), M, N, K, _ptr(Y), _ptr(acc), _ptr(workspace), ws_bytes, o,
+                                _stream(A.device)), "w4lut3_gemm_ex")
+    return Y if Y is not None else acc
+
+
+def lut3_gemm(A, blob, N: int, K: int, out=None, workspace=None):
+    """Y fp16 [M, N] = fp16(sum_k A[m,k] * fp16(T[q[n,k]] * s[n,k/128])), 3-bit q."""
+    torch = _torch()
+    _require_cuda(A, blob, out, workspace)
+    if A.dtype != torch.float16 or A.dim() != 2 or A.shape[1] != K:
+        raise W4A8Error("A must be fp16 [M, K]")
+    M = A.shape[0]
+    Y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=A.device)
+    if workspace is None:
+        workspace = _workspace_for(A.device, M, N, K)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().w4lut3_gemm(_ptr(A), _ptr(blob), M, N, K, _ptr(Y), _ptr(workspace), ws_bytes, _stream(A.device)),
+           "w4lut3_gemm")
     return Y
 
 

@@ -131,17 +131,27 @@ struct Sched {
 // Lookup-table weight tiles (weight-only GEMM, "Fast Matrix Multiplications
 // for Lookup Table-Quantized LLMs"): 8192 index bytes + 128 fp16 row scales.
 constexpr int kLutTileBytes = kTileCodeBytes + 2 * kTileN;  // 8448
+// 3-bit lookup-table tiles: per row three 16-byte bit planes (plane c holds
+// bit c of the row's 128 indices), plane c of row r at (c * 128 + r) * 16,
+// then the 128 fp16 row scales.
+constexpr int kLut3CodeBytes = 3 * 16 * kTileN;             // 6144
+constexpr int kLut3TileBytes = kLut3CodeBytes + 2 * kTileN;  // 6400
 
-template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_, int NMMA_, bool LUT_ = false>
+template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_, int NMMA_, int LUT_ = 0>
 struct GemmCfg {
   static constexpr int BN = BN_, KS = KS_, NS = NS_, NT = NT_, DQ = DQ_, NACC = NACC_, NMMA = NMMA_;
-  // LUT: lookup-table weights against fp16 activations (kind::f16 MMA, fp32
-  // accumulators); otherwise two-level 4-bit weights against int8 (kind::i8)
-  static constexpr bool kLut = LUT_;
-  static constexpr int kTileB = kLut ? kLutTileBytes : kTileBytes;  // packed bytes of one weight tile
+  // LUT_ != 0: lookup-table weights against fp16 activations (kind::f16 MMA,
+  // fp32 accumulators), 4-bit indices (1) or 3-bit indices in bit planes (3);
+  // otherwise two-level 4-bit weights against int8 (kind::i8)
+  static_assert(LUT_ == 0 || LUT_ == 1 || LUT_ == 3, "weight format");
+  static constexpr bool kLut = LUT_ != 0;
+  static constexpr bool kLut3 = LUT_ == 3;
+  static constexpr int kTileB = kLut ? (kLut3 ? kLut3TileBytes : kLutTileBytes) : kTileBytes;  // one weight tile
   static constexpr int kKbCols = kLut ? 64 : 32;                    // TMEM columns of one dequantized k-block
   static constexpr int kMmaPerKb = kLut ? 8 : 4;                    // MMAs per k-block (K = 16 / 32)
-  static constexpr int kLutTableBytes = kLut ? 256 * 32 * 4 : 0;    // pair table, one copy per lane
+  // pair table, one copy per lane: 256 entries (a byte of two 4-bit indices)
+  // or 64 (a 6-bit pair code assembled from the three planes)
+  static constexpr int kLutTableBytes = kLut ? (kLut3 ? 64 : 256) * 32 * 4 : 0;
   // One CTA per SM, persistent. Work moves in chunks of up to KS k-blocks of
   // one tile (one weight copy, one wait and one commit per chunk amortize the
   // fixed latencies of the synchronization operations).
@@ -285,6 +295,30 @@ __device__ __forceinline__ void lut_dequant_half(const uint8_t* wt, int r, int h
         const __half2 x = __hmul2(*reinterpret_cast<const __half2*>(&pair), ss);
         out[cc * 16 + jj * 4 + b] = *reinterpret_cast<const uint32_t*>(&x);
       }
+    }
+  }
+}
+
+// The same for a 3-bit tile: index pair (k, k + 1), k even, is looked up by
+// its 6-bit code f0 | f1 << 2 | f2 << 4, f_c = bits k, k + 1 of plane c (the
+// pair table is built in that order), so a half reads two 32-bit words of
+// each plane and needs no per-index bit gathering beyond the three fields.
+__device__ __forceinline__ void lut3_dequant_half(const uint8_t* wt, int r, int h, const uint32_t* lut, int lane,
+                                                  uint32_t (&out)[32]) {
+  const __half sc = *reinterpret_cast<const __half*>(wt + kLut3CodeBytes + 2 * r);
+  const __half2 ss = __halves2half2(sc, sc);
+  const uint2 p0 = *reinterpret_cast<const uint2*>(wt + (0 * kTileN + r) * 16 + 8 * h);
+  const uint2 p1 = *reinterpret_cast<const uint2*>(wt + (1 * kTileN + r) * 16 + 8 * h);
+  const uint2 p2 = *reinterpret_cast<const uint2*>(wt + (2 * kTileN + r) * 16 + 8 * h);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const uint32_t a = j ? p0.y : p0.x, b = j ? p1.y : p1.x, c = j ? p2.y : p2.x;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const uint32_t e = ((a >> (2 * i)) & 3u) | (((b >> (2 * i)) & 3u) << 2) | (((c >> (2 * i)) & 3u) << 4);
+      const uint32_t pair = lut[e * 32 + lane];
+      const __half2 x = __hmul2(*reinterpret_cast<const __half2*>(&pair), ss);
+      out[j * 16 + i] = *reinterpret_cast<const uint32_t*>(&x);
     }
   }
 }
@@ -843,7 +877,18 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
     fence_barrier_init();
     fence_proxy_async_smem();
   }
-  if constexpr (C::kLut) {
+  if constexpr (C::kLut3) {
+    // pair table: entry e = (T[lo], T[hi]) as fp16x2 with the indices' bits
+    // c taken from bits 2c (lo) and 2c + 1 (hi) of e; one copy per lane
+    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::kOffLut);
+    const uint16_t* T = reinterpret_cast<const uint16_t*>(args.lut_table);
+    for (int i = threadIdx.x; i < 64 * 32; i += C::kThreads) {
+      const int e = i >> 5;
+      const int lo = (e & 1) | ((e >> 1) & 2) | ((e >> 2) & 4);
+      const int hi = ((e >> 1) & 1) | ((e >> 2) & 2) | ((e >> 3) & 4);
+      lut[i] = static_cast<uint32_t>(__ldg(T + lo)) | (static_cast<uint32_t>(__ldg(T + hi)) << 16);
+    }
+  } else if constexpr (C::kLut) {
     // pair table: entry e = (T[e & 15], T[e >> 4]) as fp16x2, one copy per lane
     uint32_t* lut = reinterpret_cast<uint32_t*>(smem + C::kOffLut);
     const uint16_t* T = reinterpret_cast<const uint16_t*>(args.lut_table);
@@ -1031,7 +1076,11 @@ __global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_
             const uint32_t* lut = reinterpret_cast<const uint32_t*>(smem + C::kOffLut);
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              lut_dequant_half(sW + w * C::kWSlot + j * C::kTileB, r, h, lut, lane, out);
+              if constexpr (C::kLut3) {
+                lut3_dequant_half(sW + w * C::kWSlot + j * C::kTileB, r, h, lut, lane, out);
+              } else {
+                lut_dequant_half(sW + w * C::kWSlot + j * C::kTileB, r, h, lut, lane, out);
+              }
               if (C::kPipelinedStores && j == 0 && h == 0 && prev_t >= 0) {
                 tmem_wait_st();
                 tc_fence_before();

@@ -166,4 +166,75 @@ __global__ void lut_pack_meta_kernel(const __half* __restrict__ s, const __half*
   }
 }
 
+
+// ------------------------------------------------ 3-bit lookup-table blob
+// Tiles of 6400 bytes: per row three 16-byte bit planes (plane c = bit c of
+// the row's 128 indices, bit kk of the plane = bit kk % 8 of byte kk / 8),
+// plane c of row r at (c * 128 + r) * 16, then the 128 fp16 row scales; after
+// the tiles the 8 fp16 table entries, zero padded to 64 bytes.
+constexpr uint32_t kLut3Magic = 0x544C3357u;  // "W3LT"
+constexpr int kLut3CodeBytesPack = 3 * 16 * kTileN;                 // 6144
+constexpr int kLut3TileBytesPack = kLut3CodeBytesPack + 2 * kTileN;  // 6400
+
+// One warp per (row n, tile column kt): lane l reads the index of in-tile
+// k = 32w + l (w = 0..3), and a ballot of bit c gives word w of plane c.
+__global__ void lut3_pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K,
+                                       uint8_t* __restrict__ tiles) {
+  const int64_t KT = K >> 7;
+  const int64_t total = N * KT;
+  const int lane = threadIdx.x & 31;
+  const int64_t wpb = blockDim.x >> 5;
+  for (int64_t i = blockIdx.x * wpb + (threadIdx.x >> 5); i < total; i += static_cast<int64_t>(gridDim.x) * wpb) {
+    const int64_t n = i / KT, kt = i - n * KT;
+    uint32_t w0[4], w1[4], w2[4];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+      const uint32_t v = q[n * K + kt * 128 + 32 * w + lane];
+      w0[w] = __ballot_sync(0xffffffffu, (v & 1u) != 0);
+      w1[w] = __ballot_sync(0xffffffffu, (v & 2u) != 0);
+      w2[w] = __ballot_sync(0xffffffffu, (v & 4u) != 0);
+    }
+    uint8_t* tile = tiles + (n >> 7) * KT * kLut3TileBytesPack + kt * kLut3TileBytesPack;
+    const int64_t r = n & 127;
+    if (lane == 0) *reinterpret_cast<uint4*>(tile + (0 * kTileN + r) * 16) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+    if (lane == 1) *reinterpret_cast<uint4*>(tile + (1 * kTileN + r) * 16) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+    if (lane == 2) *reinterpret_cast<uint4*>(tile + (2 * kTileN + r) * 16) = make_uint4(w2[0], w2[1], w2[2], w2[3]);
+  }
+}
+
+// Row scales into their tiles, the table after the tiles, and the header.
+__global__ void lut3_pack_meta_kernel(const __half* __restrict__ s, const __half* __restrict__ table, int64_t N,
+                                      int64_t K, uint8_t* __restrict__ blob, int64_t table_offset) {
+  const int64_t G = K >> 7;
+  const int64_t total = N * G;
+  uint8_t* tiles = blob + kHeaderBytes;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = i / G, g = i - n * G;
+    *reinterpret_cast<__half*>(tiles + ((n >> 7) * G + g) * kLut3TileBytesPack + kLut3CodeBytesPack + 2 * (n & 127)) =
+        s[i];
+  }
+  if (blockIdx.x == 0 && threadIdx.x < 32) {
+    __half* t = reinterpret_cast<__half*>(blob + table_offset);
+    t[threadIdx.x] = threadIdx.x < 8 ? table[threadIdx.x] : __ushort_as_half(0);
+  }
+  if (blockIdx.x == 0 && threadIdx.x < kHeaderBytes / 4) {
+    uint32_t w = 0;
+    switch (threadIdx.x) {
+      case 0: w = kLut3Magic; break;
+      case 1: w = kLayoutVersion; break;
+      case 2: w = static_cast<uint32_t>(N); break;
+      case 3: w = static_cast<uint32_t>(static_cast<uint64_t>(N) >> 32); break;
+      case 4: w = static_cast<uint32_t>(K); break;
+      case 5: w = static_cast<uint32_t>(static_cast<uint64_t>(K) >> 32); break;
+      case 6: w = 128u; break;
+      case 7: w = static_cast<uint32_t>(kLut3TileBytesPack); break;
+      case 8: w = static_cast<uint32_t>(table_offset); break;
+      case 9: w = static_cast<uint32_t>(static_cast<uint64_t>(table_offset) >> 32); break;
+      default: w = 0; break;
+    }
+    reinterpret_cast<uint32_t*>(blob)[threadIdx.x] = w;
+  }
+}
+
 }  // namespace w4a8

@@ -109,6 +109,9 @@ int64_t packed_s1_offset(int64_t N, int64_t K) { return kHeaderBytes + (N / kTil
 int64_t lut_table_offset(int64_t N, int64_t K) {
   return kHeaderBytes + (N / kTileN) * (K / kTileK) * kLutTileBytesPack;
 }
+int64_t lut3_table_offset(int64_t N, int64_t K) {
+  return kHeaderBytes + (N / kTileN) * (K / kTileK) * kLut3TileBytesPack;
+}
 
 // ------------------------------------------------------------------ GEMM
 // Resident CTAs per SM of a configuration (shared memory, threads and tensor
@@ -211,8 +214,11 @@ using Cfg64 = GemmCfg<64, 2, 6, 6, 2, 2, 2>;
 // lookup-table weights against fp16 activations (decode tile sizes; larger M
 // uses several 32-token tiles): one k-block per chunk and a third
 // dequantizer group (the table lookups, not the weight bytes, limit it)
-using CfgL16 = GemmCfg<16, 1, 12, 6, 3, 2, 2, true>;
-using CfgL32 = GemmCfg<32, 1, 6, 6, 3, 2, 2, true>;
+using CfgL16 = GemmCfg<16, 1, 12, 6, 3, 2, 2, 1>;
+using CfgL32 = GemmCfg<32, 1, 6, 6, 3, 2, 2, 1>;
+// the same with 3-bit indices in bit planes
+using CfgL3_16 = GemmCfg<16, 1, 12, 6, 3, 2, 2, 3>;
+using CfgL3_32 = GemmCfg<32, 1, 6, 6, 3, 2, 2, 3>;
 using Cfg128 = GemmCfg<128, 4, 2, 2, 1, 2, 2>;
 
 size_t ws_counter_bytes(int64_t M, int64_t N) {
@@ -310,7 +316,9 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   int dev_id = 0;
   cudaGetDevice(&dev_id);
   int per_sm = 1;
-  if (lut) {
+  if (lut == 3) {
+    st = bn == 16 ? ctas_per_sm<CfgL3_16>(dev_id, &per_sm) : ctas_per_sm<CfgL3_32>(dev_id, &per_sm);
+  } else if (lut) {
     st = bn == 16 ? ctas_per_sm<CfgL16>(dev_id, &per_sm) : ctas_per_sm<CfgL32>(dev_id, &per_sm);
   } else {
     switch (bn) {
@@ -332,7 +340,9 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
     for (int S = 4; S >= 2 && split == 1; --S) {
       if (S > KB) continue;
       int nclu = 0;
-      if (lut) {
+      if (lut == 3) {
+        st = bn == 16 ? max_clusters<CfgL3_16>(dev_id, S, &nclu) : max_clusters<CfgL3_32>(dev_id, S, &nclu);
+      } else if (lut) {
         st = bn == 16 ? max_clusters<CfgL16>(dev_id, S, &nclu) : max_clusters<CfgL32>(dev_id, S, &nclu);
       } else {
         st = bn == 16 ? max_clusters<Cfg16>(dev_id, S, &nclu) : max_clusters<Cfg32>(dev_id, S, &nclu);
@@ -392,8 +402,9 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   GemmArgs a;
   a.tiles = static_cast<const uint8_t*>(packed) + kHeaderBytes;
   a.s1 = lut ? nullptr : reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + packed_s1_offset(N, K));
-  a.lut_table = lut ? reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + lut_table_offset(N, K))
-                    : nullptr;
+  a.lut_table = lut == 3 ? reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + lut3_table_offset(N, K))
+                : lut ? reinterpret_cast<const __half*>(static_cast<const uint8_t*>(packed) + lut_table_offset(N, K))
+                      : nullptr;
   a.sA = static_cast<const __half*>(sA);
   a.rowsum = rowsum;
   a.Y = static_cast<__half*>(Y);
@@ -412,6 +423,9 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   if (lut) {
     a.sA = nullptr;
     a.rowsum = nullptr;
+    if (lut == 3)
+      return bn == 16 ? launch_gemm_cfg<CfgL3_16>(A8, M, K, a, grid, stream)
+                      : launch_gemm_cfg<CfgL3_32>(A8, M, K, a, grid, stream);
     return bn == 16 ? launch_gemm_cfg<CfgL16>(A8, M, K, a, grid, stream)
                     : launch_gemm_cfg<CfgL32>(A8, M, K, a, grid, stream);
   }
@@ -646,6 +660,46 @@ w4a8_status_t w4lut_gemm_ex(const void* A, const void* packed, int64_t M, int64_
                             w4a8_stream_t stream) {
   return gemm_impl(A, nullptr, nullptr, packed, M, N, K, Y, reinterpret_cast<int32_t*>(acc), workspace,
                    workspace_bytes, opts, reinterpret_cast<cudaStream_t>(stream), 0, 1);
+}
+
+size_t w4lut3_packed_bytes(int64_t N, int64_t K, int32_t group) {
+  if (group != 128 || N <= 0 || K <= 0 || N % 128 != 0 || K % 128 != 0 || K > kMaxK) return 0;
+  return static_cast<size_t>(lut3_table_offset(N, K) + 64);
+}
+
+w4a8_status_t w4lut3_pack_weights(const uint8_t* q, const void* s, const void* table, int64_t N, int64_t K,
+                                  int32_t group, void* packed, size_t packed_bytes, w4a8_stream_t stream) {
+  if (N < 0 || K < 0) return W4A8_ERR_INVALID_ARG;
+  if (group != 128 || N == 0 || K == 0 || N % 128 != 0 || K % 128 != 0 || K > kMaxK)
+    return W4A8_ERR_UNSUPPORTED_SHAPE;
+  if (q == nullptr || s == nullptr || table == nullptr || packed == nullptr) return W4A8_ERR_INVALID_ARG;
+  if (!aligned(s, 2) || !aligned(table, 2) || !aligned(packed, 16)) return W4A8_ERR_MISALIGNED;
+  if (packed_bytes < w4lut3_packed_bytes(N, K, group)) return W4A8_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* blob = static_cast<uint8_t*>(packed);
+  const int64_t warps = N * (K / 128);
+  const int64_t blocks1 = (warps + 7) / 8;
+  lut3_pack_codes_kernel<<<static_cast<int>(blocks1 < 65535 * 16 ? blocks1 : 65535 * 16), 256, 0, st>>>(
+      q, N, K, blob + kHeaderBytes);
+  if (cudaPeekAtLastError() != cudaSuccess) return launch_status();
+  const int64_t metas = N * (K / 128);
+  const int64_t blocks2 = (metas + 255) / 256;
+  lut3_pack_meta_kernel<<<static_cast<int>(blocks2 < 65535 ? blocks2 : 65535), 256, 0, st>>>(
+      static_cast<const __half*>(s), static_cast<const __half*>(table), N, K, blob, lut3_table_offset(N, K));
+  return launch_status();
+}
+
+w4a8_status_t w4lut3_gemm(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
+                          void* workspace, size_t workspace_bytes, w4a8_stream_t stream) {
+  return gemm_impl(A, nullptr, nullptr, packed, M, N, K, Y, nullptr, workspace, workspace_bytes, nullptr,
+                   reinterpret_cast<cudaStream_t>(stream), 0, 3);
+}
+
+w4a8_status_t w4lut3_gemm_ex(const void* A, const void* packed, int64_t M, int64_t N, int64_t K, void* Y,
+                             float* acc, void* workspace, size_t workspace_bytes, const w4a8_gemm_opts_t* opts,
+                             w4a8_stream_t stream) {
+  return gemm_impl(A, nullptr, nullptr, packed, M, N, K, Y, reinterpret_cast<int32_t*>(acc), workspace,
+                   workspace_bytes, opts, reinterpret_cast<cudaStream_t>(stream), 0, 3);
 }
 
 w4a8_status_t w4a8_get_device_error(w4a8_stream_t stream, int32_t* code) {
