@@ -14,12 +14,15 @@
 // Decode attention: for sequence b (cache length L_b), query head h and its
 // kv head g = h / (Hq / Hkv): s_j = scale * (s_j^K * sum_d q[d] (code - z)),
 // o = sum_j softmax(s)_j (code^V_j - z^V_j) s^V_j, Y = fp16_rn(o). The cache is
-// read once (HBM-bound for grouped queries on the workloads' sizes): a CTA
-// takes up to kKvChunk tokens of one (sequence, kv head) for up to four of its
-// query heads, scores them, exponentiates against the chunk's own maximum
-// and accumulates the weighted values; the last CTA of a (sequence, kv head,
-// head group) to finish (a ticket in the workspace, no waiting) merges the
-// chunks' partial results with exp(m_chunk - m) factors and writes Y.
+// read once per four query heads: a CTA takes up to kKvChunk tokens of one
+// (sequence, kv head) for up to four of its query heads, scores them,
+// exponentiates against the chunk's own maximum and accumulates the weighted
+// values; the last CTA of a (sequence, kv head, head group) to finish (a
+// ticket in the workspace, no waiting) merges the chunks' partial results
+// with exp(m_chunk - m) factors and writes Y. The scores and the weighted
+// sums run on CUDA cores in fp32, about 14 operations per cache byte for four
+// query heads per kv head, so at that grouping the arithmetic, not HBM, is
+// expected to set the pace.
 //
 // Mapping inside a CTA (both phases): 8 lanes per token, lane slice li owns
 // elements [16 li, 16 li + 16) (8 code bytes, one 8-byte load), so a warp
