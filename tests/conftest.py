@@ -8,5 +8,3 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
-    config.addinivalue_line("markers", "gpu_pending: GPU parity of a kernel not yet run on a B200 "
-                                       "(selected explicitly with -m gpu_pending; becomes gpu once it passes)")

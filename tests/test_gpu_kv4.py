@@ -16,7 +16,7 @@ import w4a8_quantized_gemm_quantize_b200 as w4a8
 from w4a8_quantized_gemm_quantize_b200 import inputs as I
 from oracle import kv4_oracle as KV
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)

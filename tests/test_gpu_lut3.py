@@ -5,8 +5,7 @@ the CPU oracle, through the C ABI.
 Bars as for the 4-bit table: the blob byte-exact; one-hot activation rows
 reproduce the dequantized weights bit for bit; general activations within
 the fp32 accumulation bound, Y within half an fp16 ulp plus it; every
-schedule and both token-tile sizes. Marked gpu_pending until the kernel
-path has run on a B200.
+schedule and both token-tile sizes.
 """
 import numpy as np
 import pytest
@@ -17,7 +16,7 @@ import w4a8_quantized_gemm_quantize_b200 as w4a8
 from w4a8_quantized_gemm_quantize_b200 import inputs as I
 from oracle import w4a8_oracle as O
 
-pytestmark = pytest.mark.gpu_pending
+pytestmark = pytest.mark.gpu
 
 if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
