@@ -280,13 +280,11 @@ w4a8_status_t check_quantize_args(const void* A, int64_t M, int64_t K, const voi
 
 }  // namespace
 
-// A8: the int8 activation codes [M, K], or with a4 the packed 4-bit codes
-// [M, K / 2] (W4A4).
-w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
-                        int64_t N, int64_t K, void* Y, int32_t* acc, void* ws, size_t ws_bytes,
-                        const w4a8_gemm_opts_t* opts, cudaStream_t stream, int a4 = 0, int lut = 0) {
-  w4a8_gemm_opts_t o = {0, 0, 0, 0};
-  if (opts != nullptr) o = *opts;
+// Host-side checks shared by every GEMM entry point: options, shape limits,
+// pointers and alignment. W4A8_OK with M == 0 or N == 0 means "nothing to do".
+w4a8_status_t check_gemm_args(const void* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+                              int64_t N, int64_t K, const void* Y, const int32_t* acc, const void* ws,
+                              const w4a8_gemm_opts_t& o, int lut) {
   if (o.reserved != 0 || o.schedule < 0 || o.schedule > 3 || o.max_ctas < 0) return W4A8_ERR_INVALID_ARG;
   if (!(o.block_m == 0 || o.block_m == 16 || o.block_m == 32 || o.block_m == 64 || o.block_m == 128))
     return W4A8_ERR_INVALID_ARG;
@@ -301,6 +299,20 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   if (!aligned(A8, 16) || !aligned(packed, 16) || !aligned(Y, 16) || !aligned(acc, 16) || !aligned(sA, 2) ||
       !aligned(rowsum, 4) || !aligned(ws, 256))
     return W4A8_ERR_MISALIGNED;
+  return W4A8_OK;
+}
+
+// A8: the int8 activation codes [M, K], or with a4 the packed 4-bit codes
+// [M, K / 2] (W4A4).
+w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, const void* packed, int64_t M,
+                        int64_t N, int64_t K, void* Y, int32_t* acc, void* ws, size_t ws_bytes,
+                        const w4a8_gemm_opts_t* opts, cudaStream_t stream, int a4 = 0, int lut = 0) {
+  w4a8_gemm_opts_t o = {0, 0, 0, 0};
+  if (opts != nullptr) o = *opts;
+  {
+    const w4a8_status_t v = check_gemm_args(A8, sA, rowsum, packed, M, N, K, Y, acc, ws, o, lut);
+    if (v != W4A8_OK || M == 0 || N == 0) return v;
+  }
   DeviceInfo* dev = nullptr;
   w4a8_status_t st = device_info(&dev);
   if (st != W4A8_OK) return st;
@@ -563,17 +575,19 @@ w4a8_status_t w4a8_pack_weights(const uint8_t* q, const uint8_t* z, const uint8_
     return W4A8_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(s1, 2) || !aligned(packed, 16)) return W4A8_ERR_MISALIGNED;
   if (packed_bytes < w4a8_packed_bytes(N, K, group)) return W4A8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if (const w4a8_status_t e = device_info(&dev); e != W4A8_OK) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* blob = static_cast<uint8_t*>(packed);
   const int64_t chunks = N * (K / 32);
   const int64_t blocks1 = (chunks + 255) / 256;
   pack_codes_kernel<<<static_cast<int>(blocks1 < 65535 * 16 ? blocks1 : 65535 * 16), 256, 0, st>>>(
-      q, N, K, blob + kHeaderBytes);
+      q, N, K, blob + kHeaderBytes, dev->err);
   if (cudaPeekAtLastError() != cudaSuccess) return launch_status();
   const int64_t metas = N * (K / 128);
   const int64_t blocks2 = (metas + 255) / 256;
   pack_meta_kernel<<<static_cast<int>(blocks2 < 65535 ? blocks2 : 65535), 256, 0, st>>>(
-      z, s2, static_cast<const __half*>(s1), N, K, blob, packed_s1_offset(N, K));
+      z, s2, static_cast<const __half*>(s1), N, K, blob, packed_s1_offset(N, K), dev->err);
   return launch_status();
 }
 
@@ -635,12 +649,14 @@ w4a8_status_t w4lut_pack_weights(const uint8_t* q, const void* s, const void* ta
   if (q == nullptr || s == nullptr || table == nullptr || packed == nullptr) return W4A8_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(s, 2) || !aligned(table, 2) || !aligned(packed, 16)) return W4A8_ERR_MISALIGNED;
   if (packed_bytes < w4lut_packed_bytes(N, K, group)) return W4A8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if (const w4a8_status_t e = device_info(&dev); e != W4A8_OK) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* blob = static_cast<uint8_t*>(packed);
   const int64_t chunks = N * (K / 32);
   const int64_t blocks1 = (chunks + 255) / 256;
   lut_pack_codes_kernel<<<static_cast<int>(blocks1 < 65535 * 16 ? blocks1 : 65535 * 16), 256, 0, st>>>(
-      q, N, K, blob + kHeaderBytes);
+      q, N, K, blob + kHeaderBytes, dev->err);
   if (cudaPeekAtLastError() != cudaSuccess) return launch_status();
   const int64_t metas = N * (K / 128);
   const int64_t blocks2 = (metas + 255) / 256;
@@ -675,12 +691,14 @@ w4a8_status_t w4lut3_pack_weights(const uint8_t* q, const void* s, const void* t
   if (q == nullptr || s == nullptr || table == nullptr || packed == nullptr) return W4A8_ERR_INVALID_ARG;
   if (!aligned(s, 2) || !aligned(table, 2) || !aligned(packed, 16)) return W4A8_ERR_MISALIGNED;
   if (packed_bytes < w4lut3_packed_bytes(N, K, group)) return W4A8_ERR_INVALID_ARG;
+  DeviceInfo* dev = nullptr;
+  if (const w4a8_status_t e = device_info(&dev); e != W4A8_OK) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* blob = static_cast<uint8_t*>(packed);
   const int64_t warps = N * (K / 128);
   const int64_t blocks1 = (warps + 7) / 8;
   lut3_pack_codes_kernel<<<static_cast<int>(blocks1 < 65535 * 16 ? blocks1 : 65535 * 16), 256, 0, st>>>(
-      q, N, K, blob + kHeaderBytes);
+      q, N, K, blob + kHeaderBytes, dev->err);
   if (cudaPeekAtLastError() != cudaSuccess) return launch_status();
   const int64_t metas = N * (K / 128);
   const int64_t blocks2 = (metas + 255) / 256;
@@ -743,7 +761,11 @@ static std::mutex g_noalloc_mu;
 w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed,
                                 int64_t M, int64_t N, int64_t K, void* Y, w4a8_stream_t stream) {
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (M <= 0 || N <= 0) return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, nullptr, nullptr, 0, nullptr, st);
+  // every argument check comes before the scratch is touched: a rejected
+  // call must not clear the array under an earlier call still running on it
+  const w4a8_gemm_opts_t o = {0, 0, 0, 0};
+  const w4a8_status_t v = check_gemm_args(A8, sA, rowsum, packed, M, N, K, Y, nullptr, nullptr, o, 0);
+  if (v != W4A8_OK || M == 0 || N == 0) return v;
   const size_t need = w4a8_gemm_workspace_bytes(M, N, K);
   if (need > W4A8_NOALLOC_SCRATCH_BYTES) return W4A8_ERR_WORKSPACE;
   int dev = 0;
