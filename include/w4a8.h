@@ -74,6 +74,7 @@ typedef enum {
 #define W4A8_DEVERR_DRAIN_WAIT 5
 #define W4A8_DEVERR_SELFTEST_WAIT 6
 #define W4A8_DEVERR_KV_RANGE 7 /* a KV-cache length or position outside [0, Lmax] (clamped or skipped) */
+#define W4A8_DEVERR_PACK_RANGE 8 /* a packer met a code, zero point or scale outside its documented range */
 
 /* Human-readable name of a status code (static string, never NULL). */
 W4A8_API const char* w4a8_status_string(int status);
@@ -148,7 +149,10 @@ W4A8_API size_t w4a8_packed_bytes(int64_t N, int64_t K, int32_t group);
  *     (high nibble); word j of row r is word ((j/4)*128 + r)*4 + j%4 of the
  *     tile. Meta byte r = z | ((s2 - 1) << 4) of group kt.
  *   s1: N fp16 values, zero padded to a multiple of 16 bytes.
- * q/z/s2/s1 as produced by w4a8_quantize_weights (q and s1 16-byte aligned).
+ * q/z/s2/s1 as produced by w4a8_quantize_weights (q and s1 16-byte aligned):
+ * q and z in [0, 15], s2 in [1, 8]. A value outside its range is reported as
+ * W4A8_DEVERR_PACK_RANGE in the device error word (its field keeps only the
+ * low bits, so the blob is then wrong).
  * packed: packed_bytes >= w4a8_packed_bytes(N, K, group).
  * Limits: group == 128, N % 128 == 0, K % 128 == 0, 0 < K <= 65536.
  */
@@ -306,7 +310,8 @@ W4A8_API size_t w4lut_packed_bytes(int64_t N, int64_t K, int32_t group);
 /*
  * Packs q (uint8 [N, K], one index 0..15 per byte, 16-byte aligned), s (fp16
  * [N, K/128], 2-byte aligned) and table (16 fp16 values, 2-byte aligned) into
- * the blob above. Limits: group == 128, N % 128 == 0, K % 128 == 0,
+ * the blob above. An index above 15 is reported as W4A8_DEVERR_PACK_RANGE in
+ * the device error word (only its low 4 bits are packed). Limits: group == 128, N % 128 == 0, K % 128 == 0,
  * 0 < K <= 65536; packed_bytes >= w4lut_packed_bytes(N, K, group).
  */
 W4A8_API w4a8_status_t w4lut_pack_weights(const uint8_t* q, const void* s, const void* table, int64_t N, int64_t K,
@@ -340,7 +345,9 @@ W4A8_API w4a8_status_t w4lut_gemm_ex(const void* A, const void* packed, int64_t 
  * the index at in-tile k = kk) at (c * 128 + r) * 16; then the 128 fp16 row
  * scales (row r at 6144 + 2r); after the tiles the 8 fp16 table entries,
  * zero padded to 64 bytes. Entry points as for the 4-bit table (q holds one
- * index 0..7 per byte; table holds 8 fp16 values).
+ * index 0..7 per byte; table holds 8 fp16 values). An index above 7 is
+ * reported as W4A8_DEVERR_PACK_RANGE in the device error word (only its low
+ * 3 bits are packed, which selects a different table entry).
  */
 W4A8_API size_t w4lut3_packed_bytes(int64_t N, int64_t K, int32_t group);
 W4A8_API w4a8_status_t w4lut3_pack_weights(const uint8_t* q, const void* s, const void* table, int64_t N, int64_t K,

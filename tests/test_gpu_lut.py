@@ -54,6 +54,19 @@ def test_lut_pack_byte_exact(N, K):
     assert (host(b) == O.lut_pack_weights(q, s, T)).all()
 
 
+def test_lut_pack_reports_indices_above_15():
+    N, K = 128, 256
+    q, s = I.lut_codes(N, K, I.seed_of("t-lr", N, K))
+    bad = q.copy()
+    bad[9, 17] = 16
+    w4a8.clear_device_error(DEV)
+    blob_of(bad, s)
+    assert w4a8.get_device_error(DEV) == w4a8.DEVERR_PACK_RANGE
+    w4a8.clear_device_error(DEV)
+    blob_of(q, s)
+    assert w4a8.get_device_error(DEV) == 0
+
+
 SCHEDULES = ([(0, 0, 0), (0, 16, 5), (0, 32, 3)] + [(s, bm, c) for s in (1, 2) for bm in (16, 32) for c in (0, 7)] +
              [(3, 16, 0), (3, 32, 0)])
 

@@ -52,6 +52,21 @@ def test_lut3_pack_byte_exact(N, K):
     assert (host(b) == O.lut3_pack_weights(q, s, T)).all()
 
 
+def test_lut3_pack_reports_indices_above_7():
+    """Only bits 0-2 of an index are packed: an index of 8..15 (a 4-bit index
+    given to the 3-bit packer) is reported through the device error word."""
+    N, K = 128, 256
+    q, s = I.lut3_codes(N, K, I.seed_of("t-l3r", N, K))
+    bad = q.copy()
+    bad[7, 100] = 8
+    w4a8.clear_device_error(DEV)
+    blob_of(bad, s)
+    assert w4a8.get_device_error(DEV) == w4a8.DEVERR_PACK_RANGE
+    w4a8.clear_device_error(DEV)
+    blob_of(q, s)
+    assert w4a8.get_device_error(DEV) == 0
+
+
 SCHEDULES = ([(0, 0, 0), (0, 16, 5), (0, 32, 3)] + [(s, bm, c) for s in (1, 2) for bm in (16, 32) for c in (0, 7)] +
              [(3, 16, 0), (3, 32, 0)])
 

@@ -513,6 +513,8 @@ def clear_device_error(device=None):
 
 
 DEVERR_SELFTEST_WAIT = 6
+DEVERR_KV_RANGE = 7
+DEVERR_PACK_RANGE = 8
 
 
 def selftest_bounded_wait(limit_ns: int, device=None):

@@ -26,10 +26,13 @@ constexpr int kTileBytes = kTileCodeBytes + kTileN;  // 8320
 constexpr int kHeaderBytes = 64;
 constexpr uint32_t kMagic = 0x38413457u;  // "W4A8"
 constexpr uint32_t kLayoutVersion = 1u;
+// Device error code (W4A8_DEVERR_PACK_RANGE): a code or parameter outside its
+// documented range reached a packer; the packed field keeps only its low bits.
+constexpr int kErrPackRange = 8;
 
 // One thread per (row n, 32-k chunk): 32 codes in, one 16-byte vector out.
 __global__ void pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K,
-                                  uint8_t* __restrict__ tiles) {
+                                  uint8_t* __restrict__ tiles, int* err) {
   const int64_t KC = K >> 5;  // 32-k chunks per row
   const int64_t total = N * KC;
   const int64_t KT = K >> 7;
@@ -40,6 +43,7 @@ __global__ void pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int6
     const uint4* src = reinterpret_cast<const uint4*>(q + n * K + kc * 32);
     const uint4 a = src[0], b = src[1];
     const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};  // 4 codes per word, k ascending
+    if (((a.x | a.y | a.z | a.w | b.x | b.y | b.z | b.w) & 0xF0F0F0F0u) != 0u) atomicCAS(err, 0, kErrPackRange);
     uint32_t out[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -55,13 +59,14 @@ __global__ void pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int6
 
 __global__ void pack_meta_kernel(const uint8_t* __restrict__ z, const uint8_t* __restrict__ s2,
                                  const __half* __restrict__ s1, int64_t N, int64_t K, uint8_t* __restrict__ blob,
-                                 int64_t s1_offset) {
+                                 int64_t s1_offset, int* err) {
   const int64_t G = K >> 7;
   const int64_t total = N * G;
   uint8_t* tiles = blob + kHeaderBytes;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t n = i / G, g = i - n * G;
+    if (z[i] > 15 || s2[i] < 1 || s2[i] > 8) atomicCAS(err, 0, kErrPackRange);
     const uint8_t meta = static_cast<uint8_t>((z[i] & 0x0F) | (((s2[i] - 1) & 0x0F) << 4));
     tiles[((n >> 7) * G + g) * kTileBytes + kTileCodeBytes + (n & 127)] = meta;
   }
@@ -105,7 +110,7 @@ constexpr int kLutTileBytesPack = kTileCodeBytes + 2 * kTileN;  // 8448
 
 // One thread per (row n, 32-k chunk): 32 indices in, one 16-byte vector out.
 __global__ void lut_pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K,
-                                      uint8_t* __restrict__ tiles) {
+                                      uint8_t* __restrict__ tiles, int* err) {
   const int64_t KC = K >> 5;
   const int64_t total = N * KC;
   const int64_t KT = K >> 7;
@@ -116,6 +121,7 @@ __global__ void lut_pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, 
     const uint4* src = reinterpret_cast<const uint4*>(q + n * K + kc * 32);
     const uint4 a = src[0], b = src[1];
     const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};  // 4 indices per word, k ascending
+    if (((a.x | a.y | a.z | a.w | b.x | b.y | b.z | b.w) & 0xF0F0F0F0u) != 0u) atomicCAS(err, 0, kErrPackRange);
     uint32_t out[4];
 #pragma unroll
     for (int jj = 0; jj < 4; ++jj) {
@@ -179,7 +185,7 @@ constexpr int kLut3TileBytesPack = kLut3CodeBytesPack + 2 * kTileN;  // 6400
 // One warp per (row n, tile column kt): lane l reads the index of in-tile
 // k = 32w + l (w = 0..3), and a ballot of bit c gives word w of plane c.
 __global__ void lut3_pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N, int64_t K,
-                                       uint8_t* __restrict__ tiles) {
+                                       uint8_t* __restrict__ tiles, int* err) {
   const int64_t KT = K >> 7;
   const int64_t total = N * KT;
   const int lane = threadIdx.x & 31;
@@ -190,6 +196,7 @@ __global__ void lut3_pack_codes_kernel(const uint8_t* __restrict__ q, int64_t N,
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
       const uint32_t v = q[n * K + kt * 128 + 32 * w + lane];
+      if (v > 7u) atomicCAS(err, 0, kErrPackRange);  // only bits 0-2 are packed
       w0[w] = __ballot_sync(0xffffffffu, (v & 1u) != 0);
       w1[w] = __ballot_sync(0xffffffffu, (v & 2u) != 0);
       w2[w] = __ballot_sync(0xffffffffu, (v & 4u) != 0);
