@@ -135,33 +135,83 @@ def test_pack_byte_exact(N, K):
     assert (host(blob) == ob).all()
 
 
+def test_pack_reports_codes_out_of_range():
+    """A code, zero point or scale outside its range is reported through the
+    device error word (the packers keep only the field's low bits)."""
+    N, K = 128, 256
+    q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-pack-range", N, K))
+    for field, bad in (("q", 16), ("z", 16), ("s2", 0), ("s2", 9)):
+        qq, zz, ss = q.copy(), z.copy(), s2.copy()
+        {"q": qq, "z": zz, "s2": ss}[field][3, 1] = bad
+        w4a8.clear_device_error(DEV)
+        w4a8.pack_weights(dev(qq), dev(zz), dev(ss), dev(s1))
+        assert w4a8.get_device_error(DEV) == w4a8.DEVERR_PACK_RANGE, (field, bad)
+    w4a8.clear_device_error(DEV)
+    w4a8.pack_weights(dev(q), dev(z), dev(s2), dev(s1))
+    assert w4a8.get_device_error(DEV) == 0
+
+
 # ----------------------------------------------------------------- GEMM
 def gpu_path_from_codes(q, z, s2, s1):
     return w4a8.pack_weights(dev(q), dev(z), dev(s2), dev(s1))
 
 
+GUARD = 4096  # bytes of canary before and after every output buffer
+CANARY = 0xA5
+
+
+class Guarded:
+    """A contiguous tensor with canary bytes on both sides (stand-in for a
+    memory checker): a write past its first or last element changes them."""
+
+    def __init__(self, shape, dtype):
+        n = int(np.prod(shape)) * torch.empty((), dtype=dtype).element_size()
+        self.raw = torch.full((GUARD + n + GUARD,), CANARY, dtype=torch.uint8, device=DEV)
+        self.t = self.raw[GUARD:GUARD + n].view(dtype).view(shape)
+
+    def intact(self):
+        r = self.raw.cpu().numpy()
+        return bool((r[:GUARD] == CANARY).all() and (r[len(r) - GUARD:] == CANARY).all())
+
+
 def check_gemm(A, q, z, s2, s1, schedules=((0, 0, 0),)):
-    """A fp16 host, codes host; runs the GPU path from the same inputs."""
+    """A fp16 host, codes host; runs the GPU path from the same inputs. Every
+    buffer the library writes (codes, scales, rowsums, accumulators, Y, the
+    workspace) sits between canary regions that must survive each call."""
     M, K = A.shape
     N = q.shape[0]
     blob = gpu_path_from_codes(q, z, s2, s1)
-    A8, sA, rs = w4a8.quantize_act(dev(A))
+    gA8, gsA, grs = Guarded((M, K), torch.int8), Guarded((M,), torch.float16), Guarded((M,), torch.int32)
+    A8, sA, rs = w4a8.quantize_act(dev(A), out=(gA8.t, gsA.t, grs.t))
     oA8, osA, _ = O.quantize_act(A)
     oacc = O.gemm_acc(oA8, O.dequant_weights(q, z, s2))
     oY = O.epilogue(oacc, osA, s1)
-    ws = torch.zeros(w4a8.workspace_bytes(M, N, K), dtype=torch.uint8, device=DEV)
+    gws = Guarded((w4a8.workspace_bytes(M, N, K),), torch.uint8)
+    gws.t.zero_()
+    ws = gws.t
     for sched, bm, ctas in schedules:
-        acc = w4a8.gemm_ex(A8, None, rs, blob, N, K, acc=torch.empty((M, N), dtype=torch.int32, device=DEV),
-                           workspace=ws, schedule=sched, block_m=bm, max_ctas=ctas)
-        Y = w4a8.gemm_ex(A8, sA, rs, blob, N, K, Y=torch.empty((M, N), dtype=torch.float16, device=DEV),
-                         workspace=ws, schedule=sched, block_m=bm, max_ctas=ctas)
+        gacc, gY = Guarded((M, N), torch.int32), Guarded((M, N), torch.float16)
+        acc = w4a8.gemm_ex(A8, None, rs, blob, N, K, acc=gacc.t, workspace=ws, schedule=sched, block_m=bm,
+                           max_ctas=ctas)
+        Y = w4a8.gemm_ex(A8, sA, rs, blob, N, K, Y=gY.t, workspace=ws, schedule=sched, block_m=bm,
+                         max_ctas=ctas)
         torch.cuda.synchronize()
         ha = host(acc)
         bad = np.argwhere(ha != oacc)
         assert bad.size == 0, (sched, bm, ctas, bad[:5], ha[tuple(bad[0])], oacc[tuple(bad[0])])
         assert max_ulp_fp16(host(Y), oY) <= 1, (sched, bm, ctas)
         assert not host(ws).any(), "workspace must be left zero-filled"
+        assert gacc.intact() and gY.intact() and gws.intact(), ("write outside a buffer", sched, bm, ctas)
+    assert gA8.intact() and gsA.intact() and grs.intact(), "quantizer wrote outside its buffers"
     return oY
+
+
+def test_guard_regions_see_a_stray_write():
+    """The canary check itself: one byte written just past a buffer is seen."""
+    g = Guarded((3, 5), torch.float16)
+    assert g.intact()
+    g.raw[GUARD + 3 * 5 * 2] = 0
+    assert not g.intact()
 
 
 # (schedule, block_m, max_ctas); auto with a small grid mixes stream-K
@@ -275,20 +325,35 @@ def test_gemm_split_k_requires_workspace():
 
 
 # ------------------------------------------- full-size workload checks
+_W_CACHE = {}
+
+
+def _weights(workload, N, K):
+    """The seeded fp32 weights of one layer and their GPU blob (and codes),
+    kept for the next case of the same layer (cases are ordered by layer)."""
+    key = (workload, N, K)
+    if key not in _W_CACHE:
+        _W_CACHE.clear()
+        torch.cuda.empty_cache()
+        wl = I.WORKLOADS[workload]
+        W = I.dense_weights(N, K, wl.weight_std, I.weight_seed(workload, N, K))
+        Wd = dev(W)
+        q, z, s2, s1 = w4a8.quantize_weights(Wd)
+        del Wd
+        blob = w4a8.pack_weights(q, z, s2, s1)
+        _W_CACHE[key] = (W, q, z, s2, s1, blob)
+    return _W_CACHE[key]
+
+
 def _full_size_case(workload, lin, M, n_random_cols=64):
     """Runs the GPU path end to end from the seeded fp32 weights and fp16
     activations at full size (the launch configuration the benchmark uses)
     and compares every token against the oracle on sampled output channels:
     two whole 128-channel tiles plus random channels. The oracle quantizes
     only the weight rows it needs (rows are independent)."""
-    wl = I.WORKLOADS[workload]
     name, N, K = lin
-    W = I.dense_weights(N, K, wl.weight_std, I.weight_seed(workload, N, K))
+    W, q, z, s2, s1, blob = _weights(workload, N, K)
     A = I.activations(M, K, I.activation_seed(workload, M, K))
-    Wd = dev(W)
-    q, z, s2, s1 = w4a8.quantize_weights(Wd)
-    blob = w4a8.pack_weights(q, z, s2, s1)
-    del Wd
     A8, sA, rs = w4a8.quantize_act(dev(A))
     ws = torch.zeros(w4a8.workspace_bytes(M, N, K), dtype=torch.uint8, device=DEV)
     Y = w4a8.gemm(A8, sA, rs, blob, N, K, workspace=ws)
@@ -304,41 +369,30 @@ def _full_size_case(workload, lin, M, n_random_cols=64):
     tiles = [0, int(rng.integers(1, nt))]
     cols = np.unique(np.concatenate([np.arange(t * 128, t * 128 + 128) for t in tiles] +
                                     [rng.choice(N, n_random_cols, replace=False)]))
+    ct = torch.from_numpy(cols).to(DEV)
     oq, oz, os2, os1 = O.quantize_weights(W[cols])
-    assert (host(q[cols]) == oq).all() and (host(z[cols]) == oz).all()
-    assert (host(s2[cols]) == os2).all() and (host(s1[cols]).view(np.uint16) == os1.view(np.uint16)).all()
+    assert (host(q[ct]) == oq).all() and (host(z[ct]) == oz).all()
+    assert (host(s2[ct]) == os2).all() and (host(s1[ct]).view(np.uint16) == os1.view(np.uint16)).all()
     oacc = O.gemm_acc(oA8, O.dequant_weights(oq, oz, os2))
     oY = O.epilogue(oacc, osA, os1)
-    ha = host(acc)[:, cols]
-    assert (ha == oacc).all()
-    assert max_ulp_fp16(host(Y)[:, cols], oY) <= 1
+    assert (host(acc[:, ct]) == oacc).all()
+    assert max_ulp_fp16(host(Y[:, ct]), oY) <= 1
     # the packed tiles of one whole n-tile, byte for byte
     t = tiles[0]
     KT = K // 128
     sub = O.pack_weights(*O.quantize_weights(W[t * 128:(t + 1) * 128]))
-    hb = host(blob)
-    assert (hb[64 + t * KT * 8320:64 + (t + 1) * KT * 8320] == sub[64:64 + KT * 8320]).all()
-    assert not host(ws).any()
+    hb = host(blob[64 + t * KT * 8320:64 + (t + 1) * KT * 8320])
+    assert (hb == sub[64:64 + KT * 8320]).all()
+    assert not ws.any().item()
 
 
-@pytest.mark.parametrize("lin", I.LLAMA3_8B_LINEARS, ids=lambda l: l[0])
-@pytest.mark.parametrize("M", I.WORKLOADS["decode"].ms)
-def test_full_size_decode(lin, M):
-    _full_size_case("decode", lin, M)
+# Every (M, layer) case of the four dense-weight workloads (56 GEMMs; the tiny
+# case is compared in full above), ordered by layer so that each layer's
+# weights are generated once.
+FULL_SIZE_CASES = [(wl, lin, M) for wl in ("decode", "serving", "prefill", "qwen72b")
+                   for lin in I.WORKLOADS[wl].linears for M in I.WORKLOADS[wl].ms]
 
 
-@pytest.mark.parametrize("lin", I.LLAMA3_8B_LINEARS, ids=lambda l: l[0])
-@pytest.mark.parametrize("M", [64, 512])
-def test_full_size_serving(lin, M):
-    _full_size_case("serving", lin, M)
-
-
-@pytest.mark.parametrize("lin", [I.LLAMA3_8B_LINEARS[1], I.LLAMA3_8B_LINEARS[3]], ids=lambda l: l[0])
-def test_full_size_prefill(lin):
-    _full_size_case("prefill", lin, 2048)
-
-
-@pytest.mark.parametrize("lin", [I.QWEN15_72B_LINEARS[1], I.QWEN15_72B_LINEARS[3]], ids=lambda l: l[0])
-@pytest.mark.parametrize("M", [1, 32])
-def test_full_size_qwen(lin, M):
-    _full_size_case("qwen72b", lin, M)
+@pytest.mark.parametrize("workload,lin,M", FULL_SIZE_CASES, ids=lambda v: v[0] if isinstance(v, tuple) else str(v))
+def test_full_size(workload, lin, M):
+    _full_size_case(workload, lin, M)
