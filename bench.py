@@ -410,9 +410,22 @@ def run_gpu(args, world, rank, local):
         quantize = (w4a8.quantize_act_static if static_scales is not None else w4a8.quantize_act)
         gemm = w4a8.gemm
 
+    chain = bool(getattr(args, "chain_mode", False))
+    if chain:
+        # the step as one chain launch (w4a8_chain): the same quantize + GEMM
+        # per case, in the same order, each link after the previous one
+        chain_arrs = [w4a8.chain_links([dict(A=a_views[b][i], blob=blobs[(name, copy_of[M])], N=N, K=K,
+                                             Y=y_views[b][i], A8=outs[(M, name)][0], sA=outs[(M, name)][1],
+                                             rowsum=outs[(M, name)][2])
+                                        for i, (M, name, N, K) in enumerate(cases)]) for b in range(3)]
+        chain_ws = torch.zeros(w4a8.chain_workspace_bytes(chain_arrs[0]), dtype=torch.uint8, device=dev)
+
     def step(events=None, gemm_only=False, buf=0):
         """One pass over the cases; `buf` selects the activation and output
         buffers (the end-to-end run alternates between two)."""
+        if chain:
+            w4a8.chain(chain_arrs[buf], chain_ws)
+            return
         for i, (M, name, N, K) in enumerate(cases):
             A = a_views[buf][i]
             A8, sA, rs, _ = outs[(M, name)]
@@ -461,14 +474,16 @@ def run_gpu(args, world, rank, local):
     g_plain = capture(None)
     # ---- timed region 2: the GEMM launches of the same K steps alone (same
     # inputs, same launch configuration, same weight rotation), events only at
-    # the ends: the GEMM kernel's average duration for the roofline
+    # the ends: the GEMM kernel's average duration for the roofline (a chain
+    # step is one launch: this graph is the same K chain launches)
     g_gemm = capture(None, gemm_only=True)
     # ---- timed region 3: the full steps with an external event pair around
     # every GEMM (a per-case breakdown; these events add a few microseconds
-    # to each launch and stop consecutive kernels from overlapping)
+    # to each launch and stop consecutive kernels from overlapping); a chain
+    # step has no per-case launches, so it is timed as a whole
     ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in cases]
           for _ in range(K_steps)]
-    g_ev = capture(ev)
+    g_ev = capture(None if chain else ev)
     for g in (g_plain, g_gemm, g_ev):  # untimed replays: settle clocks and caches
         g.replay()
     torch.cuda.synchronize()
@@ -496,10 +511,11 @@ def run_gpu(args, world, rank, local):
     assert w4a8.get_device_error(dev) == 0
 
     per_case_ms = np.zeros(len(cases))
-    for s in range(K_steps):
-        for i in range(len(cases)):
-            per_case_ms[i] += ev[s][i][0].elapsed_time(ev[s][i][1])
-    per_case_ms /= K_steps
+    if not chain:
+        for s in range(K_steps):
+            for i in range(len(cases)):
+                per_case_ms[i] += ev[s][i][0].elapsed_time(ev[s][i][1])
+        per_case_ms /= K_steps
     del g_plain, g_gemm, g_ev
 
     # ---- end to end through the public API: each step copies its fp16
@@ -941,6 +957,10 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the CPU-oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--chain", default="off", choices=["off", "on"],
+                    help="on: run the step as one w4a8_chain launch (8-bit dynamic activations, every M <= 32, at "
+                         "most 16 cases; measured slower than separate launches on the decode workload); the "
+                         "per-launch figures are reported beside it")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-case sweep of all five workloads (the `configs` block)")
     ap.add_argument("--cases", default=None,
@@ -1046,6 +1066,43 @@ def main():
         "cases": per_case,
         "gpu": r["gpu_name"],
     }
+    use_chain = args.chain == "on" and not lut and args.act == "dynamic" and \
+        max(M for (M, _, _, _) in cases) <= 32 and len(cases) <= 16
+    if use_chain:
+        # The step as one w4a8_chain launch (the same quantize + GEMM per case,
+        # each case after the previous one): value, roofline and e2e come from
+        # it; the per-launch figures above move to `per_launch`.
+        args.chain_mode = True
+        rc = run_gpu(args, world, rank, local)
+        args.chain_mode = False
+        ms_c = rc["max_ms"] / args.steps
+        launch_c = rc["gemm_ms"] / args.steps  # one chain launch per step
+        # bytes the chain must move: weights, fp16 activations in, their codes,
+        # scales and rowsums out, Y out
+        cbytes = [weight_bytes(N, K) + 2 * M * K + M * K + 6 * M + 2 * M * N for (M, _, N, K) in cases]
+        achieved_c = sum(cbytes) / (launch_c * 1e-3) / 1e9
+        line["per_launch"] = {"value": line["value"], "ms_per_step": line["ms_per_step"], "tops": line["tops"],
+                              "roofline": roofline, "e2e": line["e2e"], "gpu_launches": line["gpu_launches"],
+                              "note": "the same step as separate w4a8_quantize_act + w4a8_gemm launches per case"}
+        line["value"] = round(world * wbytes / (ms_c * 1e-3) / 1e9, 1)
+        line["ms_per_step"] = round(ms_c, 5)
+        line["tops"] = round(world * sum(ops) / (ms_c * 1e-3) / 1e12, 2)
+        line["gpu_launches"] = args.steps
+        line["roofline"] = {"bound": "hbm", "achieved": round(achieved_c, 1), "peak": hbm, "unit": "GB/s",
+                            "frac": round(achieved_c / hbm, 4), "traffic": recorded_traffic(args.workload + "-chain"),
+                            "peak_source": f"{peaks['source']} HBM copy", "kernel": "w4a8_chain_kernel",
+                            "launches": args.steps, "avg_launch_us": round(launch_c * 1e3, 3),
+                            "bytes_per_launch": int(sum(cbytes))}
+        line["e2e"] = {"value": round(world * wbytes / (rc["e2e_ms"] / args.steps * 1e-3) / 1e9, 1), "unit": "GB/s",
+                       "h2d_bytes_per_step": rc["h2d_bytes"], "d2h_bytes_per_step": rc["d2h_bytes"]}
+        line["clocks"] = rc["clocks"]
+        line["config"]["timing"] = ("value: one CUDA graph of K unrolled steps, each step one w4a8_chain launch over "
+                                    "the cases in order (each case quantized after the previous case's output is "
+                                    "complete); roofline: the chain launch's average duration over those K launches; "
+                                    "e2e: K steps in one graph, one host-to-device and one device-to-host copy per "
+                                    "step, double-buffered on two copy streams; per_launch: the same step as "
+                                    "separate launches (cases: per-launch times with events around each GEMM)")
+        line["config"]["path"] = "w4a8_chain (one persistent launch per step)"
     if world == 1 and not args.no_configs and not lut and args.act == "dynamic" and not args.cases:
         import torch
         dev = torch.device("cuda", local)

@@ -75,6 +75,8 @@ typedef enum {
 #define W4A8_DEVERR_SELFTEST_WAIT 6
 #define W4A8_DEVERR_KV_RANGE 7 /* a KV-cache length or position outside [0, Lmax] (clamped or skipped) */
 #define W4A8_DEVERR_PACK_RANGE 8 /* a packer met a code, zero point or scale outside its documented range */
+#define W4A8_DEVERR_CHAIN_WAIT 9 /* w4a8_chain: a wait on another CTA's progress gave up */
+#define W4A8_DEVERR_BOUNDS 10     /* debug builds (W4A8_DEBUG) only: an access outside its buffer was skipped */
 
 /* Human-readable name of a status code (static string, never NULL). */
 W4A8_API const char* w4a8_status_string(int status);
@@ -218,6 +220,57 @@ typedef struct {
 W4A8_API w4a8_status_t w4a8_gemm_ex(const int8_t* A8, const void* sA, const int32_t* rowsum, const void* packed,
                                     int64_t M, int64_t N, int64_t K, void* Y, int32_t* acc, void* workspace,
                                     size_t workspace_bytes, const w4a8_gemm_opts_t* opts, w4a8_stream_t stream);
+
+/*
+ * GEMM chain for the decode regime: a sequence of up to 16 W4A8 GEMMs ("links")
+ * in ONE persistent launch. Link j computes exactly what
+ *   w4a8_quantize_act(A_j) -> (A8_j, sA_j, rowsum_j);  w4a8_gemm(...) -> Y_j
+ * computes (bit for bit), in order: link j's activations A_j are read only
+ * after every element of Y_{j-1} is written (link 0's after the preceding
+ * kernel in the stream has completed), so A_j may be Y_{j-1} (K_j == N_{j-1})
+ * or anything computed before the call. The weight stream of all links runs
+ * ahead without waiting on any activation: in a per-GEMM launch sequence every
+ * launch pays a chain of start-up and tail latencies during which HBM idles,
+ * here only the dependent part (quantize, load the codes, the remaining MMAs,
+ * the epilogue) sits between links ("LiquidGEMM: Hardware-Efficient W4A8 GEMM
+ * Kernel for High-Performance LLM Serving", Method: weight loading,
+ * dequantization and MMA overlapped in one pipeline).
+ *
+ * links: HOST array of n_links link descriptors (1 <= n_links <= 16), read
+ * during the call. Per link: A fp16 [M, K] (16-byte aligned); packed the blob
+ * of w4a8_pack_weights for N x K; A8 int8 [M, K] (16-byte aligned), sA fp16
+ * [M] (2-byte aligned), rowsum int32 [M] (4-byte aligned): written with the
+ * link's quantized activations (links may share these three buffers); Y fp16
+ * [M, N] (16-byte aligned). Limits per link: 1 <= M <= 32, N % 128 == 0,
+ * K % 128 == 0, 0 < K <= 65536.
+ * workspace: 256-byte aligned, at least w4a8_chain_workspace_bytes(links,
+ * n_links) bytes (it depends on the shapes and the device's SM count),
+ * zero-filled by the caller once; every call that completes without a device
+ * error leaves it zero-filled again. Calls sharing a workspace must not
+ * overlap on the GPU. The launch uses one CTA per SM and needs all of them
+ * resident at once (its CTAs wait on each other's progress; every such wait
+ * is bounded and reports W4A8_DEVERR_CHAIN_WAIT if it gives up, after which
+ * the workspace must be zero-filled again).
+ */
+typedef struct {
+  const void* A;       /* fp16 [M, K] activations */
+  const void* packed;  /* packed weights (w4a8_pack_weights) for N x K */
+  int64_t M, N, K;
+  int8_t* A8;          /* int8 [M, K] codes (written) */
+  void* sA;            /* fp16 [M] scales (written) */
+  int32_t* rowsum;     /* int32 [M] code sums (written) */
+  void* Y;             /* fp16 [M, N] output */
+} w4a8_chain_link_t;
+
+#define W4A8_CHAIN_MAX_LINKS 16
+#define W4A8_CHAIN_MAX_M 32
+
+/* Workspace bytes of w4a8_chain for these links on the current device (0 if
+ * the links are invalid). */
+W4A8_API size_t w4a8_chain_workspace_bytes(const w4a8_chain_link_t* links, int32_t n_links);
+
+W4A8_API w4a8_status_t w4a8_chain(const w4a8_chain_link_t* links, int32_t n_links, void* workspace,
+                                  size_t workspace_bytes, w4a8_stream_t stream);
 
 /*
  * W4A4: 4-bit weights against 4-bit activations, the W4A4KV4 models of

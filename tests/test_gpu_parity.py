@@ -84,6 +84,44 @@ def test_quantize_act_static_bit_exact(M, K, s):
     assert (host(rs) == ors).all()
 
 
+def half_integer_rows(K, scale_exp):
+    """Rows whose values over the scale 2^scale_exp are half-integers n + 1/2
+    (ties) or one fp16 step above or below one; one element 127 * 2^e sets
+    amax, so the dynamic scale is exactly 2^e."""
+    n = np.arange(-127, 127, dtype=np.float64)
+    ties = ((n + 0.5) * 2.0 ** scale_exp).astype(np.float16)
+    up = np.nextafter(ties, np.float16(np.inf))
+    down = np.nextafter(ties, np.float16(-np.inf))
+    vals = np.concatenate([ties, up, down])
+    rows = []
+    for shift in range(3):
+        r = np.zeros(K, np.float16)
+        r[:vals.size] = np.roll(vals, 37 * shift)
+        r[K - 1] = np.float16(127 * 2.0 ** scale_exp)
+        rows.append(r)
+    return np.stack(rows)
+
+
+@pytest.mark.parametrize("scale_exp", [-4, -9, 3])
+def test_quantize_act_half_integer_quotients(scale_exp):
+    """Quotients exactly at and one fp16 step beside half-integers: the codes
+    follow the IEEE divide and ties-to-even exactly."""
+    A = half_integer_rows(4096, scale_exp)
+    A8, sA, rs = w4a8.quantize_act(dev(A))
+    oA8, osA, ors = O.quantize_act(A)
+    torch.cuda.synchronize()
+    assert (host(sA).view(np.uint16) == osA.view(np.uint16)).all()
+    assert (host(A8) == oA8).all() and (host(rs) == ors).all()
+    s = np.array([2.0 ** scale_exp], np.float16)
+    sA8, _, srs = w4a8.quantize_act_static(dev(A), dev(s))
+    oS8, _, osrs = O.quantize_act_static(A, s[0])
+    A4, sA4, rs4 = w4a8.w4a4_quantize_act(dev(A))
+    oA4, osA4, ors4 = O.quantize_act4(A)
+    torch.cuda.synchronize()
+    assert (host(sA8) == oS8).all() and (host(srs) == osrs).all()
+    assert (host(A4) == O.pack_act4(oA4)).all() and (host(rs4) == ors4).all()
+
+
 def test_static_quantization_through_the_gemm():
     """Static activation codes feed the unchanged GEMM: bit-exact int32
     accumulators and Y within 1 ulp of the oracle's static path."""

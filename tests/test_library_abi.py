@@ -210,3 +210,34 @@ def test_lut3_validation(L):
     assert g(FAKE, FAKE, 0, 128, 256, FAKE, None, 0, None) == 0
     bad = w4a8.GemmOpts(0, 64, 0, 0)
     assert L.w4lut3_gemm_ex(FAKE, FAKE, 4, 128, 256, FAKE, None, None, 0, ctypes.byref(bad), None) == 1
+
+
+def test_chain_validation_on_the_host():
+    """w4a8_chain checks its links before touching the device."""
+    import ctypes
+    L = w4a8.lib()
+    Link = w4a8.ChainLink
+    buf = ctypes.create_string_buffer(1 << 16)
+    base = (ctypes.addressof(buf) + 255) // 256 * 256
+
+    def link(**kw):
+        d = dict(A=base, packed=base, M=4, N=256, K=512, A8=base, sA=base, rowsum=base, Y=base)
+        d.update(kw)
+        return Link(*(d[f] for f, _ in Link._fields_))
+
+    def status(links, ws=base, nbytes=1 << 15):
+        arr = (Link * max(len(links), 1))(*links)
+        return w4a8.status_string(L.w4a8_chain(arr, len(links), ctypes.c_void_p(ws), nbytes, None))
+
+    assert status([]) == "W4A8_ERR_INVALID_ARG"
+    assert status([link()] * 17) == "W4A8_ERR_INVALID_ARG"
+    assert status([link(M=33)]) == "W4A8_ERR_UNSUPPORTED_SHAPE"
+    assert status([link(M=0)]) == "W4A8_ERR_INVALID_ARG"
+    assert status([link(N=200)]) == "W4A8_ERR_UNSUPPORTED_SHAPE"
+    assert status([link(K=65536 + 128)]) == "W4A8_ERR_UNSUPPORTED_SHAPE"
+    assert status([link(Y=0)]) == "W4A8_ERR_INVALID_ARG"
+    assert status([link(A=base + 8)]) == "W4A8_ERR_MISALIGNED"
+    assert status([link(rowsum=base + 2)]) == "W4A8_ERR_MISALIGNED"
+    assert status([link()], ws=base + 16) == "W4A8_ERR_MISALIGNED"
+    arr = (Link * 1)(link(M=40))
+    assert L.w4a8_chain_workspace_bytes(arr, 1) == 0

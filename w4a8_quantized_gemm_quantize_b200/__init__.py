@@ -22,6 +22,7 @@ __all__ = [
     "selftest_bounded_wait", "quantize_act_static", "w4a4_quantize_act", "w4a4_quantize_act_static",
     "w4a4_gemm", "w4a4_gemm_ex", "w4a4_workspace_bytes", "lut_packed_bytes", "lut_pack_weights", "lut_gemm",
     "lut_gemm_ex", "lut3_packed_bytes", "lut3_pack_weights", "lut3_gemm", "lut3_gemm_ex", "kv4_quantize", "kv4_append", "kv4_workspace_bytes", "kv4_attention_decode",
+    "ChainLink", "chain_links", "chain_workspace_bytes", "chain",
 ]
 
 _PKG_DIR = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +37,7 @@ EXPORTED_SYMBOLS = (
     "w4lut_packed_bytes", "w4lut_pack_weights", "w4lut_gemm", "w4lut_gemm_ex",
     "w4kv_quantize", "w4kv_append", "w4kv_attention_workspace_bytes", "w4kv_attention_decode",
     "w4lut3_packed_bytes", "w4lut3_pack_weights", "w4lut3_gemm", "w4lut3_gemm_ex",
+    "w4a8_chain_workspace_bytes", "w4a8_chain",
 )
 
 SCHEDULE_AUTO, SCHEDULE_WHOLE_TILES, SCHEDULE_SPLIT_K, SCHEDULE_CLUSTER = 0, 1, 2, 3
@@ -48,6 +50,13 @@ class W4A8Error(RuntimeError):
 class GemmOpts(ctypes.Structure):
     _fields_ = [("schedule", ctypes.c_int32), ("block_m", ctypes.c_int32),
                 ("max_ctas", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+class ChainLink(ctypes.Structure):
+    """w4a8_chain_link_t: one GEMM of a chain (device pointers and shape)."""
+    _fields_ = [("A", ctypes.c_void_p), ("packed", ctypes.c_void_p), ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+                ("K", ctypes.c_int64), ("A8", ctypes.c_void_p), ("sA", ctypes.c_void_p), ("rowsum", ctypes.c_void_p),
+                ("Y", ctypes.c_void_p)]
 
 
 _lib = None
@@ -99,6 +108,8 @@ def lib() -> ctypes.CDLL:
         "w4kv_attention_workspace_bytes": (sz, [i64, i64, i64, i64, i32]),
         "w4kv_attention_decode": (ctypes.c_int, [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, ctypes.c_float,
                                                  vp, vp, sz, vp]),
+        "w4a8_chain_workspace_bytes": (sz, [ctypes.POINTER(ChainLink), i32]),
+        "w4a8_chain": (ctypes.c_int, [ctypes.POINTER(ChainLink), i32, vp, sz, vp]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -515,6 +526,8 @@ def clear_device_error(device=None):
 DEVERR_SELFTEST_WAIT = 6
 DEVERR_KV_RANGE = 7
 DEVERR_PACK_RANGE = 8
+DEVERR_CHAIN_WAIT = 9
+DEVERR_BOUNDS = 10
 
 
 def selftest_bounded_wait(limit_ns: int, device=None):
@@ -592,3 +605,38 @@ def kv4_attention_decode(q, k_codes, k_params, v_codes, v_params, seq_lens, scal
                                        _ptr(seq_lens), B, Hq, Hkv, Lmax, D, float(scale), _ptr(Y), _ptr(workspace),
                                        ws_bytes, _stream(q.device)), "w4kv_attention_decode")
     return Y
+
+
+# ------------------------------------------------------------- GEMM chain
+def chain_links(links):
+    """ctypes array of w4a8_chain_link_t from dicts with the tensors A (fp16
+    [M, K]), blob, N, K, Y (fp16 [M, N]) and A8 / sA / rowsum (int8 [M, K],
+    fp16 [M], int32 [M]: where the link's quantized activations go)."""
+    torch = _torch()
+    arr = (ChainLink * len(links))()
+    for i, d in enumerate(links):
+        A, Y = d["A"], d["Y"]
+        _require_cuda(A, d["blob"], Y, d["A8"], d["sA"], d["rowsum"])
+        if A.dtype != torch.float16 or A.dim() != 2 or A.shape[1] != d["K"]:
+            raise W4A8Error("A must be fp16 [M, K]")
+        if Y.dtype != torch.float16 or tuple(Y.shape) != (A.shape[0], d["N"]):
+            raise W4A8Error("Y must be fp16 [M, N]")
+        arr[i] = ChainLink(_ptr(A), _ptr(d["blob"]), A.shape[0], d["N"], d["K"], _ptr(d["A8"]), _ptr(d["sA"]),
+                           _ptr(d["rowsum"]), _ptr(Y))
+    return arr
+
+
+def chain_workspace_bytes(links) -> int:
+    arr = links if isinstance(links, ctypes.Array) else chain_links(links)
+    return int(lib().w4a8_chain_workspace_bytes(arr, len(arr)))
+
+
+def chain(links, workspace):
+    """Runs the links in order in one launch (w4a8_chain): link j quantizes
+    its A after link j - 1's Y is complete, then computes its Y. `workspace`
+    is a zero-filled uint8 CUDA tensor of at least chain_workspace_bytes."""
+    arr = links if isinstance(links, ctypes.Array) else chain_links(links)
+    _require_cuda(workspace)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    dev = workspace.device
+    _check(lib().w4a8_chain(arr, len(arr), _ptr(workspace), ws_bytes, _stream(dev)), "w4a8_chain")

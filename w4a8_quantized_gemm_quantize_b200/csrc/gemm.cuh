@@ -137,9 +137,11 @@ constexpr int kLutTileBytes = kTileCodeBytes + 2 * kTileN;  // 8448
 constexpr int kLut3CodeBytes = 3 * 16 * kTileN;             // 6144
 constexpr int kLut3TileBytes = kLut3CodeBytes + 2 * kTileN;  // 6400
 
-template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_, int NMMA_, int LUT_ = 0>
+template <int BN_, int KS_, int NS_, int NT_, int DQ_, int NACC_, int NMMA_, int LUT_ = 0, int MINB_ = 1>
 struct GemmCfg {
   static constexpr int BN = BN_, KS = KS_, NS = NS_, NT = NT_, DQ = DQ_, NACC = NACC_, NMMA = NMMA_;
+  // CTAs meant to be resident per SM (the register budget the compiler gets)
+  static constexpr int kMinBlocks = MINB_;
   // LUT_ != 0: lookup-table weights against fp16 activations (kind::f16 MMA,
   // fp32 accumulators), 4-bit indices (1) or 3-bit indices in bit planes (3);
   // otherwise two-level 4-bit weights against int8 (kind::i8)
@@ -368,6 +370,7 @@ struct RowStage {
 __device__ __forceinline__ void store_output(const GemmArgs& a, int64_t o, uint32_t biased, int32_t rowsum, float sa,
                                              float s1f) {
   const int32_t acc = static_cast<int32_t>(biased - (static_cast<uint32_t>(rowsum) << 7));
+  if (!in_bounds(o >= 0 && o < static_cast<int64_t>(a.M) * a.N, a.err)) return;
   if (a.acc_out != nullptr) {
     a.acc_out[o] = acc;
   } else {
@@ -389,6 +392,7 @@ template <bool LUT>
 __device__ __forceinline__ void store_out(const GemmArgs& a, int64_t o, uint32_t v, int32_t rowsum, float sa,
                                           float s1f) {
   if constexpr (LUT) {
+    if (!in_bounds(o >= 0 && o < static_cast<int64_t>(a.M) * a.N, a.err)) return;
     if (a.acc_out != nullptr) {
       a.acc_out[o] = static_cast<int32_t>(v);
     } else {
@@ -429,7 +433,8 @@ __device__ __forceinline__ void store_y_rows16(const GemmArgs& a, __half* stage,
     const int r = pass * 8 + (lane >> 2), q = lane & 3;
     const uint4 v = *reinterpret_cast<const uint4*>(stage + r * 32 + q * 8);
     const int m = m_start + r;
-    if (m < a.M) *reinterpret_cast<uint4*>(a.Y + static_cast<int64_t>(m) * a.N + n_base + q * 8) = v;
+    if (m < a.M && in_bounds(m >= 0 && n_base >= 0 && n_base + q * 8 + 8 <= a.N, a.err))
+      *reinterpret_cast<uint4*>(a.Y + static_cast<int64_t>(m) * a.N + n_base + q * 8) = v;
   }
   __syncwarp();  // the stage is reused by the next block
 }
@@ -487,7 +492,8 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const int m = m0 + c + j;
-        if (m < args.M) red_add_acc<LUT>(args.ws_acc + static_cast<int64_t>(m) * N + n, v[j]);
+        if (m < args.M && in_bounds(n < N && args.ws_acc != nullptr, args.err))
+          red_add_acc<LUT>(args.ws_acc + static_cast<int64_t>(m) * N + n, v[j]);
       }
     } else if (args.acc_out != nullptr) {
 #pragma unroll
@@ -515,7 +521,9 @@ __device__ __forceinline__ bool epilogue_segment(const GemmArgs& args, const Seg
     if (quarter == 0 && lane == 0) {
       const int add = sg.kb1 - sg.kb0;
       fence_acq_rel_gpu();
-      const int old = atom_add_relaxed_gpu(args.ws_cnt + sg.tile, add);
+      const int old = in_bounds(sg.tile < args.num_tiles && args.ws_cnt != nullptr, args.err)
+                          ? atom_add_relaxed_gpu(args.ws_cnt + sg.tile, add)
+                          : -add;
       fence_acq_rel_gpu();
       *last_flag = (old + add == args.KB) ? 1 : 0;
     }
@@ -792,7 +800,7 @@ __device__ __forceinline__ void act4_producer(const GemmArgs& args, const CUtens
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::kThreads, 1) w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
+__global__ void __launch_bounds__(C::kThreads, C::kMinBlocks) w4a8_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                                                                     const GemmArgs args) {
   constexpr int BN = C::BN, KS = C::KS, NS = C::NS, NT = C::NT, DQ = C::DQ, NACC = C::NACC, NMMA = C::NMMA;
   extern __shared__ __align__(1024) uint8_t smem_raw[];

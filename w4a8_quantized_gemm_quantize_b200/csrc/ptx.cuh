@@ -31,6 +31,22 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
   return t;
 }
 
+// Debug builds (-DW4A8_DEBUG): every global store and workspace access of
+// the GEMM, the chain and the quantizers is checked against its buffer's
+// extent; a failed check records W4A8_DEVERR_BOUNDS in the device error word
+// and the access is skipped (no trap). Release builds compile the checks away.
+constexpr int kErrBounds = 10;  // W4A8_DEVERR_BOUNDS
+__device__ __forceinline__ bool in_bounds(bool ok, int* err) {
+#ifdef W4A8_DEBUG
+  if (!ok) atomicCAS(err, 0, kErrBounds);
+  return ok;
+#else
+  (void)ok;
+  (void)err;
+  return true;
+#endif
+}
+
 // ------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -40,6 +56,16 @@ __device__ __forceinline__ void fence_barrier_init() {
 }
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+// Orders this thread's generic-proxy global writes before later async-proxy
+// (TMA) accesses, here or, after a release/acquire, in another CTA.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");

@@ -7,6 +7,7 @@
 #include <mutex>
 #include <utility>
 
+#include "chain.cuh"
 #include "gemm.cuh"
 #include "kv4_attention.cuh"
 #include "pack.cuh"
@@ -317,9 +318,23 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   w4a8_status_t st = device_info(&dev);
   if (st != W4A8_OK) return st;
 
-  int bn = o.block_m;
-  if (bn == 0) bn = M <= 16 ? 16 : M <= 32 || lut ? 32 : M <= 64 ? 64 : 128;
+  // Tokens per tile: the smallest of 16 / 32 that holds M up to 32 tokens;
+  // up to 64 tokens, two 32-token tiles when every tile then still gets a
+  // cluster of two or more CTAs (the k-range split reduced on chip), else one
+  // 64-token tile; beyond, 128.
   const int n_tiles = static_cast<int>(N / kTileN);
+  int bn = o.block_m;
+  if (bn == 0) {
+    if (M <= 16) {
+      bn = 16;
+    } else if (M <= 32 || lut) {
+      bn = 32;
+    } else if (M <= 64) {
+      bn = 2 * (2 * static_cast<int64_t>(n_tiles)) <= dev->sms ? 32 : 64;
+    } else {
+      bn = 128;
+    }
+  }
   const int m_tiles = static_cast<int>((M + bn - 1) / bn);
   const int64_t num_tiles64 = static_cast<int64_t>(n_tiles) * m_tiles;
   if (num_tiles64 > INT32_MAX) return W4A8_ERR_UNSUPPORTED_SHAPE;
@@ -398,8 +413,23 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   } else if (o.schedule == 2) {
     if (!ws_ok) return W4A8_ERR_WORKSPACE;
     sk_tiles = num_tiles;
-  } else if (o.schedule == 0 && ws_ok) {
-    sk_tiles = num_tiles < max_ctas ? num_tiles : num_tiles % max_ctas;
+  } else if (o.schedule == 0 && ws_ok && bn <= 32) {
+    // Token tiles of up to 32: with fewer tiles than CTAs (and no cluster
+    // split) every tile is split over all CTAs, partial sums reduced through
+    // the workspace. With at least a wave of tiles, the tiles of the last,
+    // partial wave are split that way only when whole tiles would leave the
+    // CTAs idle for more than about 20 k-blocks each on average (measured
+    // break-even against the cost of the partial-sum reduction). Token tiles
+    // of 64 and more always go whole: their partial tiles (64 x 128 int32
+    // sums and up, one global atomic per element) measured slower than idle
+    // CTAs on every such shape.
+    if (num_tiles < max_ctas) {
+      sk_tiles = num_tiles;
+    } else {
+      const int64_t rem = num_tiles % max_ctas;
+      const int64_t idle_kb = rem == 0 ? 0 : (max_ctas - rem) * static_cast<int64_t>(KB) / max_ctas;
+      sk_tiles = idle_kb > 20 ? static_cast<int>(rem) : 0;
+    }
   }
   int grid;
   if (split > 1) {
@@ -449,6 +479,72 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   }
 }
 
+
+// ------------------------------------------------------------- GEMM chain
+using CfgChain = GemmCfg<kChainMaxM, 3, 4, 4, 2, 2, 2>;
+
+// Per-link split and workspace layout of a chain on a device with `sms` SMs:
+// counters (done[n], ready[n], exits) first, then per link with split > 1
+// its tickets and partial sums, each from a 256-byte boundary.
+struct ChainPlan {
+  int split[kChainMaxLinks];
+  int seg0[kChainMaxLinks];
+  size_t ticket_off[kChainMaxLinks];
+  size_t part_off[kChainMaxLinks];
+  size_t total;
+};
+
+size_t round256u(size_t x) { return (x + 255) / 256 * 256; }
+
+void chain_plan(const w4a8_chain_link_t* links, int n, int sms, ChainPlan* p) {
+  size_t off = round256u(static_cast<size_t>(2 * n + 1) * 4);
+  int seg = 0;
+  for (int j = 0; j < n; ++j) {
+    const int T = static_cast<int>(links[j].N / kTileN), KB = static_cast<int>(links[j].K / kTileK);
+    int S = 1;
+    for (int s2 = 4; s2 >= 2; --s2)
+      if (T * s2 <= sms && s2 <= KB) {
+        S = s2;
+        break;
+      }
+    p->split[j] = S;
+    p->seg0[j] = seg;
+    seg += T * S;
+    p->ticket_off[j] = p->part_off[j] = 0;
+    if (S > 1) {
+      p->ticket_off[j] = off;
+      off += round256u(static_cast<size_t>(T) * 4);
+      p->part_off[j] = off;
+      off += round256u(static_cast<size_t>(T) * S * static_cast<size_t>(links[j].M) * kTileN * 4);
+    }
+  }
+  p->total = off;
+}
+
+w4a8_status_t check_chain_links(const w4a8_chain_link_t* links, int32_t n) {
+  if (links == nullptr || n < 1 || n > kChainMaxLinks) return W4A8_ERR_INVALID_ARG;
+  for (int j = 0; j < n; ++j) {
+    const w4a8_chain_link_t& L = links[j];
+    if (L.M < 1 || L.N < 1 || L.K < 1) return W4A8_ERR_INVALID_ARG;
+    if (L.M > kChainMaxM || L.N % kTileN != 0 || L.N > INT32_MAX || L.K % kTileK != 0 || L.K > kMaxK)
+      return W4A8_ERR_UNSUPPORTED_SHAPE;
+    if (L.A == nullptr || L.packed == nullptr || L.A8 == nullptr || L.sA == nullptr || L.rowsum == nullptr ||
+        L.Y == nullptr)
+      return W4A8_ERR_INVALID_ARG;
+    if (!aligned(L.A, 16) || !aligned(L.packed, 16) || !aligned(L.A8, 16) || !aligned(L.Y, 16) ||
+        !aligned(L.sA, 2) || !aligned(L.rowsum, 4))
+      return W4A8_ERR_MISALIGNED;
+  }
+  return W4A8_OK;
+}
+
+w4a8_status_t chain_sms(int* sms) {
+  DeviceInfo* dev = nullptr;
+  const w4a8_status_t st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+  *sms = dev->sms;
+  return W4A8_OK;
+}
 
 // ------------------------------------------------------------ 4-bit KV cache
 constexpr int64_t kKvMaxLen = int64_t(1) << 24;
@@ -786,6 +882,77 @@ w4a8_status_t w4a8_gemm_noalloc(const int8_t* A8, const void* sA, const int32_t*
   return gemm_impl(A8, sA, rowsum, packed, M, N, K, Y, nullptr, scratch, need, nullptr, st);
 }
 
+
+size_t w4a8_chain_workspace_bytes(const w4a8_chain_link_t* links, int32_t n_links) {
+  if (check_chain_links(links, n_links) != W4A8_OK) return 0;
+  int sms = 0;
+  if (chain_sms(&sms) != W4A8_OK) return 0;
+  ChainPlan p;
+  chain_plan(links, n_links, sms, &p);
+  return p.total;
+}
+
+w4a8_status_t w4a8_chain(const w4a8_chain_link_t* links, int32_t n_links, void* workspace, size_t workspace_bytes,
+                         w4a8_stream_t stream) {
+  w4a8_status_t st = check_chain_links(links, n_links);
+  if (st != W4A8_OK) return st;
+  if (workspace != nullptr && !aligned(workspace, 256)) return W4A8_ERR_MISALIGNED;
+  DeviceInfo* dev = nullptr;
+  st = device_info(&dev);
+  if (st != W4A8_OK) return st;
+  int dev_id = 0;
+  cudaGetDevice(&dev_id);
+  ChainPlan p;
+  chain_plan(links, n_links, dev->sms, &p);
+  if (workspace == nullptr || workspace_bytes < p.total) return W4A8_ERR_WORKSPACE;
+  {
+    static int attr_set[kMaxDevices] = {};
+    if (!attr_set[dev_id]) {
+      if (cudaFuncSetAttribute(w4a8_chain_kernel<CfgChain>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               CfgChain::kSmemBytes) != cudaSuccess)
+        return launch_status();
+      attr_set[dev_id] = 1;
+    }
+  }
+  ChainMaps maps;
+  ChainArgs a;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  a.n_links = n_links;
+  a.done = reinterpret_cast<int32_t*>(ws);
+  a.ready = a.done + n_links;
+  a.exits = a.ready + n_links;
+  a.err = dev->err;
+  for (int j = 0; j < n_links; ++j) {
+    const w4a8_chain_link_t& L = links[j];
+    ChainLink& c = a.link[j];
+    c.tiles = static_cast<const uint8_t*>(L.packed) + kHeaderBytes;
+    c.s1 = reinterpret_cast<const __half*>(static_cast<const uint8_t*>(L.packed) + packed_s1_offset(L.N, L.K));
+    c.A = static_cast<const __half*>(L.A);
+    c.A8 = L.A8;
+    c.sA = static_cast<__half*>(L.sA);
+    c.rowsum = L.rowsum;
+    c.Y = static_cast<__half*>(L.Y);
+    c.M = static_cast<int>(L.M);
+    c.N = static_cast<int>(L.N);
+    c.KB = static_cast<int>(L.K / kTileK);
+    c.num_tiles = static_cast<int>(L.N / kTileN);
+    c.split = p.split[j];
+    c.seg0 = p.seg0[j];
+    c.ticket = p.split[j] > 1 ? reinterpret_cast<int32_t*>(ws + p.ticket_off[j]) : nullptr;
+    c.part = p.split[j] > 1 ? reinterpret_cast<int32_t*>(ws + p.part_off[j]) : nullptr;
+    // the link's int8 codes, read as 128-byte rows with the 128-byte swizzle
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(L.K), static_cast<cuuint64_t>(L.M)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(L.K)};
+    const cuuint32_t box[2] = {128u, static_cast<cuuint32_t>(CfgChain::BN)};
+    const cuuint32_t estr[2] = {1u, 1u};
+    if (g_encode(&maps.m[j], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, L.A8, dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return W4A8_ERR_CUDA;
+  }
+  return launch_pdl(w4a8_chain_kernel<CfgChain>, dim3(dev->sms), dim3(CfgChain::kThreads), CfgChain::kSmemBytes,
+                    reinterpret_cast<cudaStream_t>(stream), 1, maps, a);
+}
 
 w4a8_status_t w4kv_quantize(const void* X, int64_t n, int32_t D, uint8_t* codes, uint32_t* params,
                             w4a8_stream_t stream) {
