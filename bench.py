@@ -1046,6 +1046,8 @@ def main():
         "scaling": "weak", "vs_baseline": None, "dtype": "fp16" if lut else "int8", "data": "synthetic",
         "config": {"workload": args.workload, "weights": args.weights,
                    "activation_scales": "none (fp16 activations)" if lut else args.act, "cases": len(cases),
+                   "gemm_call": ("w4a4_gemm" if ACT_BITS[args.act] == 4 and not lut
+                                 else "w4lut3_gemm" if lut == 3 else "w4lut_gemm" if lut else "w4a8_gemm"),
                    "shapes": [f"M={M} {n} {N}x{K}" for (M, n, N, K) in cases][:: max(1, len(cases) // 16)],
                    "group": 128, "weights_per_step_MB": round(wbytes / 1e6, 1),
                    "l2": f"inputs larger than L2: {r['n_copies']} weight copies, {wbytes / 1e6:.0f} MB per step",

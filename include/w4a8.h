@@ -77,6 +77,7 @@ typedef enum {
 #define W4A8_DEVERR_PACK_RANGE 8 /* a packer met a code, zero point or scale outside its documented range */
 #define W4A8_DEVERR_CHAIN_WAIT 9 /* w4a8_chain: a wait on another CTA's progress gave up */
 #define W4A8_DEVERR_BOUNDS 10     /* debug builds (W4A8_DEBUG) only: an access outside its buffer was skipped */
+#define W4A8_DEVERR_KV_WAIT 11    /* w4kv_attention_decode: a chunk's cache copies did not land in time */
 
 /* Human-readable name of a status code (static string, never NULL). */
 W4A8_API const char* w4a8_status_string(int status);

@@ -24,10 +24,12 @@
 // query heads per kv head, so at that grouping the arithmetic, not HBM, is
 // expected to set the pace.
 //
-// Mapping inside a CTA (both phases): 8 lanes per token, lane slice li owns
-// elements [16 li, 16 li + 16) (8 code bytes, one 8-byte load), so a warp
-// reads 4 consecutive tokens = 256 contiguous bytes per step. Products of an
-// fp16 query element and a small integer (code - z) are exact in fp32.
+// Mapping inside a CTA (both phases): the chunk's K and V codes are staged in
+// shared memory by two bulk copies issued at the start (all 2 x n x 64 bytes
+// in flight at once); 8 lanes per token, lane slice li owns elements
+// [16 li, 16 li + 16) (8 code bytes), so a warp reads 4 consecutive tokens =
+// 256 contiguous bytes of shared memory per step. Products of an fp16 query
+// element and a small integer (code - z) are exact in fp32.
 #pragma once
 #include "ptx.cuh"
 
@@ -39,6 +41,7 @@ constexpr int kKvChunk = 256;          // tokens per CTA
 constexpr int kKvThreads = 256;        // 8 warps
 constexpr int kKvWarps = kKvThreads / 32;
 constexpr int kErrKvRange = 7;         // W4A8_DEVERR_KV_RANGE
+constexpr int kErrKvWait = 11;         // W4A8_DEVERR_KV_WAIT
 
 // ------------------------------------------------------------ quantizer
 struct KvQuantArgs {
@@ -140,10 +143,21 @@ __device__ __forceinline__ void kv_param(uint32_t p, float& s, float& bias) {
 template <int GC>
 __global__ void __launch_bounds__(kKvThreads) kv4_decode_kernel(KvAttnArgs a) {
   static_assert(GC == 1 || GC == 2 || GC == 4, "query heads per CTA");
+  // the chunk's K and V codes, staged by two bulk copies (kKvChunk x 64 bytes
+  // each); once the scores are done the K codes' space holds the per-warp
+  // weighted values (s_o)
+  constexpr int kKcBytes = kKvChunk * kKvRowBytes;
+  constexpr int kOBytes = kKvWarps * GC * kKvD * 4;
+  static_assert(kOBytes <= kKcBytes, "the weighted values fit in the K codes' space");
+  __shared__ __align__(128) uint8_t s_kc[kKcBytes];
+  __shared__ __align__(128) uint8_t s_vc[kKvChunk * kKvRowBytes];
+  __shared__ float2 s_kpar[kKvChunk];  // per token: (s, 2^23 + z)
+  __shared__ float2 s_vpar[kKvChunk];
+  __shared__ uint64_t s_bar;
   __shared__ float s_q[GC][kKvD];
   __shared__ float s_p[GC][kKvChunk];
   __shared__ float s_m[GC], s_l[GC];
-  __shared__ float s_o[kKvWarps][GC][kKvD];
+  float(*s_o)[GC][kKvD] = reinterpret_cast<float(*)[GC][kKvD]>(s_kc);
   __shared__ int s_last;
 
   const int split = blockIdx.x;
@@ -156,6 +170,10 @@ __global__ void __launch_bounds__(kKvThreads) kv4_decode_kernel(KvAttnArgs a) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int grp = lane >> 3, li = lane & 7;
 
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_barrier_init();
+  }
   grid_dependency_wait();  // q and the cache come from the preceding kernels
   grid_launch_dependents();
 
@@ -166,12 +184,34 @@ __global__ void __launch_bounds__(kKvThreads) kv4_decode_kernel(KvAttnArgs a) {
   }
   const int t0 = split * kKvChunk;
   const int n = max(0, min(L - t0, kKvChunk));  // tokens of this chunk
-
+  const int64_t cache_row0 = (static_cast<int64_t>(b) * a.Hkv + g) * a.Lmax + t0;
+  __syncthreads();  // the barrier is initialized
+  // The chunk's codes are contiguous in the cache (64 bytes per token, rows
+  // 64-byte aligned): two bulk copies put all of them in flight at once, so
+  // the CTA streams its 2 x 16 KB instead of waiting once per token step.
+  if (threadIdx.x == 0 && n > 0) {
+    const uint64_t pol = l2_policy_evict_first();
+    mbar_arrive_expect_tx(&s_bar, 2u * n * kKvRowBytes);
+    bulk_load(s_kc, a.kc + cache_row0 * kKvRowBytes, n * kKvRowBytes, &s_bar, pol);
+    bulk_load(s_vc, a.vc + cache_row0 * kKvRowBytes, n * kKvRowBytes, &s_bar, pol);
+  }
+  // parameter words (4 bytes per token: no 16-byte alignment to rely on) by plain loads
+  for (int j = threadIdx.x; j < n; j += kKvThreads) {
+    float sk, bk, sv, bv;
+    kv_param(__ldg(a.kp + cache_row0 + j), sk, bk);
+    kv_param(__ldg(a.vp + cache_row0 + j), sv, bv);
+    s_kpar[j] = make_float2(sk, bk);
+    s_vpar[j] = make_float2(sv, bv);
+  }
   for (int i = threadIdx.x; i < GC * kKvD; i += kKvThreads)
     s_q[i / kKvD][i % kKvD] = __half2float(a.q[(static_cast<int64_t>(b) * a.Hq + h0 + i / kKvD) * kKvD + i % kKvD]);
   __syncthreads();
+  if (n > 0 && !mbar_wait_limit(&s_bar, 0, nullptr, DevErr{a.err}, kErrKvWait, kWaitLimitNs)) {
+    // the copies did not land in time (recorded): no result for this chunk
+    // beyond zeros, and no exit while copies may still be in flight
+    mbar_wait_limit(&s_bar, 0, nullptr, DevErr{a.err}, kErrKvWait, kWaitLimitNs);
+  }
 
-  const int64_t cache_row0 = (static_cast<int64_t>(b) * a.Hkv + g) * a.Lmax + t0;
   // ---- scores: s_p[h][j] = scale * (s^K_j * sum_d q[d] (code - z))
   {
     float qr[GC][16];
@@ -183,13 +223,12 @@ __global__ void __launch_bounds__(kKvThreads) kv4_decode_kernel(KvAttnArgs a) {
       const int j = j0 + grp;
       const bool valid = j < n;
       uint2 w = make_uint2(0u, 0u);
-      uint32_t p = 0u;
+      float2 par = make_float2(0.0f, 8388608.0f);
       if (valid) {
-        w = __ldg(reinterpret_cast<const uint2*>(a.kc + (cache_row0 + j) * kKvRowBytes) + li);
-        p = __ldg(a.kp + cache_row0 + j);
+        w = *reinterpret_cast<const uint2*>(s_kc + j * kKvRowBytes + li * 8);
+        par = s_kpar[j];
       }
-      float sk, bias;
-      kv_param(p, sk, bias);
+      const float sk = par.x, bias = par.y;
       float x[16];
       kv_unpack16(w, bias, x);
       float acc[GC];
@@ -240,9 +279,8 @@ __global__ void __launch_bounds__(kKvThreads) kv4_decode_kernel(KvAttnArgs a) {
     for (int j0 = warp * 4; j0 < n; j0 += kKvWarps * 4) {
       const int j = j0 + grp;
       if (j < n) {
-        const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.vc + (cache_row0 + j) * kKvRowBytes) + li);
-        float sv, bias;
-        kv_param(__ldg(a.vp + cache_row0 + j), sv, bias);
+        const uint2 w = *reinterpret_cast<const uint2*>(s_vc + j * kKvRowBytes + li * 8);
+        const float sv = s_vpar[j].x, bias = s_vpar[j].y;
         float x[16];
         kv_unpack16(w, bias, x);
 #pragma unroll
@@ -291,20 +329,48 @@ __global__ void __launch_bounds__(kKvThreads) kv4_decode_kernel(KvAttnArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
+  // Merge, in a fixed order (bit-reproducible): warp h finds head h's maximum
+  // over the chunks that hold tokens and the denominator sum_c exp(m_c - m) l_c,
+  // keeping the chunk factors exp(m_c - m) in shared memory (the spent V codes'
+  // space); then every (head, element) thread sums its weighted values over the
+  // chunks with independent loads.
+  constexpr int kMergeSmem = kKcBytes / (4 * GC);  // chunk factors kept per head
+  float* s_f = reinterpret_cast<float*>(s_vc);
+  if (warp < GC) {
+    const float* pp = a.part + (static_cast<int64_t>(b) * a.Hq + h0 + warp) * a.nsplit * pstride;
+    float m = -INFINITY;
+    for (int c = lane; c < a.nsplit; c += 32)
+      if (__ldcg(pp + c * pstride + 1) > 0.0f) m = fmaxf(m, __ldcg(pp + c * pstride));
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float den = 0.0f;
+    for (int c = lane; c < a.nsplit; c += 32) {
+      const float lc = __ldcg(pp + c * pstride + 1);
+      const float f = lc > 0.0f ? expf(__ldcg(pp + c * pstride) - m) : 0.0f;
+      if (c < kMergeSmem) s_f[warp * kMergeSmem + c] = f;
+      den = fmaf(f, lc, den);
+    }
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane == 0) {
+      s_m[warp] = m;
+      s_l[warp] = den;
+    }
+  }
+  __syncthreads();
   for (int i = threadIdx.x; i < GC * kKvD; i += kKvThreads) {
     const int h = i / kKvD, d = i % kKvD;
     const float* pp = a.part + (static_cast<int64_t>(b) * a.Hq + h0 + h) * a.nsplit * pstride;
-    float m = -INFINITY;
-    for (int c = 0; c < a.nsplit; ++c)
-      if (__ldcg(pp + c * pstride + 1) > 0.0f) m = fmaxf(m, __ldcg(pp + c * pstride));
-    float den = 0.0f, num = 0.0f;
+    const float m = s_m[h], den = s_l[h];
+    float num = 0.0f;
+#pragma unroll 8
     for (int c = 0; c < a.nsplit; ++c) {
-      const float lc = __ldcg(pp + c * pstride + 1);
-      if (lc > 0.0f) {
-        const float f = expf(__ldcg(pp + c * pstride) - m);
-        den = fmaf(f, lc, den);
-        num = fmaf(f, __ldcg(pp + c * pstride + 2 + d), num);
+      float f;
+      if (c < kMergeSmem) {
+        f = s_f[h * kMergeSmem + c];
+      } else {
+        const float lc = __ldcg(pp + c * pstride + 1);
+        f = lc > 0.0f ? expf(__ldcg(pp + c * pstride) - m) : 0.0f;
       }
+      num = fmaf(f, __ldcg(pp + c * pstride + 2 + d), num);
     }
     a.out[(static_cast<int64_t>(b) * a.Hq + h0 + h) * kKvD + d] = __float2half_rn(den > 0.0f ? num / den : 0.0f);
   }
