@@ -187,11 +187,13 @@ struct GemmCfg {
   // their last MMA and start the weight stream after the set-up (measured
   // faster for their long launches).
   static constexpr bool kEarlyStart = BN <= 32;
-  // Weight chunks requested at kernel entry. Two, not the whole ring: when
-  // every CTA of a launch requests its whole ring at once, the first chunk of
-  // each waits behind everyone's burst in the memory queues (measured: a
-  // full-ring start delayed the first weight bytes by ~1 us per launch).
-  static constexpr int kStartChunks = kEarlyStart ? (NS < 2 ? NS : 2) : 0;
+  // Weight chunks requested at kernel entry, before the set-up. None: the
+  // weight stream starts after the set-up. Measured on the decode step: two
+  // chunks at entry 203.0 us per step, one 204.4, none 201.1 (the activation
+  // tile, requested after the dependency wait, lands sooner behind fewer
+  // queued weight bytes); the whole ring at entry delayed every CTA's first
+  // weight bytes by about 1 us.
+  static constexpr int kStartChunks = 0;
   static constexpr int kTmemA = NACC * BN;  // accumulators first, then the TMEM weight ring
   static constexpr int kTSlotCols = KS * kKbCols;
   // tensor memory columns allocated (a power of two >= 32)
