@@ -927,10 +927,13 @@ def main_kv(args, world, rank, local):
                    "tokens": int(np.sum(lens)), "layers_per_step": KV_LAYERS,
                    "l2": f"inputs larger than L2: {KV_LAYERS} layer caches, {cache_b / 1e6:.0f} MB per step",
                    "parallelism": f"replicas x{world}"},
-        "gpu_launches": 3 * KV_LAYERS * args.steps,
+        # per layer: the append's two quantizer launches, the attention's two
+        # (partial results per chunk, then the merge)
+        "gpu_launches": 4 * KV_LAYERS * args.steps,
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": None,
-                     "peak_source": f"{peaks['source']} HBM copy", "kernel": "kv4_decode_kernel",
+                     "peak_source": f"{peaks['source']} HBM copy",
+                     "kernel": "kv4_decode_kernel + kv4_merge_kernel (one attention call)",
                      "avg_launch_us": round(attn_launch_ms * 1e3, 3)},
         "e2e": {"value": round(world * cache_b / (r["e2e_ms"] / args.steps * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"]},

@@ -454,7 +454,9 @@ W4A8_API w4a8_status_t w4kv_append(const void* K_new, const void* V_new, const i
                                    int64_t Hkv, int64_t Lmax, int32_t D, uint8_t* k_codes, uint32_t* k_params,
                                    uint8_t* v_codes, uint32_t* v_params, w4a8_stream_t stream);
 
-/* Workspace bytes of w4kv_attention_decode (0 if the shape is unsupported). */
+/* Workspace bytes of w4kv_attention_decode (0 if the shape is unsupported):
+ * one partial result (2 + 128 floats) per (sequence, query head, chunk of 128
+ * cache positions). */
 W4A8_API size_t w4kv_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lmax, int32_t D);
 
 /*
@@ -464,9 +466,13 @@ W4A8_API size_t w4kv_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hk
  * outside [0, Lmax] is clamped and recorded as W4A8_DEVERR_KV_RANGE).
  * Limits: D == 128, Hkv >= 1, Hq % Hkv == 0, Hq <= 65536, 1 <= Lmax <= 2^24,
  * B <= 65535. workspace: 256-byte aligned, at least
- * w4kv_attention_workspace_bytes(...) bytes, zero-filled before its first
- * use; the call leaves its first part (the per-head-group tickets) zero again.
- * Calls that share a workspace must not overlap on the GPU.
+ * w4kv_attention_workspace_bytes(...) bytes, any contents (it holds the
+ * chunks' partial results between the call's two kernels). Calls that share a
+ * workspace must not overlap on the GPU. Both contractions run on tensor
+ * cores with fp32 accumulation: the scores from fp16 q and the exact small
+ * integers code - z, the weighted values from the same integers (bf16) and
+ * the softmax weights split into three bf16 terms (relative error below
+ * 2^-24), within the fp32 evaluation bound above.
  */
 W4A8_API w4a8_status_t w4kv_attention_decode(const void* q, const uint8_t* k_codes, const uint32_t* k_params,
                                              const uint8_t* v_codes, const uint32_t* v_params,

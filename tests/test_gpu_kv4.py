@@ -5,7 +5,7 @@ Bars: codes and parameter words bit-exact (the quantizer's integer
 decisions are taken in fp32 with IEEE divides on both sides); attention
 output within half an fp16 ulp of the exact result plus the oracle's fp32
 evaluation bound; repeated launches bit-identical (the chunk merge runs in
-a fixed order); the workspace tickets left zero.
+a fixed order), whatever the workspace held before.
 """
 import numpy as np
 import pytest
@@ -118,7 +118,10 @@ def test_kv4_attention_within_the_bound(Hq, Hkv, lens):
     q, kc, kp, vc, vp = make_cache(3, Hq, Hkv, 300, I.seed_of("t-kva", Hq, Hkv))
     Y, ws = run(q, kc, kp, vc, vp, lens)
     check(Y, q, kc, kp, vc, vp, lens)
-    assert not host(ws)[:256].any(), "tickets must be left zero"
+    # a workspace full of garbage gives the same bits
+    ws.fill_(0xA7)
+    Y2, _ = run(q, kc, kp, vc, vp, lens, ws)
+    assert np.array_equal(Y.view(np.uint16), Y2.view(np.uint16))
 
 
 def test_kv4_attention_padding_is_not_read():
@@ -163,7 +166,6 @@ def test_kv4_repeated_launches_bit_identical():
             bad += (o.view(torch.int16) != ref).any()
     torch.cuda.synchronize()
     assert int(bad) == 0
-    assert not host(ws)[:256].any()
 
 
 def test_kv4_length_out_of_range_is_clamped_and_reported():

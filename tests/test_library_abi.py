@@ -178,7 +178,7 @@ def test_kv4_validation(L):
     assert q(FAKE_ODD, 4, 128, FAKE, FAKE, None) == 3
     assert q(None, 0, 128, None, None, None) == 0                         # n == 0: no-op
     ws = L.w4kv_attention_workspace_bytes
-    assert ws(2, 32, 8, 4096, 128) == 256 + 2 * 32 * 16 * 130 * 4         # tickets, then partials
+    assert ws(2, 32, 8, 4096, 128) == 2 * 32 * 32 * 130 * 4               # partials of 128-token chunks
     assert ws(2, 6, 4, 4096, 128) == 0                                    # Hq % Hkv
     assert ws(2, 32, 8, 4096, 64) == 0                                    # D
     a = L.w4kv_attention_decode

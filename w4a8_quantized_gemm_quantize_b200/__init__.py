@@ -576,8 +576,8 @@ _kv_ws = {}
 
 
 def _kv_workspace_for(device, nbytes: int):
-    """A zero-filled workspace per device, grown on demand and reused: the
-    attention call leaves the part it must find zero (its tickets) zero."""
+    """A workspace per device for the chunks' partial results, grown on
+    demand and reused (any contents will do)."""
     torch = _torch()
     key = str(device)
     ws = _kv_ws.get(key)

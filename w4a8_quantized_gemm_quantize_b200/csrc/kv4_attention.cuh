@@ -19,26 +19,23 @@
 // exponentiates against the chunk's own maximum and accumulates the weighted
 // values; the last CTA of a (sequence, kv head, head group) to finish (a
 // ticket in the workspace, no waiting) merges the chunks' partial results
-// with exp(m_chunk - m) factors and writes Y. The scores and the weighted
-// sums run on CUDA cores in fp32, about 14 operations per cache byte for four
-// query heads per kv head, so at that grouping the arithmetic, not HBM, is
-// expected to set the pace.
-//
-// Mapping inside a CTA (both phases): the chunk's K and V codes are staged in
-// shared memory by two bulk copies issued at the start (all 2 x n x 64 bytes
-// in flight at once); 8 lanes per token, lane slice li owns elements
-// [16 li, 16 li + 16) (8 code bytes), so a warp reads 4 consecutive tokens =
-// 256 contiguous bytes of shared memory per step. Products of an fp16 query
-// element and a small integer (code - z) are exact in fp32.
+// with exp(m_chunk - m) factors and writes Y. Both contractions (the scores
+// and the weighted values) run on the tensor cores (tcgen05 kind::f16, fp32
+// accumulation); the CUDA cores only unpack the codes (about one operation
+// per code) and take the softmax. A CTA takes one chunk of 128 tokens, four
+// CTAs share an SM; a second kernel merges the chunks of each (sequence,
+// query head).
 #pragma once
+#include <cuda_bf16.h>
+
 #include "ptx.cuh"
 
 namespace w4a8 {
 
 constexpr int kKvD = 128;              // head dimension
 constexpr int kKvRowBytes = kKvD / 2;  // packed codes of one cached vector
-constexpr int kKvChunk = 256;          // tokens per CTA
-constexpr int kKvThreads = 256;        // 8 warps
+constexpr int kKvChunk = 128;          // tokens per CTA (one M = 128 tile)
+constexpr int kKvThreads = 256;        // 8 warps (the quantizer)
 constexpr int kKvWarps = kKvThreads / 32;
 constexpr int kErrKvRange = 7;         // W4A8_DEVERR_KV_RANGE
 constexpr int kErrKvWait = 11;         // W4A8_DEVERR_KV_WAIT
@@ -117,264 +114,418 @@ struct KvAttnArgs {
   const int32_t* seq_lens; // [B]
   __half* out;             // [B, Hq, 128]
   float* part;             // [B, Hq, nsplit, 2 + 128]: chunk max, chunk sum, weighted values
-  int32_t* tickets;        // [B, Hkv, Hq / Hkv / GC], zero between launches
-  int Hq, Hkv, nsplit;
+  int B, Hq, Hkv, nsplit, groups;  // groups: head groups (of GC query heads) per kv head
   int64_t Lmax;
   float scale;
   int* err;
 };
 
-// (code - z) for the 16 codes of an 8-byte slice, exact: the code is placed
-// in the mantissa of 2^23 (0x4B000000 | c = 2^23 + c) and 2^23 + z subtracted.
-__device__ __forceinline__ void kv_unpack16(uint2 w, float bias, float (&x)[16]) {
-  const uint32_t ww[2] = {w.x, w.y};
+constexpr int kKvAttnThreads = 256;      // 8 warps: thread = (token, half of the head dimension)
+constexpr int kKvPartStride = 2 + kKvD;  // floats per partial result
+
+// Shared-memory layout of one attention CTA (offsets from a 1024-byte aligned
+// base), sized for four CTAs per SM. The MMA operands built here use the
+// 128-byte swizzle: within every 1024-byte atom of eight 128-byte rows, the
+// 16-byte chunk c of row r sits at chunk position c ^ (r & 7).
+struct KvSmem {
+  static constexpr int kCodes = kKvChunk * kKvRowBytes;   // one matrix's codes of the chunk (8 KB)
+  static constexpr int kPlane = kKvChunk * 128;           // 64 values x 2 bytes per token row
+  static constexpr int kOpBlock = 16 * 128;               // one 64-column block of an N = 16 operand
+  static constexpr int kOffVpl = 0;                       // V values, two planes (d 0-63, 64-127)
+  static constexpr int kOffKc = kOffVpl + 2 * kPlane;     // K codes (bulk copy); later the weights
+  static constexpr int kOffW = kOffKc;                    // (two blocks: tokens 0-63, 64-127)
+  static constexpr int kOffVc = kOffKc + kCodes;          // V codes (bulk copy)
+  static constexpr int kOffQ = kOffVc + kCodes;           // q: two blocks (d 0-63, 64-127)
+  static constexpr int kOffScale = kOffQ + 2 * kOpBlock;  // per token (s^K, s^V)
+  static constexpr int kOffZ = kOffScale + kKvChunk * 8;  // per token the z bits (K, V)
+  static constexpr int kOffRed = kOffZ + kKvChunk * 4;    // [warp][head] max, then sum
+  static constexpr int kOffMisc = kOffRed + 2 * 8 * 4 * 4;  // barriers, TMEM address, (m, l)
+  static constexpr int kBytes = kOffMisc + 64 + 1024;       // + alignment slack
+  static_assert(kOffKc % 1024 == 0 && kOffQ % 1024 == 0 && kOffW % 1024 == 0, "swizzle atoms 1024-aligned");
+  static_assert(2 * kOpBlock <= kCodes, "the weights fit in the spent K codes");
+  static_assert(kBytes + 1024 <= 232448 / 4, "four CTAs per SM");
+};
+
+// TMEM columns of one CTA: the dequantized K operand (64 columns of fp16
+// pairs), the scores (16 fp32 columns) and the weighted values (16).
+constexpr int kKvTmemK = 0, kKvTmemS = 64, kKvTmemO = 80, kKvTmemCols = 128;
+
+// Position p (0..7) of an 8-value group of a dequantized row holds element
+// kv_perm8(p) of the group: the unpacking below forms the pairs (e, e + 4)
+// of the eight 4-bit codes of one 32-bit word.
+__host__ __device__ constexpr int kv_perm8(int p) { return (p >> 1) + 4 * (p & 1); }
+
+// (code - z) of the eight codes of word w as four fp16 pairs, exact: a code
+// in bits 0-3 of a half goes into the mantissa of 1024 (0x6400 | c = 1024 +
+// c) and bias = -(1024 + z) is added; one in bits 4-7 gives 1024 + 16 c,
+// scaled by 1/16 in the fused multiply-add that adds bias16 = -(64 + z).
+// Pair e holds elements (e, e + 4).
+__device__ __forceinline__ void kv_unpack8_f16(uint32_t w, __half2 bias, __half2 bias16, uint32_t (&o)[4]) {
+  const __half2 sixteenth = __float2half2_rn(0.0625f);
+  const uint32_t w8 = w >> 8;
+  const uint32_t x[4] = {(w & 0x000F000Fu) | 0x64006400u, (w & 0x00F000F0u) | 0x64006400u,
+                         (w8 & 0x000F000Fu) | 0x64006400u, (w8 & 0x00F000F0u) | 0x64006400u};
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
+  for (int e = 0; e < 4; ++e) {
+    const __half2 h = *reinterpret_cast<const __half2*>(&x[e]);
+    const __half2 v = (e & 1) ? __hfma2(h, sixteenth, bias16) : __hadd2(h, bias);
+    o[e] = *reinterpret_cast<const uint32_t*>(&v);
+  }
+}
+// The same as bf16 pairs (0x4300 | c = 128 + c; bf16 keeps 7 mantissa bits,
+// so every code is shifted down to bits 0-3 first).
+__device__ __forceinline__ void kv_unpack8_bf16(uint32_t w, __nv_bfloat162 bias, uint32_t (&o)[4]) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) x[8 * k + e] = __uint_as_float(0x4B000000u | ((ww[k] >> (4 * e)) & 0xFu)) - bias;
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t x = ((w >> (4 * e)) & 0x000F000Fu) | 0x43004300u;
+    const __nv_bfloat162 v = __hsub2(*reinterpret_cast<const __nv_bfloat162*>(&x), bias);
+    o[e] = *reinterpret_cast<const uint32_t*>(&v);
   }
 }
 
-__device__ __forceinline__ void kv_param(uint32_t p, float& s, float& bias) {
-  s = __half2float(__ushort_as_half(static_cast<unsigned short>(p & 0xFFFFu)));
-  bias = 8388608.0f + __half2float(__ushort_as_half(static_cast<unsigned short>(p >> 16)));
+// Byte offset of element (row, col) of an N = 16 operand whose 64-column
+// blocks are kOpBlock apart (16-bit elements, 128-byte swizzle).
+__device__ __forceinline__ int kv_op_offset(int row, int col) {
+  const int c = (col & 63) >> 3;
+  return (col >> 6) * KvSmem::kOpBlock + row * 128 + ((c ^ (row & 7)) << 4) + ((col & 7) << 1);
 }
 
+// Decode attention on tensor cores. A CTA takes up to kKvChunk = 128 tokens
+// of one (sequence, kv head) for GC of its query heads (a chunk without
+// tokens only writes its empty partial result):
+//  * the chunk's K and V codes arrive in shared memory by two bulk copies,
+//    issued first;
+//  * thread (token j, half hf) unpacks token j's K values of half hf, code -
+//    z as fp16 (exact small integers), into TMEM lane j (the A operand of the
+//    scores) and its V values as bf16 into row j of shared-memory plane hf;
+//  * one thread issues S = K^ q^T: M = 128 tokens, N = 16 (the GC query
+//    heads, fp16, the other rows zero), K = 128, fp32 accumulation: the
+//    products of an fp16 query element and a small integer are exact;
+//  * the threads read the scores of their token (heads hf, hf + 2),
+//    s_j = scale * (s^K_j * S_j), take the chunk maximum and sum per head and
+//    write the weights w_j = exp(s_j - m) s^V_j as three bf16 terms (w = t0 +
+//    t1 + t2 up to 2^-24 relative: t0 = bf16(w), t1 = bf16(w - t0), t2 =
+//    bf16(w - t0 - t1), the differences exact in fp32);
+//  * one thread issues O = V^T W^T: M = 128 (the head dimension, V read
+//    MN-major from the planes), N = 16 (three terms x GC heads), K = 128
+//    tokens, products exact in fp32 (bf16 x small integer), fp32 sums;
+//  * the threads read O, add the three terms of each head and write the
+//    chunk's partial result (m, l, O); kv4_merge_kernel combines the chunks.
+// The unpacking permutes each 8-value group of the head dimension
+// (kv_perm8): q is staged in the same order, and row p of O is element
+// 8 (p / 8) + kv_perm8(p % 8). Every wait is bounded.
 template <int GC>
-__global__ void __launch_bounds__(kKvThreads) kv4_decode_kernel(KvAttnArgs a) {
+__global__ void __launch_bounds__(kKvAttnThreads, 4) kv4_decode_kernel(KvAttnArgs a) {
   static_assert(GC == 1 || GC == 2 || GC == 4, "query heads per CTA");
-  // the chunk's K and V codes, staged by two bulk copies (kKvChunk x 64 bytes
-  // each); once the scores are done the K codes' space holds the per-warp
-  // weighted values (s_o)
-  constexpr int kKcBytes = kKvChunk * kKvRowBytes;
-  constexpr int kOBytes = kKvWarps * GC * kKvD * 4;
-  static_assert(kOBytes <= kKcBytes, "the weighted values fit in the K codes' space");
-  __shared__ __align__(128) uint8_t s_kc[kKcBytes];
-  __shared__ __align__(128) uint8_t s_vc[kKvChunk * kKvRowBytes];
-  __shared__ float2 s_kpar[kKvChunk];  // per token: (s, 2^23 + z)
-  __shared__ float2 s_vpar[kKvChunk];
-  __shared__ uint64_t s_bar;
-  __shared__ float s_q[GC][kKvD];
-  __shared__ float s_p[GC][kKvChunk];
-  __shared__ float s_m[GC], s_l[GC];
-  float(*s_o)[GC][kKvD] = reinterpret_cast<float(*)[GC][kKvD]>(s_kc);
-  __shared__ int s_last;
+  extern __shared__ __align__(1024) uint8_t kv_smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(kv_smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* s_vpl = sm + KvSmem::kOffVpl;
+  uint8_t* s_kc = sm + KvSmem::kOffKc;
+  uint8_t* s_vc = sm + KvSmem::kOffVc;
+  uint8_t* s_q = sm + KvSmem::kOffQ;
+  uint8_t* s_w = sm + KvSmem::kOffW;
+  float2* s_scale = reinterpret_cast<float2*>(sm + KvSmem::kOffScale);
+  uint32_t* s_z = reinterpret_cast<uint32_t*>(sm + KvSmem::kOffZ);  // z bits: K low half, V high half
+  float* s_rmax = reinterpret_cast<float*>(sm + KvSmem::kOffRed);   // [warp][head]
+  float* s_rsum = s_rmax + 32;
+  uint64_t* bar_ld = reinterpret_cast<uint64_t*>(sm + KvSmem::kOffMisc);
+  uint64_t* bar_mma = bar_ld + 1;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(bar_ld + 2);
+  float* s_m = reinterpret_cast<float*>(s_tmem + 1);  // [4]
+  float* s_l = s_m + 4;                               // [4]
 
   const int split = blockIdx.x;
   const int hg = blockIdx.y;  // (kv head, head group)
   const int b = blockIdx.z;
-  const int G = a.Hq / a.Hkv;
-  const int groups = G / GC;
-  const int g = hg / groups;
-  const int h0 = g * G + (hg % groups) * GC;  // first query head of this CTA
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int grp = lane >> 3, li = lane & 7;
+  const int g = hg / a.groups;
+  const int h0 = g * (a.Hq / a.Hkv) + (hg % a.groups) * GC;  // first query head of this CTA
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int qd = warp & 3, hf = warp >> 2;  // TMEM lane quarter, half of the head dimension / head pair
+  const int j = qd * 32 + lane;             // this thread's token (and TMEM lane)
+  const DevErr err{a.err};
 
-  if (threadIdx.x == 0) {
-    mbar_init(&s_bar, 1);
-    fence_barrier_init();
-  }
-  grid_dependency_wait();  // q and the cache come from the preceding kernels
+  grid_dependency_wait();  // q, the cache and the lengths come from the preceding kernels
   grid_launch_dependents();
-
-  int L = a.seq_lens[b];
+  int L = __ldg(a.seq_lens + b);
   if (L < 0 || L > a.Lmax) {
-    if (threadIdx.x == 0 && split == 0) atomicCAS(a.err, 0, kErrKvRange);
+    if (t == 0 && split == 0) atomicCAS(a.err, 0, kErrKvRange);
     L = L < 0 ? 0 : static_cast<int>(a.Lmax);
   }
   const int t0 = split * kKvChunk;
   const int n = max(0, min(L - t0, kKvChunk));  // tokens of this chunk
+  const int64_t pbase = (static_cast<int64_t>(b) * a.Hq + h0) * a.nsplit + split;  // head h0's partial
+  if (n == 0) {
+    // no tokens: the empty partial result (m = -inf, l = 0, O = 0)
+    for (int i = t; i < GC * kKvPartStride; i += kKvAttnThreads) {
+      const int h = i / kKvPartStride, e = i % kKvPartStride;
+      a.part[(pbase + static_cast<int64_t>(h) * a.nsplit) * kKvPartStride + e] = e == 0 ? -INFINITY : 0.0f;
+    }
+    return;
+  }
   const int64_t cache_row0 = (static_cast<int64_t>(b) * a.Hkv + g) * a.Lmax + t0;
-  __syncthreads();  // the barrier is initialized
-  // The chunk's codes are contiguous in the cache (64 bytes per token, rows
-  // 64-byte aligned): two bulk copies put all of them in flight at once, so
-  // the CTA streams its 2 x 16 KB instead of waiting once per token step.
-  if (threadIdx.x == 0 && n > 0) {
+  if (t == 0) {
+    // the chunk's codes are contiguous in the cache (64 bytes per token):
+    // two bulk copies put all of them in flight before anything else
+    mbar_init(bar_ld, 1);
+    mbar_init(bar_mma, 1);
+    fence_barrier_init();
     const uint64_t pol = l2_policy_evict_first();
-    mbar_arrive_expect_tx(&s_bar, 2u * n * kKvRowBytes);
-    bulk_load(s_kc, a.kc + cache_row0 * kKvRowBytes, n * kKvRowBytes, &s_bar, pol);
-    bulk_load(s_vc, a.vc + cache_row0 * kKvRowBytes, n * kKvRowBytes, &s_bar, pol);
+    mbar_arrive_expect_tx(bar_ld, 2u * n * kKvRowBytes);
+    bulk_load(s_kc, a.kc + cache_row0 * kKvRowBytes, n * kKvRowBytes, bar_ld, pol);
+    bulk_load(s_vc, a.vc + cache_row0 * kKvRowBytes, n * kKvRowBytes, bar_ld, pol);
   }
-  // parameter words (4 bytes per token: no 16-byte alignment to rely on) by plain loads
-  for (int j = threadIdx.x; j < n; j += kKvThreads) {
-    float sk, bk, sv, bv;
-    kv_param(__ldg(a.kp + cache_row0 + j), sk, bk);
-    kv_param(__ldg(a.vp + cache_row0 + j), sv, bv);
-    s_kpar[j] = make_float2(sk, bk);
-    s_vpar[j] = make_float2(sv, bv);
+  if (warp == 0) {
+    tmem_alloc(s_tmem, kKvTmemCols);
+    tmem_relinquish();
   }
-  for (int i = threadIdx.x; i < GC * kKvD; i += kKvThreads)
-    s_q[i / kKvD][i % kKvD] = __half2float(a.q[(static_cast<int64_t>(b) * a.Hq + h0 + i / kKvD) * kKvD + i % kKvD]);
-  __syncthreads();
-  if (n > 0 && !mbar_wait_limit(&s_bar, 0, nullptr, DevErr{a.err}, kErrKvWait, kWaitLimitNs)) {
-    // the copies did not land in time (recorded): no result for this chunk
-    // beyond zeros, and no exit while copies may still be in flight
-    mbar_wait_limit(&s_bar, 0, nullptr, DevErr{a.err}, kErrKvWait, kWaitLimitNs);
+  // q's operand: rows 0..GC-1 the heads' queries in the unpack order of the
+  // head dimension, the other rows zero
+  for (int i = t; i < 2 * KvSmem::kOpBlock / 16; i += kKvAttnThreads)
+    reinterpret_cast<uint4*>(s_q)[i] = make_uint4(0u, 0u, 0u, 0u);
+  // per-token scales and z bits (plain loads: 4 bytes per token); tokens past
+  // the chunk get s = 0, z = 0
+  {
+    const int jj = t & (kKvChunk - 1);
+    const uint32_t* src = t < kKvChunk ? a.kp : a.vp;
+    const uint32_t p = jj < n ? __ldg(src + cache_row0 + jj) : 0u;
+    reinterpret_cast<float*>(s_scale)[2 * jj + (t < kKvChunk ? 0 : 1)] =
+        __half2float(__ushort_as_half(static_cast<unsigned short>(p & 0xFFFFu)));
+    reinterpret_cast<uint16_t*>(s_z)[2 * jj + (t < kKvChunk ? 0 : 1)] = static_cast<uint16_t>(p >> 16);
+  }
+  __syncthreads();  // zeroed before the queries are placed
+  for (int i = t; i < GC * kKvD; i += kKvAttnThreads) {
+    const int h = i / kKvD, p = i % kKvD;
+    const int d = (p & ~7) + kv_perm8(p & 7);
+    *reinterpret_cast<__half*>(s_q + kv_op_offset(h, p)) =
+        a.q[(static_cast<int64_t>(b) * a.Hq + h0 + h) * kKvD + d];
+  }
+  tc_fence_before();
+  __syncthreads();  // barriers, TMEM address, scales staged
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t lane_base = static_cast<uint32_t>(qd * 32) << 16;
+  if (!mbar_wait_limit(bar_ld, 0, nullptr, err, kErrKvWait, kWaitLimitNs)) {
+    // the copies did not land in time (recorded): no exit while they may
+    // still be in flight
+    mbar_wait_limit(bar_ld, 0, nullptr, err, kErrKvWait, kWaitLimitNs);
   }
 
-  // ---- scores: s_p[h][j] = scale * (s^K_j * sum_d q[d] (code - z))
+  // ---- unpack: thread (token j, half hf)
   {
-    float qr[GC][16];
+    const uint32_t zz = s_z[j];
+    const __half kz = __ushort_as_half(static_cast<unsigned short>(zz & 0xFFFFu));
+    const __half kb1 = __hadd(__float2half_rn(1024.0f), kz);
+    const __half kb16 = __hadd(__float2half_rn(64.0f), kz);
+    const __half2 kbias = __halves2half2(__hneg(kb1), __hneg(kb1));
+    const __half2 kbias16 = __halves2half2(__hneg(kb16), __hneg(kb16));
+    const __nv_bfloat16 vzb = __float2bfloat16_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(zz >> 16))));
+    const __nv_bfloat16 vb1 = __hadd(__float2bfloat16_rn(128.0f), vzb);
+    const __nv_bfloat162 vbias = __halves2bfloat162(vb1, vb1);
+    // the 32 code bytes of this half, read in an order that spreads the
+    // banks (rows are 64 bytes: lanes two tokens apart share banks)
+    const int rot = (j >> 1) & 1;
+    const int base = j * kKvRowBytes + hf * 32;
+    const uint4 ka = *reinterpret_cast<const uint4*>(s_kc + base + rot * 16);
+    const uint4 kb = *reinterpret_cast<const uint4*>(s_kc + base + (rot ^ 1) * 16);
+    const uint4 vx = *reinterpret_cast<const uint4*>(s_vc + base + rot * 16);
+    const uint4 vy = *reinterpret_cast<const uint4*>(s_vc + base + (rot ^ 1) * 16);
+    const uint4 k0 = rot ? kb : ka, k1 = rot ? ka : kb, v0 = rot ? vy : vx, v1 = rot ? vx : vy;
+    const uint32_t kws[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+    const uint32_t vws[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint8_t* row = s_vpl + hf * KvSmem::kPlane + j * 128;
 #pragma unroll
-    for (int h = 0; h < GC; ++h)
-#pragma unroll
-      for (int e = 0; e < 16; ++e) qr[h][e] = s_q[h][16 * li + e];
-    for (int j0 = warp * 4; j0 < n; j0 += kKvWarps * 4) {
-      const int j = j0 + grp;
-      const bool valid = j < n;
-      uint2 w = make_uint2(0u, 0u);
-      float2 par = make_float2(0.0f, 8388608.0f);
-      if (valid) {
-        w = *reinterpret_cast<const uint2*>(s_kc + j * kKvRowBytes + li * 8);
-        par = s_kpar[j];
-      }
-      const float sk = par.x, bias = par.y;
-      float x[16];
-      kv_unpack16(w, bias, x);
-      float acc[GC];
-#pragma unroll
-      for (int h = 0; h < GC; ++h) {
-        acc[h] = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) acc[h] = fmaf(qr[h][e], x[e], acc[h]);
-      }
-#pragma unroll
-      for (int h = 0; h < GC; ++h) {
-        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 1);
-        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 2);
-        acc[h] += __shfl_xor_sync(0xffffffffu, acc[h], 4);
-      }
-      if (valid && li == 0) {
-#pragma unroll
-        for (int h = 0; h < GC; ++h) s_p[h][j] = (sk * acc[h]) * a.scale;
-      }
+    for (int wi = 0; wi < 8; ++wi) {
+      uint32_t o[4];
+      kv_unpack8_bf16(vws[wi], vbias, o);
+      *reinterpret_cast<uint4*>(row + ((wi ^ (j & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
     }
+    uint32_t kr[32];
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      uint32_t o[4];
+      kv_unpack8_f16(kws[wi], kbias, kbias16, o);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) kr[4 * wi + e] = o[e];
+    }
+    tmem_st_32(tmem + kKvTmemK + 32 * hf + lane_base, kr);
   }
+  tmem_wait_st();
+  fence_proxy_async_smem();  // the generic-proxy operand stores, before the MMAs read them
+  tc_fence_before();
   __syncthreads();
-  // ---- softmax over the chunk: warp h handles head h
-  if (warp < GC) {
-    float m = -INFINITY;
-    for (int j = lane; j < n; j += 32) m = fmaxf(m, s_p[warp][j]);
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float l = 0.0f;
-    for (int j = lane; j < n; j += 32) {
-      const float e = expf(s_p[warp][j] - m);
-      s_p[warp][j] = e;
-      l += e;
+  tc_fence_after();
+  if (t == 0) {
+    // S[token, head] = sum_d K^[token, d] q[head, d]
+    constexpr uint32_t idesc = idesc_f16(128, 16);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint64_t bdesc = smem_desc_k128_sw128(smem_u32(s_q) + (kk >> 2) * KvSmem::kOpBlock + (kk & 3) * 32);
+      mma_f16_ts(tmem + kKvTmemS, tmem + kKvTmemK + kk * 8, bdesc, idesc, kk > 0 ? 1u : 0u);
     }
-    for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
-    if (lane == 0) {
-      s_m[warp] = m;
-      s_l[warp] = l;
-    }
+    mma_commit(bar_mma);
   }
-  __syncthreads();
-  // ---- weighted values: lane (grp, li) sums its tokens for elements 16 li ..
+  if (!mbar_wait_limit(bar_mma, 0, nullptr, err, kErrKvWait, kWaitLimitNs))
+    mbar_wait_limit(bar_mma, 0, nullptr, err, kErrKvWait, kWaitLimitNs);
+  tc_fence_after();
+
+  // ---- softmax over the chunk: thread (token j, heads hf and hf + 2)
+  constexpr int kHp = GC >= 2 ? GC / 2 : 1;  // heads per thread
+  const bool active = hf < GC;               // (GC == 1: the second half has no head)
   {
-    float o[GC][16];
+    uint32_t sv[16];
+    tmem_ld_16_wait(tmem + kKvTmemS + lane_base, sv);
+    const bool valid = j < n;
+    const float2 sc = s_scale[j];
+    float s[kHp], m[kHp], e[kHp];
 #pragma unroll
-    for (int h = 0; h < GC; ++h)
+    for (int k = 0; k < kHp; ++k) {
+      const int h = hf + 2 * k;
+      // column h = hf + 2k of the scores (selected without indexing by hf)
+      const float sk = __uint_as_float(hf ? sv[(1 + 2 * k) & 3] : sv[(2 * k) & 3]);
+      s[k] = (valid && active && h < GC) ? (sc.x * sk) * a.scale : -INFINITY;
+      m[k] = s[k];
+      for (int o = 16; o > 0; o >>= 1) m[k] = fmaxf(m[k], __shfl_xor_sync(0xffffffffu, m[k], o));
+      if (lane == 0) s_rmax[warp * 4 + k] = m[k];
+    }
+    __syncthreads();
 #pragma unroll
-      for (int e = 0; e < 16; ++e) o[h][e] = 0.0f;
-    for (int j0 = warp * 4; j0 < n; j0 += kKvWarps * 4) {
-      const int j = j0 + grp;
-      if (j < n) {
-        const uint2 w = *reinterpret_cast<const uint2*>(s_vc + j * kKvRowBytes + li * 8);
-        const float sv = s_vpar[j].x, bias = s_vpar[j].y;
-        float x[16];
-        kv_unpack16(w, bias, x);
+    for (int k = 0; k < kHp; ++k) {
+      const int w0 = hf * 4;  // the four warps of this head pair
+      m[k] = fmaxf(fmaxf(s_rmax[(w0 + 0) * 4 + k], s_rmax[(w0 + 1) * 4 + k]),
+                   fmaxf(s_rmax[(w0 + 2) * 4 + k], s_rmax[(w0 + 3) * 4 + k]));
+      e[k] = (valid && active) ? expf(s[k] - m[k]) : 0.0f;
+      float l = e[k];
+      for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+      if (lane == 0) s_rsum[warp * 4 + k] = l;
+    }
+    // the weights w = e s^V as three bf16 terms: rows term * 4 + head of the
+    // values' B operand, column = token (written over the spent K codes)
+    if (active) {
 #pragma unroll
-        for (int h = 0; h < GC; ++h) {
-          const float wgt = s_p[h][j] * sv;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[h][e] = fmaf(wgt, x[e], o[h][e]);
-        }
+      for (int k = 0; k < kHp; ++k) {
+        const int h = hf + 2 * k;
+        if (h >= GC) break;
+        const float wt = e[k] * sc.y;
+        const __nv_bfloat16 w0 = __float2bfloat16_rn(wt);
+        const float r1 = wt - __bfloat162float(w0);
+        const __nv_bfloat16 w1 = __float2bfloat16_rn(r1);
+        const __nv_bfloat16 w2 = __float2bfloat16_rn(r1 - __bfloat162float(w1));
+        *reinterpret_cast<__nv_bfloat16*>(s_w + kv_op_offset(h, j)) = w0;
+        *reinterpret_cast<__nv_bfloat16*>(s_w + kv_op_offset(4 + h, j)) = w1;
+        *reinterpret_cast<__nv_bfloat16*>(s_w + kv_op_offset(8 + h, j)) = w2;
       }
     }
-    // the four token groups of the warp, then the warps
+    // (rows of the weights' operand beyond the heads keep the spent codes:
+    // they only reach columns of O that are not read)
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (t < GC) {
+    const int k = t >> 1, w0 = (t & 1) * 4;  // head t: pair t & 1, slot t >> 1
+    s_m[t] = fmaxf(fmaxf(s_rmax[(w0 + 0) * 4 + k], s_rmax[(w0 + 1) * 4 + k]),
+                   fmaxf(s_rmax[(w0 + 2) * 4 + k], s_rmax[(w0 + 3) * 4 + k]));
+    s_l[t] = (s_rsum[(w0 + 0) * 4 + k] + s_rsum[(w0 + 1) * 4 + k]) +
+             (s_rsum[(w0 + 2) * 4 + k] + s_rsum[(w0 + 3) * 4 + k]);
+  }
+  if (t == 0) {
+    // O[d, n] = sum_token V^[token, d] W[n, token]: A = the V planes read
+    // MN-major (64-value atoms along d: the second plane at +kPlane; 8-token
+    // groups 1024 bytes apart), B = the weights, K-major
+    constexpr uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | (2u << 17) | (8u << 24);
 #pragma unroll
-    for (int h = 0; h < GC; ++h)
+    for (int kk = 0; kk < 8; ++kk) {
+      const uint64_t adesc = smem_desc_mn_sw128(smem_u32(s_vpl) + kk * 2048, KvSmem::kPlane, 1024);
+      const uint64_t bdesc = smem_desc_k128_sw128(smem_u32(s_w) + (kk >> 2) * KvSmem::kOpBlock + (kk & 3) * 32);
+      mma_f16_ss(tmem + kKvTmemO, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(bar_mma);
+  }
+  if (!mbar_wait_limit(bar_mma, 1, nullptr, err, kErrKvWait, kWaitLimitNs))
+    mbar_wait_limit(bar_mma, 1, nullptr, err, kErrKvWait, kWaitLimitNs);
+  tc_fence_after();
+
+  // ---- the chunk's partial result: thread (output row j, heads hf, hf + 2)
+  {
+    uint32_t ov[16];
+    tmem_ld_16_wait(tmem + kKvTmemO + lane_base, ov);
+    const int d = (j & ~7) + kv_perm8(j & 7);
 #pragma unroll
-      for (int e = 0; e < 16; ++e) {
-        o[h][e] += __shfl_xor_sync(0xffffffffu, o[h][e], 8);
-        o[h][e] += __shfl_xor_sync(0xffffffffu, o[h][e], 16);
+    for (int k = 0; k < kHp; ++k) {
+      const int h = hf + 2 * k;
+      if (h >= GC) break;
+      float* pp = a.part + (pbase + static_cast<int64_t>(h) * a.nsplit) * kKvPartStride;
+      const int c0 = 2 * k;  // columns term * 4 + h, selected without indexing by hf
+      const float o0 = __uint_as_float(hf ? ov[c0 + 1] : ov[c0]);
+      const float o1 = __uint_as_float(hf ? ov[4 + c0 + 1] : ov[4 + c0]);
+      const float o2 = __uint_as_float(hf ? ov[8 + c0 + 1] : ov[8 + c0]);
+      pp[2 + d] = (o0 + o1) + o2;
+      if (j == 0) {
+        pp[0] = s_m[h];
+        pp[1] = s_l[h];
       }
-    if (grp == 0) {
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kKvTmemCols);
+  }
+}
+
+// Merges the chunks' partial results of one (sequence, query head): m = max
+// over the chunks that hold tokens, factors f_c = exp(m_c - m), den =
+// sum_c f_c l_c, Y[d] = fp16_rn(sum_c f_c O_c[d] / den). One CTA per
+// (sequence, head), thread d = element d; the factors of up to kMergeBlock
+// chunks at a time are computed in parallel into shared memory, and every
+// thread keeps 16 chunks' values in flight. Every sum runs in a fixed order
+// (bit-reproducible).
+constexpr int kMergeBlock = 1024;
+__global__ void __launch_bounds__(kKvD) kv4_merge_kernel(KvAttnArgs a) {
+  __shared__ float s_f[kMergeBlock];
+  __shared__ float s_red[kKvD / 32];
+  grid_dependency_wait();  // the partial results come from the preceding kernel
+  grid_launch_dependents();
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const float* pp = a.part + (static_cast<int64_t>(b) * a.Hq + h) * a.nsplit * kKvPartStride;
+  // m over the chunks with tokens
+  float m = -INFINITY;
+  for (int c = t; c < a.nsplit; c += kKvD)
+    if (pp[c * kKvPartStride + 1] > 0.0f) m = fmaxf(m, pp[c * kKvPartStride]);
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) s_red[warp] = m;
+  __syncthreads();
+  m = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+  __syncthreads();
+  float den_part = 0.0f, num = 0.0f;
+  constexpr int kBatch = 16;
+  for (int c0 = 0; c0 < a.nsplit; c0 += kMergeBlock) {
+    const int cn = min(kMergeBlock, a.nsplit - c0);
+    for (int c = t; c < cn; c += kKvD) {
+      const float lc = pp[(c0 + c) * kKvPartStride + 1];
+      const float f = lc > 0.0f ? expf(pp[(c0 + c) * kKvPartStride] - m) : 0.0f;
+      s_f[c] = f;
+      den_part = fmaf(f, lc, den_part);
+    }
+    __syncthreads();
+    for (int c1 = 0; c1 < cn; c1 += kBatch) {
+      float v[kBatch];
 #pragma unroll
-      for (int h = 0; h < GC; ++h)
+      for (int q = 0; q < kBatch; ++q) v[q] = c1 + q < cn ? pp[(c0 + c1 + q) * kKvPartStride + 2 + t] : 0.0f;
 #pragma unroll
-        for (int e = 0; e < 16; ++e) s_o[warp][h][16 * li + e] = o[h][e];
+      for (int q = 0; q < kBatch; ++q)
+        if (c1 + q < cn) num = fmaf(s_f[c1 + q], v[q], num);
     }
+    __syncthreads();
   }
+  for (int o = 16; o > 0; o >>= 1) den_part += __shfl_xor_sync(0xffffffffu, den_part, o);
+  if (lane == 0) s_red[warp] = den_part;
   __syncthreads();
-  // ---- this chunk's partial result
-  const int64_t pstride = 2 + kKvD;
-  for (int i = threadIdx.x; i < GC * kKvD; i += kKvThreads) {
-    const int h = i / kKvD, d = i % kKvD;
-    float sum = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kKvWarps; ++w) sum += s_o[w][h][d];
-    float* pp = a.part + ((static_cast<int64_t>(b) * a.Hq + h0 + h) * a.nsplit + split) * pstride;
-    pp[2 + d] = sum;
-    if (d == 0) {
-      pp[0] = s_m[h];
-      pp[1] = n > 0 ? s_l[h] : 0.0f;
-    }
-  }
-  // ---- the last chunk of this (sequence, head group) to finish merges them
-  __threadfence();
-  __syncthreads();
-  int32_t* ticket = a.tickets + static_cast<int64_t>(b) * a.Hkv * groups + hg;
-  if (threadIdx.x == 0) s_last = atomicAdd(ticket, 1) == a.nsplit - 1;
-  __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // Merge, in a fixed order (bit-reproducible): warp h finds head h's maximum
-  // over the chunks that hold tokens and the denominator sum_c exp(m_c - m) l_c,
-  // keeping the chunk factors exp(m_c - m) in shared memory (the spent V codes'
-  // space); then every (head, element) thread sums its weighted values over the
-  // chunks with independent loads.
-  constexpr int kMergeSmem = kKcBytes / (4 * GC);  // chunk factors kept per head
-  float* s_f = reinterpret_cast<float*>(s_vc);
-  if (warp < GC) {
-    const float* pp = a.part + (static_cast<int64_t>(b) * a.Hq + h0 + warp) * a.nsplit * pstride;
-    float m = -INFINITY;
-    for (int c = lane; c < a.nsplit; c += 32)
-      if (__ldcg(pp + c * pstride + 1) > 0.0f) m = fmaxf(m, __ldcg(pp + c * pstride));
-    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float den = 0.0f;
-    for (int c = lane; c < a.nsplit; c += 32) {
-      const float lc = __ldcg(pp + c * pstride + 1);
-      const float f = lc > 0.0f ? expf(__ldcg(pp + c * pstride) - m) : 0.0f;
-      if (c < kMergeSmem) s_f[warp * kMergeSmem + c] = f;
-      den = fmaf(f, lc, den);
-    }
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
-    if (lane == 0) {
-      s_m[warp] = m;
-      s_l[warp] = den;
-    }
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < GC * kKvD; i += kKvThreads) {
-    const int h = i / kKvD, d = i % kKvD;
-    const float* pp = a.part + (static_cast<int64_t>(b) * a.Hq + h0 + h) * a.nsplit * pstride;
-    const float m = s_m[h], den = s_l[h];
-    float num = 0.0f;
-#pragma unroll 8
-    for (int c = 0; c < a.nsplit; ++c) {
-      float f;
-      if (c < kMergeSmem) {
-        f = s_f[h * kMergeSmem + c];
-      } else {
-        const float lc = __ldcg(pp + c * pstride + 1);
-        f = lc > 0.0f ? expf(__ldcg(pp + c * pstride) - m) : 0.0f;
-      }
-      num = fmaf(f, __ldcg(pp + c * pstride + 2 + d), num);
-    }
-    a.out[(static_cast<int64_t>(b) * a.Hq + h0 + h) * kKvD + d] = __float2half_rn(den > 0.0f ? num / den : 0.0f);
-  }
-  if (threadIdx.x == 0) *ticket = 0;  // ready for the next launch
+  const float den = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
+  a.out[(static_cast<int64_t>(b) * a.Hq + h) * kKvD + t] = __float2half_rn(den > 0.0f ? num / den : 0.0f);
 }
 
 }  // namespace w4a8

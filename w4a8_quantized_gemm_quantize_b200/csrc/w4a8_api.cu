@@ -562,10 +562,6 @@ w4a8_status_t check_kv_shape(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lmax, i
   return W4A8_OK;
 }
 
-int64_t kv_ticket_bytes(int64_t B, int64_t Hq, int64_t Hkv) {
-  const int64_t G = Hq / Hkv;
-  return round256(B * Hkv * (G / kv_heads_per_cta(G)) * 4);
-}
 
 w4a8_status_t kv_quantize_launch(const void* X, int64_t n, const int32_t* pos, int64_t H, int64_t Lmax,
                                  uint8_t* codes, uint32_t* params, cudaStream_t stream) {
@@ -983,9 +979,35 @@ w4a8_status_t w4kv_append(const void* K_new, const void* V_new, const int32_t* p
   return kv_quantize_launch(V_new, B * Hkv, positions, Hkv, Lmax, v_codes, v_params, st);
 }
 
+}  // extern "C"
+
+// The attention kernel (partial results per chunk), then the merge. The
+// attention kernel's dynamic shared memory is above the 48 KB default: raised
+// once per (device, instantiation).
+template <int GC>
+w4a8_status_t kv_decode_launch(dim3 grid, dim3 merge_grid, cudaStream_t s, const KvAttnArgs& a) {
+  static bool done[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return launch_status();
+  if (!done[dev]) {
+    // four CTAs per SM: the whole unified L1 / shared array as shared memory
+    if (cudaFuncSetAttribute(kv4_decode_kernel<GC>, cudaFuncAttributeMaxDynamicSharedMemorySize, KvSmem::kBytes) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(kv4_decode_kernel<GC>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared) != cudaSuccess)
+      return launch_status();
+    done[dev] = true;
+  }
+  const w4a8_status_t st = launch_pdl(kv4_decode_kernel<GC>, grid, dim3(kKvAttnThreads), KvSmem::kBytes, s, 1, a);
+  if (st != W4A8_OK) return st;
+  return launch_pdl(kv4_merge_kernel, merge_grid, dim3(kKvD), 0, s, 1, a);
+}
+
+extern "C" {
+
 size_t w4kv_attention_workspace_bytes(int64_t B, int64_t Hq, int64_t Hkv, int64_t Lmax, int32_t D) {
   if (check_kv_shape(B, Hq, Hkv, Lmax, D) != W4A8_OK) return 0;
-  return static_cast<size_t>(kv_ticket_bytes(B, Hq, Hkv) + B * Hq * kv_splits(Lmax) * (2 + kKvD) * 4);
+  return static_cast<size_t>(round256(B * Hq * kv_splits(Lmax) * kKvPartStride * 4));
 }
 
 w4a8_status_t w4kv_attention_decode(const void* q, const uint8_t* k_codes, const uint32_t* k_params,
@@ -1016,20 +1038,23 @@ w4a8_status_t w4kv_attention_decode(const void* q, const uint8_t* k_codes, const
   a.vp = v_params;
   a.seq_lens = seq_lens;
   a.out = static_cast<__half*>(out);
-  a.tickets = static_cast<int32_t*>(workspace);
-  a.part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + kv_ticket_bytes(B, Hq, Hkv));
+  a.part = static_cast<float*>(workspace);
+  a.B = static_cast<int>(B);
+  a.groups = static_cast<int>(G / gc);
   a.Hq = static_cast<int>(Hq);
   a.Hkv = static_cast<int>(Hkv);
   a.nsplit = static_cast<int>(kv_splits(Lmax));
   a.Lmax = Lmax;
   a.scale = scale;
   a.err = dev->err;
+  // one CTA per (chunk, head group, sequence)
   const dim3 grid(static_cast<unsigned>(a.nsplit), static_cast<unsigned>(Hkv * (G / gc)), static_cast<unsigned>(B));
+  const dim3 merge_grid(static_cast<unsigned>(Hq), static_cast<unsigned>(B));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   switch (gc) {
-    case 4: return launch_pdl(kv4_decode_kernel<4>, grid, dim3(kKvThreads), 0, s, 1, a);
-    case 2: return launch_pdl(kv4_decode_kernel<2>, grid, dim3(kKvThreads), 0, s, 1, a);
-    default: return launch_pdl(kv4_decode_kernel<1>, grid, dim3(kKvThreads), 0, s, 1, a);
+    case 4: return kv_decode_launch<4>(grid, merge_grid, s, a);
+    case 2: return kv_decode_launch<2>(grid, merge_grid, s, a);
+    default: return kv_decode_launch<1>(grid, merge_grid, s, a);
   }
 }
 
