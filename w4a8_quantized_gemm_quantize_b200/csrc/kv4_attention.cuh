@@ -310,35 +310,24 @@ __global__ void __launch_bounds__(kKvAttnThreads, 4) kv4_decode_kernel(KvAttnArg
     mbar_wait_limit(bar_ld, 0, nullptr, err, kErrKvWait, kWaitLimitNs);
   }
 
-  // ---- unpack: thread (token j, half hf)
+  // ---- unpack: thread (token j, half hf); the K values first, so that the
+  // scores' MMAs run while the V values are unpacked
+  const uint32_t zz = s_z[j];
+  const __half kz = __ushort_as_half(static_cast<unsigned short>(zz & 0xFFFFu));
+  const __nv_bfloat16 vzb = __float2bfloat16_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(zz >> 16))));
+  // the 32 code bytes of this half, read in an order that spreads the banks
+  // (rows are 64 bytes: lanes two tokens apart share banks)
+  const int rot = (j >> 1) & 1;
+  const int base = j * kKvRowBytes + hf * 32;
   {
-    const uint32_t zz = s_z[j];
-    const __half kz = __ushort_as_half(static_cast<unsigned short>(zz & 0xFFFFu));
     const __half kb1 = __hadd(__float2half_rn(1024.0f), kz);
     const __half kb16 = __hadd(__float2half_rn(64.0f), kz);
     const __half2 kbias = __halves2half2(__hneg(kb1), __hneg(kb1));
     const __half2 kbias16 = __halves2half2(__hneg(kb16), __hneg(kb16));
-    const __nv_bfloat16 vzb = __float2bfloat16_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(zz >> 16))));
-    const __nv_bfloat16 vb1 = __hadd(__float2bfloat16_rn(128.0f), vzb);
-    const __nv_bfloat162 vbias = __halves2bfloat162(vb1, vb1);
-    // the 32 code bytes of this half, read in an order that spreads the
-    // banks (rows are 64 bytes: lanes two tokens apart share banks)
-    const int rot = (j >> 1) & 1;
-    const int base = j * kKvRowBytes + hf * 32;
     const uint4 ka = *reinterpret_cast<const uint4*>(s_kc + base + rot * 16);
     const uint4 kb = *reinterpret_cast<const uint4*>(s_kc + base + (rot ^ 1) * 16);
-    const uint4 vx = *reinterpret_cast<const uint4*>(s_vc + base + rot * 16);
-    const uint4 vy = *reinterpret_cast<const uint4*>(s_vc + base + (rot ^ 1) * 16);
-    const uint4 k0 = rot ? kb : ka, k1 = rot ? ka : kb, v0 = rot ? vy : vx, v1 = rot ? vx : vy;
+    const uint4 k0 = rot ? kb : ka, k1 = rot ? ka : kb;
     const uint32_t kws[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
-    const uint32_t vws[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-    uint8_t* row = s_vpl + hf * KvSmem::kPlane + j * 128;
-#pragma unroll
-    for (int wi = 0; wi < 8; ++wi) {
-      uint32_t o[4];
-      kv_unpack8_bf16(vws[wi], vbias, o);
-      *reinterpret_cast<uint4*>(row + ((wi ^ (j & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-    }
     uint32_t kr[32];
 #pragma unroll
     for (int wi = 0; wi < 8; ++wi) {
@@ -350,7 +339,7 @@ __global__ void __launch_bounds__(kKvAttnThreads, 4) kv4_decode_kernel(KvAttnArg
     tmem_st_32(tmem + kKvTmemK + 32 * hf + lane_base, kr);
   }
   tmem_wait_st();
-  fence_proxy_async_smem();  // the generic-proxy operand stores, before the MMAs read them
+  fence_proxy_async_smem();  // q's operand, before the MMAs read it
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -364,6 +353,22 @@ __global__ void __launch_bounds__(kKvAttnThreads, 4) kv4_decode_kernel(KvAttnArg
     }
     mma_commit(bar_mma);
   }
+  {
+    const __nv_bfloat16 vb1 = __hadd(__float2bfloat16_rn(128.0f), vzb);
+    const __nv_bfloat162 vbias = __halves2bfloat162(vb1, vb1);
+    const uint4 vx = *reinterpret_cast<const uint4*>(s_vc + base + rot * 16);
+    const uint4 vy = *reinterpret_cast<const uint4*>(s_vc + base + (rot ^ 1) * 16);
+    const uint4 v0 = rot ? vy : vx, v1 = rot ? vx : vy;
+    const uint32_t vws[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    uint8_t* row = s_vpl + hf * KvSmem::kPlane + j * 128;
+#pragma unroll
+    for (int wi = 0; wi < 8; ++wi) {
+      uint32_t o[4];
+      kv_unpack8_bf16(vws[wi], vbias, o);
+      *reinterpret_cast<uint4*>(row + ((wi ^ (j & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+  }
+  fence_proxy_async_smem();  // the V planes, before the second MMAs read them (after the next barrier)
   if (!mbar_wait_limit(bar_mma, 0, nullptr, err, kErrKvWait, kWaitLimitNs))
     mbar_wait_limit(bar_mma, 0, nullptr, err, kErrKvWait, kWaitLimitNs);
   tc_fence_after();
