@@ -62,6 +62,7 @@ struct GemmArgs {
   int m_tiles, num_tiles;
   int sk_tiles;          // the first sk_tiles tiles are split stream-K over all CTAs
   int split;             // > 1: cluster split-K, `split` CTAs (one cluster) per tile
+  int band;              // whole tiles walk bands of `band` token tiles, channels fastest (0: no bands)
   int a4;                // activation codes are 4-bit, two per byte (W4A4), unpacked in shared memory
   const __half* lut_table;  // lookup-table weights: the 16 fp16 table entries (inside the blob)
 };
@@ -82,13 +83,21 @@ struct Seg {
 // direct one. With cluster split-K instead, tile t is split into `split`
 // k-ranges taken by the CTAs of cluster t (CTA rank r takes k-blocks
 // [KB r / split, KB (r + 1) / split)) and reduced on chip.
+// Whole tiles with band > 0 (and no stream-K tiles) are visited in bands of
+// `band` token tiles: within a band the token tile changes fastest, then the
+// channel tile, so that the CTAs running at one time share a band's
+// activation rows (band x 128 rows x K bytes) in L2 instead of sweeping all
+// of them once per channel column (tile index = channel tile x m_tiles +
+// token tile throughout).
 struct Sched {
   int64_t u, u_end;
-  int tile_it, KB, num_tiles, split;
+  int tile_it, KB, num_tiles, split, band, m_tiles;
   __device__ __forceinline__ void init(const GemmArgs& a) {
     KB = a.KB;
     num_tiles = a.num_tiles;
     split = a.split;
+    band = a.sk_tiles == 0 ? a.band : 0;
+    m_tiles = a.m_tiles;
     u = u_end = 0;
     if (split > 1) {
       tile_it = static_cast<int>(blockIdx.x) / split;
@@ -121,6 +130,14 @@ struct Sched {
     }
     if (tile_it >= num_tiles) return false;
     s.tile = tile_it;
+    if (band > 0 && band < m_tiles) {
+      const int n_tiles = num_tiles / m_tiles;
+      const int per_band = band * n_tiles;
+      const int b = tile_it / per_band;               // bands before the last are full
+      const int bm = min(band, m_tiles - b * band);  // token tiles of this band
+      const int r = tile_it - b * per_band;
+      s.tile = (r / bm) * m_tiles + b * band + r % bm;
+    }
     s.kb0 = 0;
     s.kb1 = KB;
     tile_it += gridDim.x;

@@ -461,6 +461,9 @@ w4a8_status_t gemm_impl(const void* A8, const void* sA, const int32_t* rowsum, c
   a.num_tiles = num_tiles;
   a.sk_tiles = sk_tiles;
   a.split = split;
+  // bands of 16 token tiles (16 x 128 tokens of activation rows shared in L2
+  // by the CTAs of a wave) when the activation codes exceed ~a quarter of L2
+  a.band = static_cast<int64_t>(M) * K > (int64_t(32) << 20) ? 16 : 0;
   a.a4 = a4;
   if (lut) {
     a.sA = nullptr;
