@@ -291,6 +291,18 @@ def test_gemm_cluster_split_sizes(K):
     check_gemm(A, q, z, s2, s1, [(0, 0, 0)] + CLUSTER)
 
 
+@pytest.mark.parametrize("M,N", [(2500, 384), (3000, 128), (2432, 256)])
+def test_gemm_banded_tile_order_ragged_bands(M, N):
+    """Activation codes above 32 MiB (K = 14336) switch whole tiles to bands
+    of 16 token tiles; 20, 24 and 19 token tiles leave a last band of 4, 8
+    and 3. Whole tiles (the automatic choice at 128-token tiles) and a
+    reduced grid, so that every CTA walks several bands."""
+    K = 14336
+    q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-band-w", M, N))
+    A = I.activations(M, K, I.seed_of("t-band-a", M, N))
+    check_gemm(A, q, z, s2, s1, [(0, 0, 0), (1, 128, 7)])
+
+
 def test_gemm_cluster_split_needs_two_k_blocks():
     N, K, M = 256, 128, 4
     q, z, s2, s1 = I.uniform_codes(N, K, 12)
