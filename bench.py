@@ -420,9 +420,10 @@ def run_gpu(args, world, rank, local):
                                         for i, (M, name, N, K) in enumerate(cases)]) for b in range(3)]
         chain_ws = torch.zeros(w4a8.chain_workspace_bytes(chain_arrs[0]), dtype=torch.uint8, device=dev)
 
-    def step(events=None, gemm_only=False, buf=0):
+    def step(events=None, gemm_only=False, buf=0, quant_only=False):
         """One pass over the cases; `buf` selects the activation and output
-        buffers (the end-to-end run alternates between two)."""
+        buffers (the end-to-end run alternates between two); `quant_only`
+        runs the activation quantizers alone (their roofline)."""
         if chain:
             w4a8.chain(chain_arrs[buf], chain_ws)
             return
@@ -437,6 +438,8 @@ def run_gpu(args, world, rank, local):
                     quantize(A, static_scales[(M, name)], out=(A8, sA, rs))
                 else:
                     quantize(A, out=(A8, sA, rs))
+            if quant_only:
+                continue
             if events is not None:
                 events[i][0].record()
             gemm(A8, sA, rs, blobs[(name, copy_of[M])], N, K, out=Y, workspace=ws)
@@ -459,14 +462,15 @@ def run_gpu(args, world, rank, local):
 
     # ---- timed region 1: K steps (unrolled) in one CUDA graph, no events
     # inside, so consecutive kernels overlap through programmatic launch
-    def capture(events_per_step, gemm_only=False):
+    def capture(events_per_step, gemm_only=False, quant_only=False):
         g = torch.cuda.CUDAGraph()
         cap_stream = torch.cuda.Stream(dev)
         cap_stream.wait_stream(torch.cuda.current_stream(dev))
         with torch.cuda.stream(cap_stream):
             with torch.cuda.graph(g, stream=cap_stream):
                 for s in range(args.steps):
-                    step(events=None if events_per_step is None else events_per_step[s], gemm_only=gemm_only)
+                    step(events=None if events_per_step is None else events_per_step[s], gemm_only=gemm_only,
+                         quant_only=quant_only)
         torch.cuda.current_stream(dev).wait_stream(cap_stream)
         return g
 
@@ -484,12 +488,15 @@ def run_gpu(args, world, rank, local):
     ev = [[[torch.cuda.Event(enable_timing=True, external=True) for _ in range(2)] for _ in cases]
           for _ in range(K_steps)]
     g_ev = capture(None if chain else ev)
-    for g in (g_plain, g_gemm, g_ev):  # untimed replays: settle clocks and caches
-        g.replay()
+    # ---- timed region 4: the activation quantizers of the same K steps alone
+    g_quant = None if (chain or lut) else capture(None, quant_only=True)
+    for g in (g_plain, g_gemm, g_ev, g_quant):  # untimed replays: settle clocks and caches
+        if g is not None:
+            g.replay()
     torch.cuda.synchronize()
 
     stream = torch.cuda.current_stream(dev)
-    t0, t1, t2, t3 = (torch.cuda.Event(enable_timing=True) for _ in range(4))
+    t0, t1, t2, t3, t4, t5 = (torch.cuda.Event(enable_timing=True) for _ in range(6))
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
@@ -504,10 +511,17 @@ def run_gpu(args, world, rank, local):
         torch.cuda.synchronize()
         g_ev.replay()
         torch.cuda.synchronize()
+        if g_quant is not None:
+            barrier(world)
+            t4.record(stream)
+            g_quant.replay()
+            t5.record(stream)
+            torch.cuda.synchronize()
     barrier(world)
     elapsed_ms = t0.elapsed_time(t1)
     max_ms = max_over_ranks(elapsed_ms, world)
     gemm_ms = max_over_ranks(t2.elapsed_time(t3), world)
+    quant_ms = max_over_ranks(t4.elapsed_time(t5), world) if g_quant is not None else None
     assert w4a8.get_device_error(dev) == 0
 
     per_case_ms = np.zeros(len(cases))
@@ -516,7 +530,7 @@ def run_gpu(args, world, rank, local):
             for i in range(len(cases)):
                 per_case_ms[i] += ev[s][i][0].elapsed_time(ev[s][i][1])
         per_case_ms /= K_steps
-    del g_plain, g_gemm, g_ev
+    del g_plain, g_gemm, g_ev, g_quant
 
     # ---- end to end through the public API: each step copies its fp16
     # activations in from pinned host memory (one copy) and its outputs back
@@ -583,7 +597,8 @@ def run_gpu(args, world, rank, local):
         assert torch.equal(y_back, y_dev)
     assert w4a8.get_device_error(dev) == 0
 
-    return dict(elapsed_ms=elapsed_ms, max_ms=max_ms, gemm_ms=gemm_ms, per_case_ms=per_case_ms, clocks=clk.summary(),
+    return dict(elapsed_ms=elapsed_ms, max_ms=max_ms, gemm_ms=gemm_ms, quant_ms=quant_ms, per_case_ms=per_case_ms,
+                clocks=clk.summary(),
                 e2e_ms=e2e_ms, cases=cases, n_copies=n_copies, h2d_bytes=h2d_bytes, d2h_bytes=d2h_bytes,
                 gpu_name=torch.cuda.get_device_name(dev))
 
@@ -1037,6 +1052,20 @@ def main():
     roofline["launches"] = len(cases) * args.steps
     roofline["avg_launch_us"] = round(gemm_ms * 1e3 / len(cases), 3)
 
+    # the activation quantizers' launches timed alone: fp16 activations in,
+    # codes (8- or 4-bit), per-token scale (2 B) and rowsum (4 B) out
+    quantizer = None
+    if r.get("quant_ms") is not None:
+        qbytes = sum(M * K * 2 + M * K * ACT_BITS[args.act] // 8 + 6 * M for (M, _, N, K) in cases)
+        q_ms = r["quant_ms"] / args.steps
+        q_ach = qbytes / (q_ms * 1e-3) / 1e9
+        quantizer = {"kernel": ("quantize_act_static_kernel" if args.act.startswith("static") else "quantize_act_kernel")
+                               + ("" if ACT_BITS[args.act] == 8 else " (4-bit codes)"),
+                     "bound": "hbm", "achieved": round(q_ach, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(q_ach / hbm, 4), "bytes_per_step": qbytes,
+                     "avg_launch_us": round(q_ms * 1e3 / len(cases), 3),
+                     "note": "latency-bound at these sizes (at most 32 x 14336 activations per launch)"}
+
     per_case = []
     for (M, name, N, K), t, b, o, rt in zip(cases, per, abytes, ops, roof_t):
         per_case.append({"M": M, "layer": name, "N": N, "K": K, "us_with_events": round(t * 1e3, 2),
@@ -1065,6 +1094,7 @@ def main():
         "gpu_launches": (1 + (0 if lut else 1) + (1 if ACT_BITS[args.act] == 4 and not lut else 0))
                         * len(cases) * args.steps,
         "roofline": roofline,
+        "quantizer": quantizer,
         "e2e": {"value": round(world * wbytes / (r["e2e_ms"] / args.steps * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": r["h2d_bytes"], "d2h_bytes_per_step": r["d2h_bytes"]},
         "clocks": r["clocks"],
