@@ -271,7 +271,8 @@ def test_gemm_tiny_config_all_schedules(M):
 
 
 @pytest.mark.parametrize("M,N,K", [(3, 384, 1024), (17, 512, 640), (65, 256, 2048), (129, 384, 512),
-                                   (200, 128, 384), (1, 1024, 4096), (300, 640, 256)])
+                                   (200, 128, 384), (1, 1024, 4096), (300, 640, 256), (100, 384, 1024),
+                                   (128, 4096, 512)])
 def test_gemm_ragged_shapes(M, N, K):
     q, z, s2, s1 = I.uniform_codes(N, K, I.seed_of("t-g", N, K))
     A = I.activations(M, K, I.seed_of("t-a", M, K))
